@@ -1,0 +1,139 @@
+// Shared device helpers and the device-side state layout of libtl.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/tl.h"
+
+namespace tl {
+
+// Status-word bits written by kernels (never __trap/assert: a bad index is
+// recorded and the access skipped).
+enum : int32_t {
+  ST_BAD_PAGE = 1 << 0,     // page id outside the pool
+  ST_BAD_POS = 1 << 1,      // position >= max_seq
+  ST_BAD_SLOT = 1 << 2,     // KV slot outside the table
+  ST_BAD_TOKEN = 1 << 3,    // token id outside [0, vocab)
+  ST_EKV = 1 << 4,          // lane asked for more iterations than its cache holds
+  ST_BAD_ROW = 1 << 5,      // row table larger than its buffers
+};
+
+enum LanePhase : int32_t { PH_IDLE = 0, PH_LOOP = 1, PH_BOUNDARY = 2, PH_DONE = 3 };
+
+// One lane's scheduling state, resident in device memory.
+struct LaneState {
+  int32_t L_req;      // requested loop count
+  int32_t L_cap;      // monotonic clamp: iterations the cache holds for new positions
+  int32_t L_run;      // iterations planned for the current token: min(L_req, L_cap)
+  int32_t iter;       // iterations done for the current token
+  int32_t pos;        // position of the row the lane is computing
+  int32_t streak;     // early-exit streak
+  int32_t phase;      // LanePhase
+  int32_t depth;      // iterations behind the lane's current hidden state
+  int32_t n_emitted;  // tokens emitted by the running decode
+  int32_t n_target;   // tokens to emit
+  int32_t token;      // last token fed (or emitted)
+  int32_t entered;    // set when the lane just took a token and still needs its pre blocks
+};
+
+// Early-exit parameters, copied by value into kernels.
+struct EEParams {
+  double tau;
+  int32_t min_L;
+  int32_t patience;
+  int32_t peek_every;
+  int32_t enabled;
+};
+
+// Compacted rows of one launch group: row r computes for lane row_lane[r] at
+// position row_pos[r], loop iteration row_iter[r] (0-based).
+struct Rows {
+  int32_t* n;        // device scalar: number of valid rows
+  int32_t* lane;
+  int32_t* pos;
+  int32_t* iter;
+};
+
+// KV cache geometry.  A page holds kv_page_tokens positions of one (lane,
+// slot): K as [H][P][hd] fp16 then V as [H][P][hd] fp16.
+struct KVGeom {
+  __half* pool;
+  const int32_t* page_table;   // [max_lanes][n_slots][pages_per_seq]
+  int32_t n_slots;
+  int32_t pages_per_seq;
+  int32_t page_tokens;
+  int32_t page_shift;          // log2(page_tokens)
+  int32_t n_pages;
+  int32_t H, hd;
+  int64_t page_elems;          // 2 * H * P * hd
+};
+
+__device__ __forceinline__ void set_status(int32_t* st, int32_t bit) { atomicOr(st, bit); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum for blockDim.x a multiple of 32 (<= 1024).  `red` holds >= 32 floats.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float t = (threadIdx.x < nw) ? red[threadIdx.x] : 0.f;
+  if (w == 0) t = warp_sum(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  return red[0];
+}
+__device__ __forceinline__ double block_sum_d(double v, double* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum_d(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  double t = (threadIdx.x < nw) ? red[threadIdx.x] : 0.0;
+  if (w == 0) t = warp_sum_d(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  return red[0];
+}
+
+// (u - 8) as an exact float for a nibble u in [0,15]: 2^23 + u read as float, minus 2^23 + 8.
+__device__ __forceinline__ float nib_to_f(uint32_t w, int sh) {
+  return __uint_as_float(((w >> sh) & 0xFu) | 0x4B000000u) - 8388616.0f;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+
+// Address of (slot, lane, pos) K row for head h; V follows at + H*P*hd.
+__device__ __forceinline__ __half* kv_k_ptr(const KVGeom& g, int lane, int slot, int pos, int h,
+                                            int32_t* status) {
+  if (slot < 0 || slot >= g.n_slots) { set_status(status, ST_BAD_SLOT); return nullptr; }
+  const int pg = pos >> g.page_shift;
+  if (pos < 0 || pg >= g.pages_per_seq) { set_status(status, ST_BAD_POS); return nullptr; }
+  const int page = g.page_table[((int64_t)lane * g.n_slots + slot) * g.pages_per_seq + pg];
+  if (page < 0 || page >= g.n_pages) { set_status(status, ST_BAD_PAGE); return nullptr; }
+  const int off = pos & (g.page_tokens - 1);
+  return g.pool + (int64_t)page * g.page_elems + ((int64_t)h * g.page_tokens + off) * g.hd;
+}
+
+}  // namespace tl

@@ -1,0 +1,775 @@
+// Decode-path kernels: lane compaction, RMSNorm, projections (W4A16 / BF16),
+// RoPE + KV append, paged per-iteration attention, early-exit rule, head
+// argmax and the boundary-stage transitions.
+//
+// Model block and head: see include/tl.h.  Every kernel that depends on a row
+// count reads it from device memory (Rows::n) so a step can be replayed with
+// no host involvement; grids are sized for the largest row count.
+#pragma once
+
+#include "common.cuh"
+
+namespace tl {
+
+// ------------------------------------------------------------- weights ----
+
+struct MatView {
+  int32_t fmt;          // TL_FMT_INT4 / TL_FMT_BF16
+  int32_t N, K, group;
+  const uint8_t* q;     // INT4 packed [N][K/2]
+  const __half* s;      // INT4 scales [N][K/group]
+  const uint16_t* bf;   // BF16 [N][K]
+};
+
+enum Epi : int32_t { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_ARGMAX = 3 };
+
+// Output side of a projection.  Row r of the activations is output row r; for
+// EPI_RESID it is added into h[map ? map[r] : r][:]; for EPI_ARGMAX each CTA
+// writes its best (value, index) per row into part_*[r * n_parts + blockIdx.x]
+// and, when logits != null, the logits into logits[lmap[r] * ldo + n].
+struct ProjOut {
+  int32_t epi;
+  float* out;            // EPI_STORE / EPI_SWIGLU: [rows][ldo]
+  int32_t ldo;
+  float* h;              // EPI_RESID: residual rows, leading dimension N
+  const int32_t* map;    // EPI_RESID row -> h row (null = identity)
+  float* logits;         // EPI_ARGMAX (nullable)
+  const int32_t* lmap;   // EPI_ARGMAX row -> logits row
+  float* part_val;
+  int32_t* part_idx;
+  int32_t n_parts;
+};
+
+// Orders (value, index) pairs: larger value first, lower index on ties.
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+// ---------------------------------------------------------- row tables ----
+
+enum RowSel : int32_t { SEL_LOOP = 0, SEL_BOUNDARY = 1, SEL_ENTERED = 2, SEL_MASK = 3 };
+
+// One CTA of 1024 threads; thread i looks at lane i.  Selects lanes, writes the
+// compacted row table (lane order), and for SEL_LOOP copies h -> h_in (the loop
+// input that the relative-L2 test compares against).  SEL_LOOP also applies an
+// optional per-lane L request: a request above the lane's cap sets ST_EKV and
+// keeps the lane out; a request at or below the iterations already done
+// finishes the lane's loop without running.
+__global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, int32_t sel,
+                                  const uint8_t* __restrict__ mask, const int32_t* __restrict__ per_lane_L,
+                                  Rows rows, uint8_t* __restrict__ exit_mask_out, int32_t* __restrict__ alive,
+                                  int32_t* __restrict__ status) {
+  __shared__ int32_t warp_cnt[32];
+  __shared__ int32_t alive_cnt;
+  const int i = threadIdx.x;
+  if (i == 0) alive_cnt = 0;
+  __syncthreads();
+  int take = 0;
+  if (i < n_lanes) {
+    LaneState& st = lanes[i];
+    const bool on = (mask == nullptr) || mask[i] != 0;
+    if (st.phase == PH_LOOP || st.phase == PH_BOUNDARY) atomicAdd(&alive_cnt, 1);
+    if (sel == SEL_LOOP) {
+      if (exit_mask_out && on) exit_mask_out[i] = 0;
+      if (on && st.phase == PH_LOOP) {
+        take = 1;
+        if (per_lane_L) {
+          const int L = per_lane_L[i];
+          if (L < 1 || L > st.L_cap) {
+            set_status(status, ST_EKV);
+            take = 0;
+          } else {
+            st.L_req = L;
+            st.L_run = L;
+            if (st.iter >= L) {  // already ran what is now requested: loop finished
+              st.phase = PH_BOUNDARY;
+              st.depth = st.iter;
+              if (exit_mask_out) exit_mask_out[i] = 1;
+              take = 0;
+            }
+          }
+        }
+      }
+    } else if (sel == SEL_BOUNDARY) {
+      take = on && st.phase == PH_BOUNDARY;
+    } else if (sel == SEL_ENTERED) {
+      take = st.entered;
+      st.entered = 0;
+    } else {
+      take = on;
+    }
+  }
+  // block-wide exclusive scan of `take`
+  const int lane = i & 31, w = i >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, take);
+  if (lane == 0) warp_cnt[w] = __popc(bal);
+  __syncthreads();
+  if (w == 0) {
+    int v = warp_cnt[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    warp_cnt[lane] = v;  // inclusive
+  }
+  __syncthreads();
+  const int base = (w == 0) ? 0 : warp_cnt[w - 1];
+  const int r = base + __popc(bal & ((1u << lane) - 1u));
+  if (take) {
+    rows.lane[r] = i;
+    rows.pos[r] = lanes[i].pos;
+    rows.iter[r] = lanes[i].iter;
+  }
+  if (i == 0) {
+    rows.n[0] = warp_cnt[31];
+    if (alive) alive[0] = alive_cnt;
+  }
+}
+
+// --------------------------------------------------------------- norms ----
+
+// out[r] = RMSNorm(h[map ? map[r] : r]) * g, fp32.  One CTA per row.  When
+// h_in is given, also copies the source row there (indexed like h).
+__global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* __restrict__ map,
+                                    const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
+                                    float eps, float* __restrict__ out, float* __restrict__ h_in) {
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  if (r >= n_rows[0]) return;
+  const int src = map ? map[r] : r;
+  const float* x = h + (int64_t)src * d;
+  float ss = 0.f;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) ss += x[k] * x[k];
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    const float v = x[k];
+    out[(int64_t)r * d + k] = v * inv * g[k];
+    if (h_in) h_in[(int64_t)src * d + k] = v;
+  }
+}
+
+// ------------------------------------------------------------ embedding ----
+
+// h[dst] = dequantised embedding row of token; one CTA per row.
+__device__ __forceinline__ void embed_row(const MatView& E, int tok, float* __restrict__ dst, int d) {
+  if (E.fmt == TL_FMT_INT4) {
+    const uint8_t* q = E.q + (int64_t)tok * (d / 2);
+    const __half* s = E.s + (int64_t)tok * (d / E.group);
+    for (int k = 2 * threadIdx.x; k < d; k += 2 * blockDim.x) {
+      const uint32_t b = q[k / 2];
+      const float sc = __half2float(s[k / E.group]);
+      dst[k] = nib_to_f(b, 0) * sc;
+      dst[k + 1] = nib_to_f(b, 4) * sc;
+    }
+  } else {
+    const uint16_t* p = E.bf + (int64_t)tok * d;
+    for (int k = threadIdx.x; k < d; k += blockDim.x) dst[k] = bf16_bits_to_f(p[k]);
+  }
+}
+
+__global__ void embed_rows_kernel(MatView E, const int32_t* __restrict__ tokens, int n, int d,
+                                  float* __restrict__ h, int32_t* __restrict__ status) {
+  const int r = blockIdx.x;
+  if (r >= n) return;
+  int tok = tokens[r];
+  if (tok < 0 || tok >= E.N) { set_status(status, ST_BAD_TOKEN); tok = 0; }
+  embed_row(E, tok, h + (int64_t)r * d, d);
+}
+
+// ---------------------------------------------------------- GEMV (few rows) ----
+//
+// y[r][n] = sum_k x[r][k] * W[n][k] for R activation rows at a time held in
+// shared memory (fp32, 16-byte slots XOR-swizzled so that 32 lanes reading
+// consecutive 128-byte segments do not collide on banks).  One warp per output
+// feature (two for EPI_SWIGLU: gate row n and up row n), 8 warps per CTA; each
+// lane owns 32-element chunks of K: 16 bytes of INT4 (one fp16 scale per chunk,
+// since the group is a multiple of 32) or 64 bytes of BF16.  INT4 values are
+// (u - 8) exactly in fp32; the group scale multiplies each chunk's partial sum.
+
+constexpr int GEMV_WARPS = 8;
+
+__device__ __forceinline__ int swz_slot(int f) { return (f & ~7) | ((f & 7) ^ ((f >> 3) & 7)); }
+
+template <int FMT>
+__device__ __forceinline__ void load_chunk(const MatView& W, int n, int c, float (&w)[32], float& sc) {
+  if constexpr (FMT == TL_FMT_INT4) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(W.q + (int64_t)n * (W.K / 2) + c * 16));
+    sc = __half2float(W.s[(int64_t)n * (W.K / W.group) + (c * 32) / W.group]);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[8 * j + e] = nib_to_f(u[j], 4 * e);
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(W.bf + (int64_t)n * W.K + c * 32);
+    sc = 1.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = __ldg(p + j);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[8 * j + 2 * e] = __uint_as_float(u[e] << 16);
+        w[8 * j + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+    }
+  }
+}
+
+template <int R>
+__device__ __forceinline__ void dot_chunk(const float* __restrict__ xs, int K, int c, const float (&w)[32],
+                                          float sc, float (&acc)[R]) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const float4* row = reinterpret_cast<const float4*>(xs + r * K);
+    float p = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 x = row[swz_slot(8 * c + j)];
+      p = fmaf(w[4 * j], x.x, p);
+      p = fmaf(w[4 * j + 1], x.y, p);
+      p = fmaf(w[4 * j + 2], x.z, p);
+      p = fmaf(w[4 * j + 3], x.w, p);
+    }
+    acc[r] = fmaf(p, sc, acc[r]);
+  }
+}
+
+template <int FMT, int R, int EPI>
+__global__ void __launch_bounds__(GEMV_WARPS * 32)
+gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o) {
+  extern __shared__ float4 smem4[];
+  float* xs = reinterpret_cast<float*>(smem4);
+  __shared__ float best_v[GEMV_WARPS][R];
+  __shared__ int best_i[GEMV_WARPS][R];
+  const int K = W.K, N = W.N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * GEMV_WARPS + warp;
+  const int rows = n_rows[0];
+  const int nch = K / 32;
+  for (int r0 = 0; r0 < rows; r0 += R) {
+    __syncthreads();
+    for (int f = threadIdx.x; f < R * K / 4; f += blockDim.x) {
+      const int r = f / (K / 4), fi = f % (K / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r0 + r < rows) v = reinterpret_cast<const float4*>(X + (int64_t)(r0 + r) * K)[fi];
+      smem4[r * (K / 4) + swz_slot(fi)] = v;
+    }
+    __syncthreads();
+    float acc[R], acc2[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = acc2[r] = 0.f;
+    if (n < N) {
+      for (int c = lane; c < nch; c += 32) {
+        float w[32], sc;
+        load_chunk<FMT>(W, n, c, w, sc);
+        dot_chunk<R>(xs, K, c, w, sc, acc);
+        if constexpr (EPI == EPI_SWIGLU) {
+          load_chunk<FMT>(W2, n, c, w, sc);
+          dot_chunk<R>(xs, K, c, w, sc, acc2);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      acc[r] = warp_sum(acc[r]);
+      if constexpr (EPI == EPI_SWIGLU) acc2[r] = warp_sum(acc2[r]);
+    }
+    if constexpr (EPI == EPI_ARGMAX) {
+      if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          best_v[warp][r] = (n < N) ? acc[r] : -INFINITY;
+          best_i[warp][r] = (n < N) ? n : 0x7fffffff;
+        }
+      }
+      if (n < N && o.logits && lane < R && r0 + lane < rows) {
+        float v = acc[0];
+#pragma unroll
+        for (int r = 1; r < R; ++r) if (lane == r) v = acc[r];
+        o.logits[(int64_t)o.lmap[r0 + lane] * o.ldo + n] = v;
+      }
+      __syncthreads();
+      if (threadIdx.x < R && r0 + threadIdx.x < rows) {
+        const int r = threadIdx.x;
+        float bv = best_v[0][r];
+        int bi = best_i[0][r];
+        for (int ww = 1; ww < GEMV_WARPS; ++ww)
+          if (better(best_v[ww][r], best_i[ww][r], bv, bi)) { bv = best_v[ww][r]; bi = best_i[ww][r]; }
+        o.part_val[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bv;
+        o.part_idx[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bi;
+      }
+    } else if (n < N && lane < R && r0 + lane < rows) {
+      float v = acc[0], v2 = acc2[0];
+#pragma unroll
+      for (int r = 1; r < R; ++r)
+        if (lane == r) { v = acc[r]; v2 = acc2[r]; }
+      const int r = r0 + lane;
+      if constexpr (EPI == EPI_STORE) {
+        o.out[(int64_t)r * o.ldo + n] = v;
+      } else if constexpr (EPI == EPI_SWIGLU) {
+        o.out[(int64_t)r * o.ldo + n] = silu_f(v) * v2;
+      } else {
+        const int hr = o.map ? o.map[r] : r;
+        o.h[(int64_t)hr * N + n] += v;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------- tiled GEMM (many rows) ----
+//
+// C[m][n] = sum_k A[m][k] * W[n][k] on CUDA cores: 64 x 64 tiles, K steps of
+// 32, 256 threads with 4 x 4 outputs each; W tiles are dequantised to fp32 in
+// shared memory (INT4: (u - 8) * scale, exact in fp32).
+
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 32;
+
+template <int FMT>
+__device__ __forceinline__ void load_w_tile(const MatView& W, int n0, int k0, float (*Ws)[SG_BN + 4]) {
+  // 256 threads: feature f = t / 4 (64 features), quarter qk = t % 4 covers 8 k values.
+  const int t = threadIdx.x, f = t >> 2, qk = t & 3;
+  const int n = n0 + f;
+  float w[8];
+  if (n < W.N) {
+    if constexpr (FMT == TL_FMT_INT4) {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(W.q + (int64_t)n * (W.K / 2) + (k0 + 8 * qk) / 2);
+      const float sc = __half2float(W.s[(int64_t)n * (W.K / W.group) + (k0 + 8 * qk) / W.group]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = nib_to_f(u, 4 * e) * sc;
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(W.bf + (int64_t)n * W.K + k0 + 8 * qk);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w[2 * e] = __uint_as_float(u[e] << 16);
+        w[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[e] = 0.f;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) Ws[8 * qk + e][f] = w[e];
+}
+
+template <int FMT, int EPI>
+__global__ void __launch_bounds__(256)
+gemm_simt_kernel(const float* __restrict__ A, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o) {
+  __shared__ float As[SG_BK][SG_BM + 4];
+  __shared__ float Ws[SG_BK][SG_BN + 4];
+  __shared__ float Ws2[(EPI == EPI_SWIGLU) ? SG_BK : 1][SG_BN + 4];
+  const int M = n_rows[0];
+  const int m0 = blockIdx.y * SG_BM, n0 = blockIdx.x * SG_BN;
+  if (m0 >= M) return;
+  const int K = W.K, N = W.N;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {}, acc2[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += SG_BK) {
+    // A tile: 64 rows x 32 k; thread t loads two float4 (row t/4 and t/4+... ) stored transposed.
+    for (int f = threadIdx.x; f < SG_BM * SG_BK / 4; f += 256) {
+      const int r = f / (SG_BK / 4), kq = f % (SG_BK / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m0 + r < M) v = *reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * K + k0 + 4 * kq);
+      As[4 * kq][r] = v.x;
+      As[4 * kq + 1][r] = v.y;
+      As[4 * kq + 2][r] = v.z;
+      As[4 * kq + 3][r] = v.w;
+    }
+    load_w_tile<FMT>(W, n0, k0, Ws);
+    if constexpr (EPI == EPI_SWIGLU) load_w_tile<FMT>(W2, n0, k0, Ws2);
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      if constexpr (EPI == EPI_SWIGLU) {
+        const float4 b2 = *reinterpret_cast<const float4*>(&Ws2[kk][tx * 4]);
+        const float bv2[4] = {b2.x, b2.y, b2.z, b2.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc2[i][j] = fmaf(av[i], bv2[j], acc2[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+  if constexpr (EPI == EPI_ARGMAX) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = m0 + ty * 4 + i;
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = n0 + tx * 4 + j;
+        if (n < N) {
+          if (better(acc[i][j], n, bv, bi)) { bv = acc[i][j]; bi = n; }
+          if (o.logits && m < M) o.logits[(int64_t)o.lmap[m] * o.ldo + n] = acc[i][j];
+        }
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+      }
+      if (tx == 0 && m < M) {
+        o.part_val[(int64_t)m * o.n_parts + blockIdx.x] = bv;
+        o.part_idx[(int64_t)m * o.n_parts + blockIdx.x] = bi;
+      }
+    }
+    return;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = m0 + ty * 4 + i;
+      if (m >= M) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = n0 + tx * 4 + j;
+        if (n >= N) continue;
+        if constexpr (EPI == EPI_STORE) {
+          o.out[(int64_t)m * o.ldo + n] = acc[i][j];
+        } else if constexpr (EPI == EPI_SWIGLU) {
+          o.out[(int64_t)m * o.ldo + n] = silu_f(acc[i][j]) * acc2[i][j];
+        } else {
+          const int hr = o.map ? o.map[m] : m;
+          o.h[(int64_t)hr * N + n] += acc[i][j];
+        }
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------- RoPE + KV ----
+
+// q_out[r] = RoPE(q), and K = RoPE(k), V = v appended (fp16) to the page of
+// (lane, slot, pos).  slot = slot_base + iter * slot_stride.  One CTA per row,
+// d/2 threads: thread t rotates pair (i, i + hd/2) of head t / (hd/2).
+__global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict__ q_out, Rows rows, KVGeom g,
+                               const float2* __restrict__ rope_cs, int slot_base, int slot_stride,
+                               const int32_t* __restrict__ map_lane, int32_t* __restrict__ status) {
+  const int r = blockIdx.x;
+  if (r >= rows.n[0]) return;
+  const int d = g.H * g.hd, half = g.hd / 2;
+  const int t = threadIdx.x;
+  if (t >= d / 2) return;
+  const int h = t / half, i = t % half;
+  const int pos = rows.pos[r];
+  const int lane = map_lane ? map_lane[r] : rows.lane[r];
+  const int slot = slot_base + rows.iter[r] * slot_stride;
+  const float2 cs = rope_cs[(int64_t)pos * half + i];
+  const float* src = qkv + (int64_t)r * 3 * d;
+  const int c0 = h * g.hd + i, c1 = c0 + half;
+  const float q0 = src[c0], q1 = src[c1];
+  q_out[(int64_t)r * d + c0] = q0 * cs.x - q1 * cs.y;
+  q_out[(int64_t)r * d + c1] = q1 * cs.x + q0 * cs.y;
+  const float k0 = src[d + c0], k1 = src[d + c1];
+  __half* kp = kv_k_ptr(g, lane, slot, pos, h, status);
+  if (kp) {
+    __half* vp = kp + (int64_t)g.H * g.page_tokens * g.hd;
+    kp[i] = __float2half_rn(k0 * cs.x - k1 * cs.y);
+    kp[i + half] = __float2half_rn(k1 * cs.x + k0 * cs.y);
+    vp[i] = __float2half_rn(src[2 * d + c0]);
+    vp[i + half] = __float2half_rn(src[2 * d + c1]);
+  }
+}
+
+// ------------------------------------------------------------- attention ----
+//
+// o[r][h] = softmax(q k^T / sqrt(hd)) v over positions 0..pos of the row's
+// (lane, slot) cache.  One CTA of 4 warps per (row, head); warp w takes key
+// blocks w, w+4, ... of 32 keys (one key per lane for the scores, then every
+// lane owns hd/32 output dimensions for the value sum); running max and sum are
+// kept per warp and merged at the end.  Requires kv_page_tokens >= 32 so a key
+// block never straddles a page.
+template <int HD>
+__global__ void __launch_bounds__(128)
+attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows, KVGeom g, int slot_base,
+                   int slot_stride, const int32_t* __restrict__ map_lane, int32_t* __restrict__ status) {
+  constexpr int DPL = HD / 32;  // output dims per lane
+  __shared__ float qs[HD];
+  __shared__ float wm[4], wl[4];
+  __shared__ float wacc[4][HD];
+  const int r = blockIdx.x, h = blockIdx.y;
+  if (r >= rows.n[0]) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = g.H * HD;
+  const int pos = rows.pos[r];
+  const int ln = map_lane ? map_lane[r] : rows.lane[r];
+  const int slot = slot_base + rows.iter[r] * slot_stride;
+  const float scale = rsqrtf((float)HD);
+  for (int i = threadIdx.x; i < HD; i += blockDim.x) qs[i] = q[(int64_t)r * d + h * HD + i] * scale;
+  __syncthreads();
+  const int ctx = pos + 1;
+  const int nblk = (ctx + 31) / 32;
+  float m = -INFINITY, l = 0.f, acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  for (int kb = warp; kb < nblk; kb += 4) {
+    const __half* kbase = kv_k_ptr(g, ln, slot, kb * 32, h, status);
+    if (!kbase) break;
+    const __half* vbase = kbase + (int64_t)g.H * g.page_tokens * HD;
+    const int j = kb * 32 + lane;
+    float s = -INFINITY;
+    if (j < ctx) {
+      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (int64_t)lane * HD);
+      float dot = 0.f;
+#pragma unroll
+      for (int c = 0; c < HD / 8; ++c) {
+        const uint4 v = kr[c];
+        const __half2* hv = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hv[e]);
+          dot = fmaf(qs[8 * c + 2 * e], f.x, dot);
+          dot = fmaf(qs[8 * c + 2 * e + 1], f.y, dot);
+        }
+      }
+      s = dot;
+    }
+    const float mb = warp_max(s);
+    const float mn = fmaxf(m, mb);
+    const float p = (j < ctx) ? expf(s - mn) : 0.f;
+    const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
+    l = l * corr + warp_sum(p);
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] *= corr;
+    m = mn;
+    const int nk = min(32, ctx - kb * 32);
+    for (int jj = 0; jj < nk; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+      const __half* vr = vbase + (int64_t)jj * HD + lane * DPL;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pj, __half2float(vr[e]), acc[e]);
+    }
+  }
+  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w]);
+  float Lsum = 0.f;
+  float f[4];
+  for (int w = 0; w < 4; ++w) {
+    f[w] = (wm[w] == -INFINITY) ? 0.f : expf(wm[w] - M);
+    Lsum += wl[w] * f[w];
+  }
+  for (int i = threadIdx.x; i < HD; i += blockDim.x) {
+    float v = 0.f;
+    for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
+    o[(int64_t)r * d + h * HD + i] = v / Lsum;
+  }
+}
+
+// ----------------------------------------------------------- exit rule ----
+//
+// After a loop iteration of the row's lane: delta = ||h - h_in|| / ||h_in||
+// (sums in fp64); probe at iteration l when l > min_L and (l - min_L - 1) %
+// peek_every == 0; a probe with delta < tau extends the streak, any other
+// probe resets it; the lane's loop finishes on streak >= patience or when l
+// reaches L_run.  One CTA per row.
+__global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ h,
+                                   const float* __restrict__ h_in, int d, EEParams ee,
+                                   uint8_t* __restrict__ exit_mask_out, unsigned long long* __restrict__ lane_iters) {
+  __shared__ double red[32];
+  const int r = blockIdx.x;
+  if (r >= rows.n[0]) return;
+  const int ln = rows.lane[r];
+  LaneState& st = lanes[ln];
+  const int l = st.iter + 1;
+  const bool probe = ee.enabled && l > ee.min_L && ((l - ee.min_L - 1) % ee.peek_every) == 0;
+  double num = 0.0, den = 0.0;
+  if (probe) {
+    const float* a = h + (int64_t)ln * d;
+    const float* b = h_in + (int64_t)ln * d;
+    for (int k = threadIdx.x; k < d; k += blockDim.x) {
+      const double x = a[k], y = b[k];
+      num += (x - y) * (x - y);
+      den += y * y;
+    }
+    num = block_sum_d(num, red);
+    den = block_sum_d(den, red);
+  }
+  if (threadIdx.x != 0) return;
+  bool ex = false;
+  if (probe) {
+    const bool below = (den > 0.0) && (sqrt(num / den) < ee.tau);
+    st.streak = below ? st.streak + 1 : 0;
+    ex = st.streak >= ee.patience;
+  }
+  st.iter = l;
+  const bool fin = ex || l >= st.L_run;
+  if (fin) {
+    st.phase = PH_BOUNDARY;
+    st.depth = l;
+  }
+  if (exit_mask_out) exit_mask_out[ln] = fin ? 1 : 0;
+  if (lane_iters) atomicAdd(lane_iters, 1ull);
+}
+
+// ------------------------------------------------------------- boundary ----
+
+enum HeadMode : int32_t { HEAD_ONLY = 0, HEAD_DECODE = 1 };
+
+// Argmax over the head's partial results for each boundary row; HEAD_DECODE
+// also records the token and the depth behind it, and either retires the lane
+// or moves it to its next position: cap = depth (monotonic clamp), L_run =
+// min(L_req, cap), embed the token, mark it for its pre blocks.  One CTA per row.
+__global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ part_val,
+                                     const int32_t* __restrict__ part_idx, int n_parts, int32_t mode,
+                                     int32_t* __restrict__ argmax_out, int32_t* __restrict__ tokens_out,
+                                     int32_t* __restrict__ depths_out, int n_new, MatView E, float* __restrict__ h,
+                                     int d, int max_seq, int32_t* __restrict__ status,
+                                     unsigned long long* __restrict__ tok_count) {
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  __shared__ int tok_s;
+  __shared__ int go_s;
+  const int r = blockIdx.x;
+  if (r >= rows.n[0]) return;
+  const int ln = rows.lane[r];
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int p = threadIdx.x; p < n_parts; p += blockDim.x) {
+    const float v = part_val[(int64_t)r * n_parts + p];
+    const int i = part_idx[(int64_t)r * n_parts + p];
+    if (better(v, i, bv, bi)) { bv = v; bi = i; }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+  }
+  if ((threadIdx.x & 31) == 0) { sv[threadIdx.x >> 5] = bv; si[threadIdx.x >> 5] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+      if (better(sv[w], si[w], bv, bi)) { bv = sv[w]; bi = si[w]; }
+    if (bi < 0 || bi >= E.N) { set_status(status, ST_BAD_TOKEN); bi = 0; }
+    tok_s = bi;
+    go_s = 0;
+    if (argmax_out) argmax_out[ln] = bi;
+    if (mode == HEAD_DECODE) {
+      LaneState& st = lanes[ln];
+      if (tokens_out) tokens_out[(int64_t)ln * n_new + st.n_emitted] = bi;
+      if (depths_out) depths_out[(int64_t)ln * n_new + st.n_emitted] = st.depth;
+      st.n_emitted += 1;
+      if (tok_count) atomicAdd(tok_count, 1ull);
+      if (st.n_emitted >= st.n_target) {
+        st.phase = PH_DONE;
+      } else if (st.pos + 1 >= max_seq) {
+        set_status(status, ST_BAD_POS);
+        st.phase = PH_DONE;
+      } else {
+        st.L_cap = st.depth;
+        st.L_run = min(st.L_req, st.L_cap);
+        st.pos += 1;
+        st.iter = 0;
+        st.streak = 0;
+        st.token = bi;
+        st.phase = PH_LOOP;
+        st.entered = 1;
+        go_s = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (go_s) embed_row(E, tok_s, h + (int64_t)ln * d, d);
+}
+
+// Teacher-forced token entry for masked lanes (see tl_embed_next).  One CTA per lane.
+__global__ void embed_next_kernel(LaneState* __restrict__ lanes, int n_lanes, const uint8_t* __restrict__ mask,
+                                  const int32_t* __restrict__ tokens, MatView E, float* __restrict__ h, int d,
+                                  int max_seq, int32_t* __restrict__ status) {
+  __shared__ int tok_s, go_s;
+  const int ln = blockIdx.x;
+  if (ln >= n_lanes) return;
+  if (threadIdx.x == 0) {
+    go_s = 0;
+    LaneState& st = lanes[ln];
+    if ((mask == nullptr || mask[ln]) && st.phase != PH_IDLE) {
+      int tok = tokens[ln];
+      if (tok < 0 || tok >= E.N) { set_status(status, ST_BAD_TOKEN); tok = 0; }
+      if (st.pos + 1 >= max_seq) {
+        set_status(status, ST_BAD_POS);
+      } else {
+        st.L_cap = st.depth;
+        st.L_run = min(st.L_req, st.L_cap);
+        st.pos += 1;
+        st.iter = 0;
+        st.streak = 0;
+        st.token = tok;
+        st.phase = PH_LOOP;
+        st.entered = 1;
+        tok_s = tok;
+        go_s = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (go_s) embed_row(E, tok_s, h + (int64_t)ln * d, d);
+}
+
+// Lanes of a decode call: set the request and token budget.  A request above
+// the lane's cap sets ST_EKV and leaves the lane out.
+__global__ void decode_init_kernel(LaneState* __restrict__ lanes, int n_lanes, const int32_t* __restrict__ req_L,
+                                   int n_new, int32_t* __restrict__ status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_lanes) return;
+  LaneState& st = lanes[i];
+  const int L = req_L[i];
+  if (st.phase != PH_BOUNDARY || L < 1 || L > st.L_cap) {
+    set_status(status, ST_EKV);
+    st.phase = PH_DONE;
+    return;
+  }
+  st.L_req = L;
+  st.n_emitted = 0;
+  st.n_target = n_new;
+}
+
+// Lane state after its prompt: hidden of the last prompt row (row Tn - 1 of
+// hrows, position last_pos), cap = depth = L, waiting for the head.
+__global__ void prefill_finish_kernel(LaneState* __restrict__ lanes, int ln, int Tn, int last_pos, int L,
+                                      const float* __restrict__ hrows, float* __restrict__ h, int d) {
+  for (int k = threadIdx.x; k < d; k += blockDim.x) h[(int64_t)ln * d + k] = hrows[(int64_t)(Tn - 1) * d + k];
+  if (threadIdx.x == 0) {
+    LaneState& st = lanes[ln];
+    st.L_req = L;
+    st.L_cap = L;
+    st.L_run = L;
+    st.iter = 0;
+    st.pos = last_pos;
+    st.streak = 0;
+    st.phase = PH_BOUNDARY;
+    st.depth = L;
+    st.n_emitted = 0;
+    st.n_target = 0;
+    st.token = -1;
+    st.entered = 0;
+  }
+}
+
+// Rows of a prefill: row t is position pos0 + t of lane ln at iteration 0.
+__global__ void prefill_rows_kernel(Rows rows, int ln, int pos0, int T) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+    rows.lane[t] = ln;
+    rows.pos[t] = pos0 + t;
+    rows.iter[t] = 0;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) rows.n[0] = T;
+}
+
+}  // namespace tl

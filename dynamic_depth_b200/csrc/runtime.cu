@@ -1,0 +1,729 @@
+// libtl runtime: workspace carve-up, weight loading, KV page allocation,
+// prefill, loop steps, boundary stages and the continuous-depth decode loop.
+// Every call below enqueues kernels on the context's stream; the only host
+// waits are the lagged "lanes still alive" polls of tl_decode and the explicit
+// synchronisations of tl_generate / tl_stats_get.
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "host_util.h"
+#include "kernels.cuh"
+
+namespace tl {
+
+static thread_local std::string g_cuda_err;
+
+int check_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return TL_OK;
+  g_cuda_err = cudaGetErrorString(e);
+  return TL_ECUDA;
+}
+
+static size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+static bool cfg_valid(const tl_config* c) {
+  if (!c) return false;
+  if (c->vocab <= 0 || c->d <= 0 || c->n_heads <= 0 || c->ffn <= 0 || c->n_pre < 0 || c->n_loop_layers < 1)
+    return false;
+  if (c->d % c->n_heads) return false;
+  const int hd = c->d / c->n_heads;
+  if (hd != 32 && hd != 64 && hd != 128) return false;
+  if (c->d % 32 || c->ffn % 32) return false;
+  const int fmts[3] = {c->fmt_pre, c->fmt_loop, c->fmt_embed_head};
+  bool any_int4 = false;
+  for (int f : fmts) {
+    if (f != TL_FMT_INT4 && f != TL_FMT_BF16) return false;
+    any_int4 |= f == TL_FMT_INT4;
+  }
+  if (any_int4 && (c->group <= 0 || c->group % 32 || c->d % c->group || c->ffn % c->group)) return false;
+  if (!(c->rms_eps >= 0.f) || !(c->rope_base > 0.f)) return false;
+  if (c->max_lanes < 1 || c->max_lanes > 1024 || c->max_seq < 1 || c->L_max < 1) return false;
+  if (c->kv_page_tokens < 32 || (c->kv_page_tokens & (c->kv_page_tokens - 1))) return false;
+  if (c->kv_pool_pages < 0 || c->max_prefill_tokens < 0 || c->max_prefill_tokens > c->max_seq) return false;
+  return true;
+}
+
+static size_t mat_bytes(const tl_config* c, int fmt, int64_t N, int64_t K) {
+  if (fmt == TL_FMT_INT4) return (size_t)(N * K / 2) + (size_t)(N * (K / c->group)) * 2;
+  return (size_t)(N * K) * 2;
+}
+
+struct MatSpec {
+  int fmt;
+  int64_t N, K;
+};
+
+static std::vector<MatSpec> mat_specs(const tl_config* c) {
+  std::vector<MatSpec> v;
+  const int64_t d = c->d, F = c->ffn, V = c->vocab;
+  v.push_back({c->fmt_embed_head, V, d});
+  for (int b = 0; b < c->n_pre + c->n_loop_layers; ++b) {
+    const int f = b < c->n_pre ? c->fmt_pre : c->fmt_loop;
+    v.push_back({f, 3 * d, d});
+    v.push_back({f, d, d});
+    v.push_back({f, F, d});
+    v.push_back({f, F, d});
+    v.push_back({f, d, F});
+  }
+  v.push_back({c->fmt_embed_head, V, d});
+  return v;
+}
+
+static constexpr size_t kBlobHeader = 8 + 48;
+
+static size_t blob_bytes(const tl_config* c) {
+  size_t s = kBlobHeader;
+  for (const auto& m : mat_specs(c)) s += mat_bytes(c, m.fmt, m.N, m.K);
+  s += (size_t)(2 * (c->n_pre + c->n_loop_layers) + 1) * c->d * 4;
+  return s;
+}
+
+// Offsets of every workspace region (computed identically by tl_workspace_bytes and tl_create).
+struct Layout {
+  int n_slots, pages_per_seq, n_pages, max_rows, n_parts, max_prefill;
+  size_t page_elems;
+  std::vector<size_t> mat_off;  // per matrix
+  size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[4], act_a, act_qkv, act_q, act_o, act_u,
+      part_val, part_idx, tok_stage, L_stage, mask_stage, out_tok, out_dep, status, counters, alive, total;
+};
+
+static Layout make_layout(const tl_config* c) {
+  Layout L;
+  const int hd = c->d / c->n_heads;
+  L.max_prefill = c->max_prefill_tokens ? c->max_prefill_tokens : c->max_seq;
+  L.n_slots = c->n_pre + c->L_max * c->n_loop_layers;
+  L.pages_per_seq = (c->max_seq + c->kv_page_tokens - 1) / c->kv_page_tokens;
+  L.n_pages = c->kv_pool_pages ? c->kv_pool_pages : c->max_lanes * L.n_slots * L.pages_per_seq;
+  L.page_elems = (size_t)2 * c->n_heads * c->kv_page_tokens * hd;
+  L.max_rows = c->max_lanes > L.max_prefill ? c->max_lanes : L.max_prefill;
+  L.n_parts = (c->vocab + GEMV_WARPS - 1) / GEMV_WARPS;
+  size_t o = 0;
+  for (const auto& m : mat_specs(c)) {
+    L.mat_off.push_back(o);
+    o = align_up(o + mat_bytes(c, m.fmt, m.N, m.K));
+  }
+  const size_t d = c->d, F = c->ffn, R = L.max_rows, lanes = c->max_lanes;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  L.gains = take((size_t)(2 * (c->n_pre + c->n_loop_layers) + 1) * d * 4);
+  L.rope = take((size_t)c->max_seq * (hd / 2) * 8);
+  L.page_table = take(lanes * L.n_slots * L.pages_per_seq * 4);
+  L.kv = take((size_t)L.n_pages * L.page_elems * 2);
+  L.lanes = take(lanes * sizeof(LaneState));
+  L.h = take(lanes * d * 4);
+  L.h_in = take(lanes * d * 4);
+  L.hrows = take((size_t)L.max_prefill * d * 4);
+  for (int i = 0; i < 4; ++i) L.rows[i] = take(4 + 3 * R * 4 + 16);
+  L.act_a = take(R * d * 4);
+  L.act_qkv = take(R * 3 * d * 4);
+  L.act_q = take(R * d * 4);
+  L.act_o = take(R * d * 4);
+  L.act_u = take(R * F * 4);
+  L.part_val = take(lanes * L.n_parts * 4);
+  L.part_idx = take(lanes * L.n_parts * 4);
+  L.tok_stage = take(R * 4);
+  L.L_stage = take(lanes * 4);
+  L.mask_stage = take(lanes);
+  L.out_tok = take(lanes * (size_t)c->max_seq * 4);
+  L.out_dep = take(lanes * (size_t)c->max_seq * 4);
+  L.status = take(4);
+  L.counters = take(4 * 8);
+  L.alive = take(4);
+  L.total = o;
+  return L;
+}
+
+struct BlockW {
+  MatView wqkv, wo, wg, wu, wd;
+  const float *g1, *g2;
+};
+
+}  // namespace tl
+
+using namespace tl;
+
+struct tl_ctx {
+  tl_config cfg;
+  Layout lay;
+  cudaStream_t stream;
+  char* ws;
+  size_t ws_bytes;
+  int hd;
+  bool loaded = false;
+  MatView embed, head;
+  std::vector<BlockW> pre, loop;
+  const float* g_final;
+  KVGeom kv;
+  float2* rope;
+  int32_t* page_table;
+  LaneState* lanes;
+  float *h, *h_in, *hrows;
+  Rows rows[4];  // 0 loop, 1 boundary, 2 entered, 3 prefill / mask
+  float *act_a, *act_qkv, *act_q, *act_o, *act_u;
+  float* part_val;
+  int32_t* part_idx;
+  int32_t *tok_stage, *L_stage, *out_tok, *out_dep, *status, *alive;
+  uint8_t* mask_stage;
+  unsigned long long* counters;  // 0 lane iterations, 1 tokens
+  EEParams ee{0.0, 2, 0, 1, 0};
+  // host state
+  std::vector<int32_t> h_page_table;  // [lanes][slots][pages]
+  std::vector<int32_t> refcount;      // per page
+  std::vector<int32_t> free_pages;
+  std::vector<int32_t> lane_L;        // prefill depth per lane (0 = empty)
+  int32_t* pinned_alive = nullptr;    // ring of alive counts
+  cudaEvent_t alive_ev[4];
+  int64_t steps = 0, prefill_tokens = 0, launches = 0;
+};
+
+static constexpr int kAliveRing = 4;
+
+namespace {
+
+// -------------------------------------------------------------- launches ----
+
+int launch_err(tl_ctx* c) {
+  c->launches++;
+  return check_cuda(cudaGetLastError());
+}
+
+template <int FMT, int R, int EPI>
+int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView& W, const MatView& W2,
+                const ProjOut& o) {
+  const size_t smem = (size_t)R * W.K * 4;
+  auto kern = gemv_kernel<FMT, R, EPI>;
+  static bool attr_done = false;  // once per instantiation
+  if (!attr_done) {
+    TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    attr_done = true;
+  }
+  if (smem > 200 * 1024) return TL_EINVAL;
+  const unsigned grid = (unsigned)((W.N + GEMV_WARPS - 1) / GEMV_WARPS);
+  kern<<<grid, GEMV_WARPS * 32, smem, c->stream>>>(X, n_rows, W, W2, o);
+  return launch_err(c);
+}
+
+template <int FMT, int EPI>
+int gemv_pick_r(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView& W2,
+                const ProjOut& o) {
+  if (max_rows <= 1) return gemv_launch<FMT, 1, EPI>(c, X, n, W, W2, o);
+  if (max_rows <= 2) return gemv_launch<FMT, 2, EPI>(c, X, n, W, W2, o);
+  if (max_rows <= 4) return gemv_launch<FMT, 4, EPI>(c, X, n, W, W2, o);
+  return gemv_launch<FMT, 8, EPI>(c, X, n, W, W2, o);
+}
+
+template <int FMT, int EPI>
+int gemm_launch(tl_ctx* c, int max_rows, const float* A, const int32_t* n, const MatView& W, const MatView& W2,
+                const ProjOut& o) {
+  dim3 grid((W.N + SG_BN - 1) / SG_BN, (max_rows + SG_BM - 1) / SG_BM);
+  gemm_simt_kernel<FMT, EPI><<<grid, 256, 0, c->stream>>>(A, n, W, W2, o);
+  return launch_err(c);
+}
+
+constexpr int kGemvMaxRows = 8;
+
+template <int EPI>
+int proj_epi(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView& W2,
+             ProjOut o) {
+  const bool gemv = max_rows <= kGemvMaxRows;
+  if (EPI == EPI_ARGMAX)
+    o.n_parts = gemv ? (W.N + GEMV_WARPS - 1) / GEMV_WARPS : (W.N + SG_BN - 1) / SG_BN;
+  if (W.fmt == TL_FMT_INT4)
+    return gemv ? gemv_pick_r<TL_FMT_INT4, EPI>(c, max_rows, X, n, W, W2, o)
+                : gemm_launch<TL_FMT_INT4, EPI>(c, max_rows, X, n, W, W2, o);
+  return gemv ? gemv_pick_r<TL_FMT_BF16, EPI>(c, max_rows, X, n, W, W2, o)
+              : gemm_launch<TL_FMT_BF16, EPI>(c, max_rows, X, n, W, W2, o);
+}
+
+int proj(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView* W2,
+         const ProjOut& o) {
+  const MatView& w2 = W2 ? *W2 : W;
+  switch (o.epi) {
+    case EPI_STORE: return proj_epi<EPI_STORE>(c, max_rows, X, n, W, w2, o);
+    case EPI_RESID: return proj_epi<EPI_RESID>(c, max_rows, X, n, W, w2, o);
+    case EPI_SWIGLU: return proj_epi<EPI_SWIGLU>(c, max_rows, X, n, W, w2, o);
+    default: return proj_epi<EPI_ARGMAX>(c, max_rows, X, n, W, w2, o);
+  }
+}
+
+int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
+  dim3 grid(max_rows, c->cfg.n_heads);
+  switch (c->hd) {
+    case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+    case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+    default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+  }
+  return launch_err(c);
+}
+
+// One transformer block on the rows of `rows`; hidden rows live in hbuf
+// (indexed through map, or by row when map is null).
+int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int32_t* map, const BlockW& w,
+              int slot_base, int slot_stride, float* h_in) {
+  const int d = c->cfg.d, F = c->cfg.ffn;
+  const float eps = c->cfg.rms_eps;
+  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in);
+  TL_TRY(launch_err(c));
+  ProjOut o{};
+  o.epi = EPI_STORE;
+  o.out = c->act_qkv;
+  o.ldo = 3 * d;
+  TL_TRY(proj(c, max_rows, c->act_a, rows.n, w.wqkv, nullptr, o));
+  rope_kv_kernel<<<max_rows, d / 2, 0, c->stream>>>(c->act_qkv, c->act_q, rows, c->kv, c->rope, slot_base,
+                                                     slot_stride, nullptr, c->status);
+  TL_TRY(launch_err(c));
+  TL_TRY(attn_launch(c, max_rows, rows, slot_base, slot_stride));
+  ProjOut r{};
+  r.epi = EPI_RESID;
+  r.h = hbuf;
+  r.map = map;
+  TL_TRY(proj(c, max_rows, c->act_o, rows.n, w.wo, nullptr, r));
+  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr);
+  TL_TRY(launch_err(c));
+  ProjOut s{};
+  s.epi = EPI_SWIGLU;
+  s.out = c->act_u;
+  s.ldo = F;
+  TL_TRY(proj(c, max_rows, c->act_a, rows.n, w.wg, &w.wu, s));
+  return proj(c, max_rows, c->act_u, rows.n, w.wd, nullptr, r);
+}
+
+// Row table `which` from lanes 0..n_consider-1 (all lanes when n_consider <= 0).
+int build_rows(tl_ctx* c, int which, int sel, const uint8_t* mask, const int32_t* per_lane_L, uint8_t* exit_mask,
+               int32_t* alive, int n_consider = 0) {
+  const int n = n_consider > 0 ? n_consider : c->cfg.max_lanes;
+  build_rows_kernel<<<1, 1024, 0, c->stream>>>(c->lanes, n, sel, mask, per_lane_L, c->rows[which], exit_mask,
+                                               alive, c->status);
+  return launch_err(c);
+}
+
+// One loop iteration for the lanes selected into rows[0].
+int loop_iteration(tl_ctx* c, int max_rows, uint8_t* exit_mask) {
+  const Rows& R = c->rows[0];
+  const int Lb = c->cfg.n_loop_layers;
+  for (int m = 0; m < Lb; ++m)
+    TL_TRY(run_block(c, R, max_rows, c->h, R.lane, c->loop[m], c->cfg.n_pre + m, Lb, m == 0 ? c->h_in : nullptr));
+  exit_update_kernel<<<max_rows, 256, 0, c->stream>>>(R, c->lanes, c->h, c->h_in, c->cfg.d, c->ee, exit_mask,
+                                                      &c->counters[0]);
+  c->steps++;
+  return launch_err(c);
+}
+
+int pre_blocks_for_entered(tl_ctx* c, int max_rows) {
+  if (c->cfg.n_pre == 0) return build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, max_rows);
+  TL_TRY(build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, max_rows));
+  const Rows& E = c->rows[2];
+  for (int b = 0; b < c->cfg.n_pre; ++b) TL_TRY(run_block(c, E, max_rows, c->h, E.lane, c->pre[b], b, 0, nullptr));
+  return TL_OK;
+}
+
+// Boundary stage for the lanes in rows[1]: final norm, head, argmax, then
+// (decode mode) token bookkeeping, embedding and pre blocks.
+int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax, int32_t* tok_out,
+               int32_t* dep_out, int n_new) {
+  const Rows& B = c->rows[1];
+  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(c->h, B.lane, B.n, c->cfg.d, c->g_final, c->cfg.rms_eps,
+                                                       c->act_a, nullptr);
+  TL_TRY(launch_err(c));
+  ProjOut o{};
+  o.epi = EPI_ARGMAX;
+  o.logits = logits;
+  o.lmap = B.lane;
+  o.ldo = c->cfg.vocab;
+  o.part_val = c->part_val;
+  o.part_idx = c->part_idx;
+  TL_TRY(proj(c, max_rows, c->act_a, B.n, c->head, nullptr, o));
+  const int n_parts = max_rows <= kGemvMaxRows ? (c->cfg.vocab + GEMV_WARPS - 1) / GEMV_WARPS
+                                               : (c->cfg.vocab + SG_BN - 1) / SG_BN;
+  head_finalize_kernel<<<max_rows, 256, 0, c->stream>>>(B, c->lanes, c->part_val, c->part_idx, n_parts, mode, argmax,
+                                                        tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
+                                                        c->cfg.max_seq, c->status, &c->counters[1]);
+  TL_TRY(launch_err(c));
+  if (mode == HEAD_DECODE) return pre_blocks_for_entered(c, max_rows);
+  return TL_OK;
+}
+
+// ------------------------------------------------------------ KV pages ----
+
+void release_lane_pages(tl_ctx* c, int lane) {
+  const int per_lane = c->lay.n_slots * c->lay.pages_per_seq;
+  int32_t* t = &c->h_page_table[(size_t)lane * per_lane];
+  for (int i = 0; i < per_lane; ++i) {
+    if (t[i] >= 0 && --c->refcount[t[i]] == 0) c->free_pages.push_back(t[i]);
+    t[i] = -1;
+  }
+  c->lane_L[lane] = 0;
+}
+
+}  // namespace
+
+// ============================================================== C ABI ====
+
+extern "C" int tl_workspace_bytes(const tl_config* cfg, size_t* out) {
+  if (!cfg_valid(cfg) || !out) return TL_EINVAL;
+  *out = make_layout(cfg).total;
+  return TL_OK;
+}
+
+extern "C" int tl_weights_bytes(const tl_config* cfg, size_t* out) {
+  if (!cfg_valid(cfg) || !out) return TL_EINVAL;
+  *out = blob_bytes(cfg);
+  return TL_OK;
+}
+
+extern "C" const char* tl_strerror(int s) {
+  switch (s) {
+    case TL_OK: return "ok";
+    case TL_EINVAL: return "invalid argument";
+    case TL_ENOMEM: return "out of memory (workspace or KV page pool)";
+    case TL_ESTATE: return "invalid state for this call";
+    case TL_EKV: return "requested depth exceeds the lane's KV cache";
+    case TL_ECUDA: return "CUDA error";
+    case TL_ETIMEOUT: return "device wait timed out";
+    case TL_EDEVICE: return "device reported an out-of-range index";
+    default: return "unknown status";
+  }
+}
+
+extern "C" const char* tl_last_cuda_error(void) { return g_cuda_err.c_str(); }
+
+__global__ void rope_table_kernel(float2* t, int max_seq, int half, double base) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)max_seq * half) return;
+  const int p = (int)(i / half), k = (int)(i % half);
+  const double theta = pow(base, -2.0 * k / (2.0 * half));
+  double s, co;
+  sincos((double)p * theta, &s, &co);
+  t[i] = make_float2((float)co, (float)s);
+}
+
+__global__ void lanes_init_kernel(LaneState* l, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    LaneState z{};
+    z.phase = PH_IDLE;
+    z.token = -1;
+    l[i] = z;
+  }
+}
+
+extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void* stream, tl_ctx** out) {
+  if (!cfg_valid(cfg) || !dev_ws || !out || ((uintptr_t)dev_ws & 255)) return TL_EINVAL;
+  Layout lay = make_layout(cfg);
+  if (bytes < lay.total) return TL_ENOMEM;
+  tl_ctx* c = new tl_ctx();
+  c->cfg = *cfg;
+  c->lay = lay;
+  c->stream = (cudaStream_t)stream;
+  c->ws = (char*)dev_ws;
+  c->ws_bytes = bytes;
+  c->hd = cfg->d / cfg->n_heads;
+  char* w = c->ws;
+  // weight views
+  auto specs = mat_specs(cfg);
+  std::vector<MatView> mv;
+  for (size_t i = 0; i < specs.size(); ++i) {
+    MatView m{};
+    m.fmt = specs[i].fmt;
+    m.N = (int)specs[i].N;
+    m.K = (int)specs[i].K;
+    m.group = cfg->group;
+    char* p = w + lay.mat_off[i];
+    if (m.fmt == TL_FMT_INT4) {
+      m.q = (const uint8_t*)p;
+      m.s = (const __half*)(p + (size_t)m.N * m.K / 2);
+    } else {
+      m.bf = (const uint16_t*)p;
+    }
+    mv.push_back(m);
+  }
+  const float* gains = (const float*)(w + lay.gains);
+  c->embed = mv[0];
+  c->head = mv.back();
+  const int nb = cfg->n_pre + cfg->n_loop_layers;
+  for (int b = 0; b < nb; ++b) {
+    BlockW bw{mv[1 + 5 * b], mv[2 + 5 * b], mv[3 + 5 * b], mv[4 + 5 * b], mv[5 + 5 * b],
+              gains + (size_t)(2 * b) * cfg->d, gains + (size_t)(2 * b + 1) * cfg->d};
+    (b < cfg->n_pre ? c->pre : c->loop).push_back(bw);
+  }
+  c->g_final = gains + (size_t)(2 * nb) * cfg->d;
+  c->rope = (float2*)(w + lay.rope);
+  c->page_table = (int32_t*)(w + lay.page_table);
+  c->kv.pool = (__half*)(w + lay.kv);
+  c->kv.page_table = c->page_table;
+  c->kv.n_slots = lay.n_slots;
+  c->kv.pages_per_seq = lay.pages_per_seq;
+  c->kv.page_tokens = cfg->kv_page_tokens;
+  int sh = 0;
+  while ((1 << sh) < cfg->kv_page_tokens) ++sh;
+  c->kv.page_shift = sh;
+  c->kv.n_pages = lay.n_pages;
+  c->kv.H = cfg->n_heads;
+  c->kv.hd = c->hd;
+  c->kv.page_elems = (int64_t)lay.page_elems;
+  c->lanes = (LaneState*)(w + lay.lanes);
+  c->h = (float*)(w + lay.h);
+  c->h_in = (float*)(w + lay.h_in);
+  c->hrows = (float*)(w + lay.hrows);
+  for (int i = 0; i < 4; ++i) {
+    int32_t* base = (int32_t*)(w + lay.rows[i]);
+    c->rows[i].n = base;
+    c->rows[i].lane = base + 4;
+    c->rows[i].pos = base + 4 + lay.max_rows;
+    c->rows[i].iter = base + 4 + 2 * lay.max_rows;
+  }
+  c->act_a = (float*)(w + lay.act_a);
+  c->act_qkv = (float*)(w + lay.act_qkv);
+  c->act_q = (float*)(w + lay.act_q);
+  c->act_o = (float*)(w + lay.act_o);
+  c->act_u = (float*)(w + lay.act_u);
+  c->part_val = (float*)(w + lay.part_val);
+  c->part_idx = (int32_t*)(w + lay.part_idx);
+  c->tok_stage = (int32_t*)(w + lay.tok_stage);
+  c->L_stage = (int32_t*)(w + lay.L_stage);
+  c->mask_stage = (uint8_t*)(w + lay.mask_stage);
+  c->out_tok = (int32_t*)(w + lay.out_tok);
+  c->out_dep = (int32_t*)(w + lay.out_dep);
+  c->status = (int32_t*)(w + lay.status);
+  c->counters = (unsigned long long*)(w + lay.counters);
+  c->alive = (int32_t*)(w + lay.alive);
+  // host-side page allocator
+  const size_t per_lane = (size_t)lay.n_slots * lay.pages_per_seq;
+  c->h_page_table.assign(per_lane * cfg->max_lanes, -1);
+  c->refcount.assign(lay.n_pages, 0);
+  c->free_pages.reserve(lay.n_pages);
+  for (int p = lay.n_pages - 1; p >= 0; --p) c->free_pages.push_back(p);
+  c->lane_L.assign(cfg->max_lanes, 0);
+  int st = TL_OK;
+  do {
+    const int half = c->hd / 2;
+    const int64_t n = (int64_t)cfg->max_seq * half;
+    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, c->stream>>>(c->rope, cfg->max_seq, half,
+                                                                         (double)cfg->rope_base);
+    if ((st = launch_err(c)) != TL_OK) break;
+    lanes_init_kernel<<<(cfg->max_lanes + 255) / 256, 256, 0, c->stream>>>(c->lanes, cfg->max_lanes);
+    if ((st = launch_err(c)) != TL_OK) break;
+    if ((st = check_cuda(cudaMemsetAsync(w + lay.page_table, 0xFF, per_lane * cfg->max_lanes * 4, c->stream))) != TL_OK) break;
+    if ((st = check_cuda(cudaMemsetAsync(c->status, 0, 4, c->stream))) != TL_OK) break;
+    if ((st = check_cuda(cudaMemsetAsync(c->counters, 0, 32, c->stream))) != TL_OK) break;
+    for (int i = 0; i < 4; ++i)
+      if ((st = check_cuda(cudaMemsetAsync(c->rows[i].n, 0, 4, c->stream))) != TL_OK) break;
+    if (st != TL_OK) break;
+    if ((st = check_cuda(cudaHostAlloc((void**)&c->pinned_alive, kAliveRing * sizeof(int32_t), cudaHostAllocDefault))) != TL_OK) break;
+    for (int i = 0; i < kAliveRing; ++i)
+      if ((st = check_cuda(cudaEventCreateWithFlags(&c->alive_ev[i], cudaEventDisableTiming))) != TL_OK) break;
+  } while (0);
+  if (st != TL_OK) {
+    if (c->pinned_alive) cudaFreeHost(c->pinned_alive);
+    delete c;
+    return st;
+  }
+  *out = c;
+  return TL_OK;
+}
+
+extern "C" int tl_destroy(tl_ctx* c) {
+  if (!c) return TL_EINVAL;
+  cudaStreamSynchronize(c->stream);
+  for (int i = 0; i < kAliveRing; ++i) cudaEventDestroy(c->alive_ev[i]);
+  if (c->pinned_alive) cudaFreeHost(c->pinned_alive);
+  delete c;
+  return TL_OK;
+}
+
+extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
+  if (!c || !blob) return TL_EINVAL;
+  const tl_config* cfg = &c->cfg;
+  if (bytes != blob_bytes(cfg)) return TL_EINVAL;
+  const char* b = (const char*)blob;
+  if (memcmp(b, "TLWBLOB1", 8) != 0) return TL_EINVAL;
+  int32_t hdr_i[10];
+  float hdr_f[2];
+  memcpy(hdr_i, b + 8, 40);
+  memcpy(hdr_f, b + 48, 8);
+  const int32_t want[10] = {cfg->vocab, cfg->d, cfg->n_heads, cfg->ffn, cfg->n_pre, cfg->n_loop_layers,
+                            cfg->fmt_pre, cfg->fmt_loop, cfg->fmt_embed_head, cfg->group};
+  if (memcmp(hdr_i, want, 40) != 0 || hdr_f[0] != cfg->rms_eps || hdr_f[1] != cfg->rope_base) return TL_EINVAL;
+  size_t off = kBlobHeader;
+  auto specs = mat_specs(cfg);
+  for (size_t i = 0; i < specs.size(); ++i) {
+    const size_t n = mat_bytes(cfg, specs[i].fmt, specs[i].N, specs[i].K);
+    TL_CUDA(cudaMemcpyAsync(c->ws + c->lay.mat_off[i], b + off, n, cudaMemcpyHostToDevice, c->stream));
+    off += n;
+  }
+  const size_t gb = (size_t)(2 * (cfg->n_pre + cfg->n_loop_layers) + 1) * cfg->d * 4;
+  TL_CUDA(cudaMemcpyAsync(c->ws + c->lay.gains, b + off, gb, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaStreamSynchronize(c->stream));
+  c->loaded = true;
+  return TL_OK;
+}
+
+extern "C" int tl_set_early_exit(tl_ctx* c, double tau, int32_t min_L, int32_t patience, int32_t peek_every) {
+  if (!c || peek_every < 1 || min_L < 0 || patience < 0) return TL_EINVAL;
+  c->ee.tau = tau;
+  c->ee.min_L = min_L;
+  c->ee.patience = patience;
+  c->ee.peek_every = peek_every;
+  c->ee.enabled = (tau > 0.0 && patience > 0) ? 1 : 0;
+  return TL_OK;
+}
+
+extern "C" int tl_prefill(tl_ctx* c, int32_t lane, const int32_t* host_tokens, int32_t T, int32_t L,
+                          int32_t share_from, int32_t shared_tokens, float* dev_hidden_out) {
+  if (!c || !host_tokens) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  const tl_config& cfg = c->cfg;
+  if (lane < 0 || lane >= cfg.max_lanes || T < 1 || T > c->lay.max_prefill || L < 1 || L > cfg.L_max)
+    return TL_EINVAL;
+  for (int i = 0; i < T; ++i)
+    if (host_tokens[i] < 0 || host_tokens[i] >= cfg.vocab) return TL_EINVAL;
+  int share_pages = 0;
+  if (share_from >= 0) {
+    if (share_from >= cfg.max_lanes || share_from == lane || c->lane_L[share_from] < L || shared_tokens < 0 ||
+        shared_tokens > T)
+      return TL_EINVAL;
+    // whole pages only, and never the last prompt position (this lane computes it)
+    share_pages = (shared_tokens < T ? shared_tokens : T - 1) / cfg.kv_page_tokens;
+  }
+  // pages: slots of the pre blocks and of iterations 1..L, for every position up to max_seq
+  const int P = cfg.n_pre, Lb = cfg.n_loop_layers, pps = c->lay.pages_per_seq;
+  const int used_slots = P + L * Lb;
+  const int need = used_slots * (pps - share_pages);
+  release_lane_pages(c, lane);
+  if ((int)c->free_pages.size() < need) return TL_ENOMEM;
+  const size_t per_lane = (size_t)c->lay.n_slots * pps;
+  int32_t* t = &c->h_page_table[(size_t)lane * per_lane];
+  const int32_t* donor = share_from >= 0 ? &c->h_page_table[(size_t)share_from * per_lane] : nullptr;
+  for (int s = 0; s < used_slots; ++s)
+    for (int p = 0; p < pps; ++p) {
+      int32_t pg;
+      if (p < share_pages) {
+        pg = donor[(size_t)s * pps + p];
+      } else {
+        pg = c->free_pages.back();
+        c->free_pages.pop_back();
+      }
+      c->refcount[pg]++;
+      t[(size_t)s * pps + p] = pg;
+    }
+  c->lane_L[lane] = L;
+  TL_CUDA(cudaMemcpyAsync(c->page_table + (size_t)lane * per_lane, t, per_lane * 4, cudaMemcpyHostToDevice, c->stream));
+  // rows: the positions not covered by the shared pages
+  const int pos0 = share_pages * cfg.kv_page_tokens;
+  const int Tn = T - pos0;
+  const Rows& R = c->rows[3];
+  TL_CUDA(cudaMemcpyAsync(c->tok_stage, host_tokens + pos0, (size_t)Tn * 4, cudaMemcpyHostToDevice, c->stream));
+  prefill_rows_kernel<<<(Tn + 255) / 256, 256, 0, c->stream>>>(R, lane, pos0, Tn);
+  TL_TRY(launch_err(c));
+  embed_rows_kernel<<<Tn, 256, 0, c->stream>>>(c->embed, c->tok_stage, Tn, cfg.d, c->hrows, c->status);
+  TL_TRY(launch_err(c));
+  for (int b = 0; b < P; ++b) TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->pre[b], b, 0, nullptr));
+  for (int l = 0; l < L; ++l)
+    for (int m = 0; m < Lb; ++m)
+      TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr));
+  prefill_finish_kernel<<<1, 256, 0, c->stream>>>(c->lanes, lane, Tn, T - 1, L, c->hrows, c->h, cfg.d);
+  TL_TRY(launch_err(c));
+  if (dev_hidden_out)
+    TL_CUDA(cudaMemcpyAsync(dev_hidden_out, c->hrows, (size_t)Tn * cfg.d * 4, cudaMemcpyDeviceToDevice, c->stream));
+  c->prefill_tokens += Tn;
+  return TL_OK;
+}
+
+extern "C" int tl_loop_step(tl_ctx* c, const int32_t* dev_L, const uint8_t* dev_mask, uint8_t* dev_exit) {
+  if (!c) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  TL_TRY(build_rows(c, 0, SEL_LOOP, dev_mask, dev_L, dev_exit, nullptr));
+  return loop_iteration(c, c->cfg.max_lanes, dev_exit);
+}
+
+extern "C" int tl_head_logits(tl_ctx* c, const uint8_t* dev_mask, float* dev_logits, int32_t* dev_argmax) {
+  if (!c) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  TL_TRY(build_rows(c, 1, dev_mask ? SEL_MASK : SEL_BOUNDARY, dev_mask, nullptr, nullptr, nullptr));
+  return head_stage(c, c->cfg.max_lanes, HEAD_ONLY, dev_logits, dev_argmax, nullptr, nullptr, 0);
+}
+
+extern "C" int tl_embed_next(tl_ctx* c, const uint8_t* dev_mask, const int32_t* dev_tokens) {
+  if (!c || !dev_tokens) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  embed_next_kernel<<<c->cfg.max_lanes, 256, 0, c->stream>>>(c->lanes, c->cfg.max_lanes, dev_mask, dev_tokens,
+                                                             c->embed, c->h, c->cfg.d, c->cfg.max_seq, c->status);
+  TL_TRY(launch_err(c));
+  return pre_blocks_for_entered(c, c->cfg.max_lanes);
+}
+
+static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
+  decode_init_kernel<<<(n_lanes + 255) / 256, 256, 0, c->stream>>>(c->lanes, n_lanes, c->L_stage, n_new, c->status);
+  TL_TRY(launch_err(c));
+  // upper bound on ticks: every token runs at most L_max iterations, plus the first
+  const int64_t max_ticks = (int64_t)n_new * (c->cfg.L_max + 1) + 4;
+  int64_t polled = 0;
+  for (int64_t t = 0; t < max_ticks; ++t) {
+    // lagged poll: tick t - (ring-1) must be known before launching tick t
+    if (t >= kAliveRing - 1) {
+      const int64_t q = t - (kAliveRing - 1);
+      TL_CUDA(cudaEventSynchronize(c->alive_ev[q % kAliveRing]));
+      polled = q;
+      if (c->pinned_alive[q % kAliveRing] == 0) break;
+    }
+    TL_TRY(build_rows(c, 1, SEL_BOUNDARY, nullptr, nullptr, nullptr, c->alive, n_lanes));
+    TL_CUDA(cudaMemcpyAsync(&c->pinned_alive[t % kAliveRing], c->alive, 4, cudaMemcpyDeviceToHost, c->stream));
+    TL_CUDA(cudaEventRecord(c->alive_ev[t % kAliveRing], c->stream));
+    TL_TRY(head_stage(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new));
+    TL_TRY(build_rows(c, 0, SEL_LOOP, nullptr, nullptr, nullptr, nullptr, n_lanes));
+    TL_TRY(loop_iteration(c, n_lanes, nullptr));
+  }
+  (void)polled;
+  return TL_OK;
+}
+
+extern "C" int tl_decode(tl_ctx* c, const int32_t* host_L, int32_t n_lanes, int32_t n_new, int32_t* tok_out,
+                         int32_t* dep_out) {
+  if (!c || !host_L) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  if (n_lanes < 1 || n_lanes > c->cfg.max_lanes || n_new < 1) return TL_EINVAL;
+  for (int i = 0; i < n_lanes; ++i) {
+    if (host_L[i] < 1 || host_L[i] > c->cfg.L_max) return TL_EINVAL;
+    if (c->lane_L[i] == 0) return TL_ESTATE;
+    if (host_L[i] > c->lane_L[i]) return TL_EKV;
+  }
+  TL_CUDA(cudaMemcpyAsync(c->L_stage, host_L, (size_t)n_lanes * 4, cudaMemcpyHostToDevice, c->stream));
+  return decode_impl(c, n_lanes, n_new, tok_out, dep_out);
+}
+
+extern "C" int tl_generate(tl_ctx* c, const int32_t* host_prompts, int32_t n_lanes, int32_t T,
+                           const int32_t* host_L, int32_t n_new, int32_t* host_tok, int32_t* host_dep) {
+  if (!c || !host_prompts || !host_L || !host_tok) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  if (n_lanes < 1 || n_lanes > c->cfg.max_lanes || n_new < 1 || T < 1 || T + n_new - 1 > c->cfg.max_seq)
+    return TL_EINVAL;
+  for (int i = 0; i < n_lanes; ++i)
+    TL_TRY(tl_prefill(c, i, host_prompts + (size_t)i * T, T, host_L[i], -1, 0, nullptr));
+  TL_CUDA(cudaMemcpyAsync(c->L_stage, host_L, (size_t)n_lanes * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_TRY(decode_impl(c, n_lanes, n_new, c->out_tok, c->out_dep));
+  TL_CUDA(cudaMemcpyAsync(host_tok, c->out_tok, (size_t)n_lanes * n_new * 4, cudaMemcpyDeviceToHost, c->stream));
+  if (host_dep)
+    TL_CUDA(cudaMemcpyAsync(host_dep, c->out_dep, (size_t)n_lanes * n_new * 4, cudaMemcpyDeviceToHost, c->stream));
+  TL_CUDA(cudaStreamSynchronize(c->stream));
+  return TL_OK;
+}
+
+extern "C" int tl_stats_get(tl_ctx* c, tl_stats* out) {
+  if (!c || !out) return TL_EINVAL;
+  unsigned long long ctr[4];
+  int32_t st = 0;
+  TL_CUDA(cudaMemcpyAsync(ctr, c->counters, 32, cudaMemcpyDeviceToHost, c->stream));
+  TL_CUDA(cudaMemcpyAsync(&st, c->status, 4, cudaMemcpyDeviceToHost, c->stream));
+  TL_CUDA(cudaMemsetAsync(c->status, 0, 4, c->stream));
+  TL_CUDA(cudaStreamSynchronize(c->stream));
+  out->loop_steps = c->steps;
+  out->lane_iterations = (int64_t)ctr[0];
+  out->tokens_emitted = (int64_t)ctr[1];
+  out->prefill_tokens = c->prefill_tokens;
+  out->kernel_launches = c->launches;
+  out->device_status = st;
+  out->kv_pages_used = c->lay.n_pages - (int32_t)c->free_pages.size();
+  return TL_OK;
+}

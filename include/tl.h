@@ -1,0 +1,259 @@
+/*
+ * tl.h -- C ABI of libtl.so: per-lane-depth decode of a weight-shared looped
+ * transformer on NVIDIA B200 (sm_100a).
+ *
+ * The model ("Benchmark Comparison" (vs generic runtimes), "Where Generic
+ * Runtimes Lose On Looped Checkpoints"):
+ *     embed -> pre blocks -> shared loop block x L -> head
+ * L is a runtime argument over the same weights ("Dynamic-L Inference", "The
+ * Core Idea"); each lane of a batch has its own L ("Dynamic-L Inference",
+ * "L-Aware Batching").  Every pre block and every (loop iteration, body layer)
+ * keeps its own K/V cache ("Benchmark Comparison" (measured benchmarks),
+ * section 9, storage for "2 pre + 8 loop" blocks).  Lanes advance one loop
+ * iteration per step, each at its own iteration index, and the exit decision of
+ * a step is taken on the device before the next step is formed ("Depth-adaptive
+ * Inference of Looped Language Models via Continuous Depth Batching", CDB
+ * design).  Early exit on the relative L2 change of the hidden state and the
+ * monotonic L clamp follow "CLI Reference", "generate" options
+ * --early-exit-patience / -min-L / -tau / -peek-every.
+ *
+ * Block (per layer): a = RMSNorm(x; g1); [q|k|v] = a Wqkv^T; RoPE(q, k, pos);
+ * o = causal softmax(q k^T / sqrt(hd)) v over the layer's cache slot;
+ * x += o Wo^T; b = RMSNorm(x; g2); x += (silu(b Wg^T) * (b Wu^T)) Wd^T.
+ * Head: logits = RMSNorm(h; g_final) Whead^T; greedy token = argmax (lowest id
+ * on ties).  RoPE pairs (i, i + hd/2) with angle pos * base^(-2i/hd).
+ *
+ * Conventions for every call:
+ *   - Return value: TL_OK (0) or a negative tl_status.  No call aborts, exits
+ *     or throws.  tl_strerror() names a status.
+ *   - Memory: the caller owns all memory.  Device memory comes from one
+ *     caller-allocated workspace of tl_workspace_bytes() bytes given to
+ *     tl_create(); pointers named dev_* are device pointers the caller owns;
+ *     host_* are host pointers, read or written before the call returns unless
+ *     stated otherwise.
+ *   - Streams: every device operation is enqueued on the stream given to
+ *     tl_create() (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream).  Device outputs are valid once the caller synchronises that
+ *     stream.
+ *   - Numbers: the residual stream, norms, softmax and every accumulation are
+ *     FP32; the K/V cache and tensor-core operands are FP16; INT4 weights are
+ *     dequantised exactly as (u - 8) * scale.
+ */
+#ifndef TL_H
+#define TL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tl_status {
+    TL_OK = 0,
+    TL_EINVAL = -1,    /* bad argument, shape or configuration */
+    TL_ENOMEM = -2,    /* workspace too small, or KV page pool exhausted */
+    TL_ESTATE = -3,    /* call not valid in the context's current state */
+    TL_EKV = -4,       /* a lane's L would rise above the depth its cache holds */
+    TL_ECUDA = -5,     /* a CUDA runtime call failed (see tl_last_cuda_error) */
+    TL_ETIMEOUT = -6,  /* a bounded device wait ran out */
+    TL_EDEVICE = -7    /* a kernel recorded an out-of-range index in the status word */
+} tl_status;
+
+typedef enum tl_weight_fmt {
+    TL_FMT_INT4 = 0,   /* packed nibbles u in [0,15], value (u - 8) * fp16 scale per group */
+    TL_FMT_BF16 = 1    /* bfloat16 bit patterns */
+} tl_weight_fmt;
+
+/* Model and capacity.  d = n_heads * head_dim, head_dim even. */
+typedef struct tl_config {
+    int32_t vocab;
+    int32_t d;
+    int32_t n_heads;
+    int32_t ffn;
+    int32_t n_pre;            /* pre blocks (own weights, own KV)                 */
+    int32_t n_loop_layers;    /* layers in the shared loop body                   */
+    int32_t fmt_pre;          /* tl_weight_fmt of pre-block matrices              */
+    int32_t fmt_loop;         /* tl_weight_fmt of loop-body matrices              */
+    int32_t fmt_embed_head;   /* tl_weight_fmt of embedding and head              */
+    int32_t group;            /* INT4 group size along K (multiple of 32)         */
+    float rms_eps;
+    float rope_base;
+    int32_t max_lanes;        /* lanes held at once                               */
+    int32_t max_seq;          /* prompt + generated tokens per lane               */
+    int32_t L_max;            /* largest per-lane loop count                      */
+    int32_t kv_page_tokens;   /* tokens per KV page (power of two, >= 16)         */
+    int32_t kv_pool_pages;    /* pages in the pool; 0 = one per lane/slot/page    */
+    int32_t max_prefill_tokens; /* rows of one prefill call; 0 = max_seq          */
+} tl_config;
+
+typedef struct tl_ctx tl_ctx;
+
+typedef struct tl_stats {
+    int64_t loop_steps;          /* loop steps run (tl_loop_step + inside tl_decode) */
+    int64_t lane_iterations;     /* sum over steps of lanes that ran an iteration */
+    int64_t tokens_emitted;      /* greedy tokens written by tl_decode/tl_generate */
+    int64_t prefill_tokens;      /* prompt positions run by tl_prefill          */
+    int64_t kernel_launches;     /* kernels this library launched               */
+    int32_t device_status;       /* last status word read back (0 = clean)      */
+    int32_t kv_pages_used;
+} tl_stats;
+
+/* ---------------------------------------------------------------- sizes -- */
+
+/* Bytes of device workspace tl_create() needs for cfg.  TL_EINVAL on a bad cfg. */
+int tl_workspace_bytes(const tl_config* cfg, size_t* out_bytes);
+
+/* Bytes of the weight blob for cfg (layout below).  Host-only; no CUDA call. */
+int tl_weights_bytes(const tl_config* cfg, size_t* out_bytes);
+
+/*
+ * Weight blob layout (little endian, no padding):
+ *   header: 8 bytes "TLWBLOB1", then the model fields of tl_config (vocab ..
+ *           rope_base: ten int32 then two float32, declaration order; 48 bytes);
+ *   matrices in this order: embed [V,d]; for each pre block then each loop
+ *   layer: wqkv [3d,d] (rows q|k|v), wo [d,d], wg [F,d], wu [F,d], wd [d,F];
+ *   head [V,d].  An INT4 matrix [N,K] is N*K/2 bytes of packed nibbles (row
+ *   major; element 2i in the low nibble of byte i, 2i+1 in the high nibble)
+ *   followed by N*(K/group) fp16 scales (row major).  A BF16 matrix is N*K
+ *   uint16 bit patterns (row major);
+ *   gains: for each pre block then loop layer g1[d], g2[d]; then g_final[d];
+ *   fp32.
+ * The INT4 convention (stored nibble u = code + 8, value (u - 8) * scale) is
+ * "Benchmark Comparison" (measured benchmarks) section 5's symmetric form; the
+ * nibble order is "CLI Reference", TINYLOOP_KV_INT4's.
+ */
+
+/* -------------------------------------------------------------- context -- */
+
+/* Carve the caller's workspace (>= tl_workspace_bytes, 256-byte aligned) and
+ * bind the stream.  The workspace must stay allocated until tl_destroy().
+ * Launches initialisation kernels (RoPE table, page table, lane state).
+ * TL_EINVAL bad cfg/pointer; TL_ENOMEM workspace too small; TL_ECUDA. */
+int tl_create(const tl_config* cfg, void* dev_workspace, size_t workspace_bytes,
+              void* cuda_stream, tl_ctx** out_ctx);
+
+/* Frees host-side state only (the workspace stays the caller's). */
+int tl_destroy(tl_ctx* ctx);
+
+/* Copy a weight blob (host memory, tl_weights_bytes(cfg) bytes, header must
+ * match cfg) into the workspace's device layout.  The caller keeps the host
+ * buffer.  Synchronous with respect to the host buffer.  TL_EINVAL on size,
+ * magic or config mismatch. */
+int tl_load_weights(tl_ctx* ctx, const void* host_blob, size_t bytes);
+
+/* ------------------------------------------------------ weight preparation -- */
+
+/* Symmetric per-group INT4 quantisation on the device ("Benchmark Comparison"
+ * (measured benchmarks), section 7: per-group min-max, no calibration):
+ * per row n and group j, scale = fp16_rne(max|w| / 7); code =
+ * clamp(rint(w / scale), -7, 7) with the division in fp64 at the fp16 scale's
+ * value (0 when scale is 0); stored nibble = code + 8.
+ * dev_w: fp64 [N, K] row major.  dev_packed: [N, K/2] bytes; dev_scales: fp16
+ * bits [N, K/group].  K % group == 0, group % 32 == 0.  Enqueued on
+ * cuda_stream.  TL_EINVAL on bad sizes. */
+int tl_quantize_int4(const double* dev_w, int64_t N, int64_t K, int32_t group,
+                     uint8_t* dev_packed, uint16_t* dev_scales, void* cuda_stream);
+
+/* Dequantise packed INT4 back to fp32 (exact): out[n,k] = (u - 8) * scale. */
+int tl_dequant_int4(const uint8_t* dev_packed, const uint16_t* dev_scales, int64_t N,
+                    int64_t K, int32_t group, float* dev_out, void* cuda_stream);
+
+/* Round fp64 to the nearest bfloat16 (ties to even); dev_out: bf16 bits [n]. */
+int tl_round_bf16(const double* dev_w, int64_t n, uint16_t* dev_out, void* cuda_stream);
+
+/* ------------------------------------------------------------ lanes -- */
+
+/* Run a lane's prompt ("CLI Reference", "benchmark": forward scoring over a
+ * token sequence at --loops L): embed, pre blocks, then L loop iterations over
+ * all T positions as one causal batch, filling the lane's K/V for the pre
+ * blocks and iterations 1..L.  The lane becomes ready for its first greedy
+ * token (tl_head_logits / tl_decode) with cap L.  Early exit does not apply to
+ * the prompt.
+ *   lane: 0..max_lanes-1 (any earlier content of the lane is dropped);
+ *   host_tokens: int32 [T], ids in [0, vocab); 1 <= T <= max_prefill_tokens;
+ *   L: 1..L_max;
+ *   share_prefix_from_lane: -1, or a lane whose prompt starts with the same
+ *     tokens and was prefilled at L' >= L; its full KV pages covering the first
+ *     shared_tokens positions are mapped (reference counted) instead of being
+ *     recomputed ("Benchmark Comparison" (measured benchmarks), section 2,
+ *     SHARED prefix reuse); shared_tokens is rounded down to whole pages;
+ *   dev_hidden_out: NULL or fp32 [T, d], the final hidden rows (before the
+ *     head norm).
+ * TL_EINVAL bad lane/T/L/token; TL_ENOMEM page pool exhausted. */
+int tl_prefill(tl_ctx* ctx, int32_t lane, const int32_t* host_tokens, int32_t T, int32_t L,
+               int32_t share_prefix_from_lane, int32_t shared_tokens, float* dev_hidden_out);
+
+/* Early-exit parameters for all lanes ("CLI Reference", generate options):
+ * probe at iteration l when l > min_L and (l - min_L - 1) % peek_every == 0;
+ * a probe with delta = ||h_l - h_{l-1}|| / ||h_{l-1}|| < tau extends the
+ * streak, any other probe resets it; exit once streak >= patience.
+ * tau <= 0 or patience == 0 disables it.  peek_every >= 1. */
+int tl_set_early_exit(tl_ctx* ctx, double tau, int32_t min_L, int32_t patience, int32_t peek_every);
+
+/* One loop step: every lane with dev_active_mask[lane] != 0 that is in its
+ * loop phase runs its next loop iteration (all body layers), at its own
+ * iteration index; then the device applies the early-exit rule.
+ *   dev_per_lane_L: NULL, or int32 [max_lanes] requested L per lane; a lane
+ *     whose request rose above the depth its cache holds sets TL_EKV in the
+ *     status word and does not run;
+ *   dev_active_mask: NULL (= all lanes) or uint8 [max_lanes];
+ *   dev_exit_mask_out: NULL or uint8 [max_lanes]: 1 where the lane's loop for
+ *     its current token finished in this step (early exit or L reached),
+ *     0 elsewhere.
+ * Device-side only: the host never waits. */
+int tl_loop_step(tl_ctx* ctx, const int32_t* dev_per_lane_L, const uint8_t* dev_active_mask,
+                 uint8_t* dev_exit_mask_out);
+
+/* Boundary stage, head: for lanes with dev_lane_mask[lane] != 0 (NULL = all
+ * lanes whose loop finished), final RMSNorm + head projection + greedy argmax.
+ *   dev_logits: NULL or fp32 [max_lanes, vocab] (rows of other lanes untouched);
+ *   dev_argmax: NULL or int32 [max_lanes]. */
+int tl_head_logits(tl_ctx* ctx, const uint8_t* dev_lane_mask, float* dev_logits, int32_t* dev_argmax);
+
+/* Boundary stage, token entry: for lanes with dev_lane_mask[lane] != 0, record
+ * that the lane's last loop ran to its finished depth (the lane's cap becomes
+ * that depth), advance its position, embed dev_tokens[lane] (int32
+ * [max_lanes]) and run the pre blocks, leaving the lane at the start of its
+ * loop.  Lets a caller drive decode with its own tokens (teacher forcing). */
+int tl_embed_next(tl_ctx* ctx, const uint8_t* dev_lane_mask, const int32_t* dev_tokens);
+
+/* Greedy continuous-depth decode of lanes 0..n_lanes-1, all prefilled.
+ * Emits n_new tokens per lane: the first from the lane's current hidden state
+ * (its prompt), each later one after a loop of min(L_requested, cap)
+ * iterations or fewer under early exit.  Steps run until every lane has
+ * emitted n_new tokens; lanes leave and re-enter the loop batch on the device.
+ *   host_per_lane_L: int32 [n_lanes] requested L (<= the prefill L);
+ *   dev_tokens_out / dev_depths_out: int32 [n_lanes, n_new] (NULL allowed):
+ *     the tokens and the iterations run behind each (the prefill L for the
+ *     first token).
+ * TL_EKV when a request exceeds the lane's cache depth. */
+int tl_decode(tl_ctx* ctx, const int32_t* host_per_lane_L, int32_t n_lanes, int32_t n_new,
+              int32_t* dev_tokens_out, int32_t* dev_depths_out);
+
+/* End to end from host memory ("Dynamic-L Inference", "L-Aware Batching":
+ * generate_batch(prompts, per_lane_loops)): copy prompts to the device,
+ * prefill every lane at its L, decode n_new tokens per lane, copy tokens and
+ * depths back.  host_prompts: int32 [n_lanes, T]; outputs int32 [n_lanes,
+ * n_new] in host memory (pinned memory makes the copies asynchronous-capable).
+ * Returns after the results are in host memory. */
+int tl_generate(tl_ctx* ctx, const int32_t* host_prompts, int32_t n_lanes, int32_t T,
+                const int32_t* host_per_lane_L, int32_t n_new, int32_t* host_tokens_out,
+                int32_t* host_depths_out);
+
+/* -------------------------------------------------------------- misc -- */
+
+/* Counters; also reads back and clears the device status word (synchronises
+ * the stream). */
+int tl_stats_get(tl_ctx* ctx, tl_stats* out);
+
+/* Name of a tl_status. */
+const char* tl_strerror(int status);
+
+/* The last CUDA error string recorded by this thread ("" if none). */
+const char* tl_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TL_H */

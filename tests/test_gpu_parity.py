@@ -1,0 +1,152 @@
+"""End-to-end parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Bars (floating point): logits max-abs <= 1e-2 and relative L2 <= 2e-3 per
+position, prompt hidden states relative L2 <= 2e-3.  Exact: per-lane depth
+schedules, exit masks, and greedy tokens wherever the oracle's top-1/top-2
+margin exceeds 1e-3."""
+import numpy as np
+import pytest
+
+import synthetic as S
+from oracle import decode as D
+from oracle import model as M
+
+from gpu_helpers import (assert_logits_close, gpu_model, oracle_weights, rel_l2, status_clean, teacher_forced,
+                         MARGIN)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_tokens(ref_tokens, ref_logits, got_tokens):
+    """Greedy tokens must agree wherever the oracle's margin exceeds 1e-3; after
+    the first near-tie the sequences may legitimately part."""
+    for t in range(len(ref_tokens)):
+        if M.top2_margin(ref_logits[t]) <= MARGIN:
+            return t
+        assert int(got_tokens[t]) == int(ref_tokens[t]), f"token {t}"
+    return len(ref_tokens)
+
+
+# --------------------------------------------------------------- tiny model ----
+
+@pytest.mark.parametrize("gain_seed", [None, 7])
+def test_tiny_generate_end_to_end(gain_seed):
+    wl = S.workload("tiny")
+    W = oracle_weights("tiny", gain_seed)
+    P = S.prompts(wl.n_lanes, wl.prompt_len, wl.shape.vocab)
+    m = gpu_model("tiny", gain_seed, max_lanes=2, max_seq=32, L_max=8)
+    tok, dep = m.generate(P, wl.per_lane_L, wl.n_new)
+    status_clean(m)
+    for i, L in enumerate(wl.per_lane_L):
+        r = D.generate_lane(W, P[i], L, wl.n_new)
+        assert dep[i].tolist() == [L] * wl.n_new
+        _check_tokens(r.tokens, r.logits, tok[i])
+
+
+def test_tiny_teacher_forced_logits():
+    wl = S.workload("tiny")
+    W = oracle_weights("tiny", 7)
+    P = S.prompts(wl.n_lanes, wl.prompt_len, wl.shape.vocab)
+    m = gpu_model("tiny", 7, max_lanes=2, max_seq=32, L_max=8)
+    ref, lg, am, dep = teacher_forced(m, W, P, list(wl.per_lane_L), wl.n_new)
+    status_clean(m)
+    for i in range(wl.n_lanes):
+        for t in range(wl.n_new):
+            assert_logits_close(lg[i, t], ref[i].logits[t], f"lane {i} token {t}")
+            if M.top2_margin(ref[i].logits[t]) > MARGIN:
+                assert am[i, t] == ref[i].tokens[t]
+        assert dep[i].tolist() == ref[i].depths.tolist()
+
+
+def test_tiny_single_lane_equals_batch():
+    # a lane's result does not depend on the other lanes in the step
+    wl = S.workload("tiny")
+    P = S.prompts(3, 12, wl.shape.vocab, seed=41)
+    Ls = [2, 5, 3]
+    m = gpu_model("tiny", None, max_lanes=3, max_seq=32, L_max=8)
+    tok_b, dep_b = m.generate(P, Ls, 6)
+    for i in range(3):
+        m1 = gpu_model("tiny", None, max_lanes=1, max_seq=32, L_max=8)
+        t1, d1 = m1.generate(P[i:i + 1], Ls[i:i + 1], 6)
+        assert np.array_equal(t1[0], tok_b[i]) and np.array_equal(d1[0], dep_b[i])
+
+
+def _probe_margins(ref, tau):
+    return [p.margin(tau) for r in ref for p in r.probes]
+
+
+@pytest.mark.parametrize("ee", [D.EarlyExit(0.9, 1, 2, 1), D.EarlyExit(0.33, 1, 1, 1), D.EarlyExit(0.5, 2, 1, 2),
+                                D.EarlyExit(1e9, 2, 2, 1)])
+def test_tiny_early_exit_schedules(ee):
+    W = oracle_weights("tiny")
+    P = S.prompts(3, 12, 512, seed=52)
+    Ls = [8, 5, 3]
+    ref = [D.generate_lane(W, P[i], Ls[i], 6, ee) for i in range(3)]
+    m = gpu_model("tiny", None, max_lanes=3, max_seq=32, L_max=8)
+    m.set_early_exit(ee.tau, ee.min_L, ee.patience, ee.peek_every)
+    tok, dep = m.generate(P, Ls, 6)
+    status_clean(m)
+    near = [x for x in _probe_margins(ref, ee.tau) if x <= 1e-2]
+    assert not near, f"probes within 1% of tau: {near}"
+    for i in range(3):
+        assert dep[i].tolist() == ref[i].depths.tolist(), i
+        _check_tokens(ref[i].tokens, ref[i].logits, tok[i])
+
+
+def test_tiny_exit_masks_per_step():
+    import torch
+    W = oracle_weights("tiny")
+    P = S.prompts(2, 10, 512, seed=52)
+    ee = D.EarlyExit(0.33, 1, 1, 1)
+    Ls = [8, 6]
+    ref, lg, am, dep = teacher_forced(gpu_model("tiny", None, max_lanes=2, max_seq=32, L_max=8), W, P, Ls, 5, ee)
+    for i in range(2):
+        assert dep[i].tolist() == ref[i].depths.tolist()
+        for t in range(5):
+            assert_logits_close(lg[i, t], ref[i].logits[t], f"lane {i} token {t}")
+
+
+def test_tiny_raising_L_is_refused():
+    from dynamic_depth_b200 import TlError
+    m = gpu_model("tiny", None, max_lanes=2, max_seq=32, L_max=8)
+    P = S.prompts(2, 8, 512, seed=3)
+    m.prefill(0, P[0], 3)
+    m.prefill(1, P[1], 3)
+    with pytest.raises(TlError) as e:
+        m.decode([3, 4], 2)
+    assert e.value.status == -4  # TL_EKV
+    with pytest.raises(TlError):
+        m.prefill(0, P[0], 0)
+    with pytest.raises(TlError):
+        m.prefill(0, np.array([600], dtype=np.int32), 2)  # token outside the vocabulary
+
+
+# ---------------------------------------------------------- 407M-class model ----
+
+def test_m407_prefill_hidden_T128_L8():
+    import torch
+    W = oracle_weights("m407")
+    wl = S.workload("m407_score")
+    P = S.prompts(1, wl.prompt_len, S.M407.vocab)
+    want, _ = M.forward(W, P[0], 8)
+    m = gpu_model("m407", None, max_lanes=1, max_seq=128, L_max=8)
+    hid = torch.zeros((128, S.M407.d), dtype=torch.float32, device="cuda")
+    m.prefill(0, P[0], 8, hidden_out=hid)
+    status_clean(m)
+    got = hid.cpu().numpy()
+    assert rel_l2(got, want) <= 2e-3
+    for t in (0, 1, 63, 127):
+        assert rel_l2(got[t], want[t]) <= 2e-3, t
+
+
+@pytest.mark.parametrize("L", [2, 32])
+def test_m407_decode_logits_teacher_forced(L):
+    W = oracle_weights("m407")
+    P = S.prompts(1, 32, S.M407.vocab)
+    m = gpu_model("m407", None, max_lanes=1, max_seq=40, L_max=32)
+    ref, lg, am, dep = teacher_forced(m, W, P, [L], 4)
+    status_clean(m)
+    for t in range(4):
+        assert_logits_close(lg[0, t], ref[0].logits[t], f"L={L} token {t}")
+        if M.top2_margin(ref[0].logits[t]) > MARGIN:
+            assert am[0, t] == ref[0].tokens[t]
