@@ -121,6 +121,27 @@ class LoopedLM:
               "tl_generate")
         return tok, dep
 
+    def lane_state_save(self):
+        """Snapshot of every lane's scheduling state and hidden row (a device tensor)."""
+        n = C.c_size_t()
+        check(lib().tl_lane_state_bytes(self.h, C.byref(n)), "tl_lane_state_bytes")
+        buf = self.torch.empty(n.value, dtype=self.torch.uint8, device=self.device)
+        check(lib().tl_lane_state_save(self.h, buf.data_ptr()), "tl_lane_state_save")
+        return buf
+
+    def lane_state_load(self, buf):
+        check(lib().tl_lane_state_load(self.h, buf.data_ptr()), "tl_lane_state_load")
+
+    def profile_begin(self, kind_mask: int):
+        """Time launch groups of the kinds in kind_mask (bit 1 attention, 2 projections, 3 head)."""
+        check(lib().tl_profile_begin(self.h, kind_mask), "tl_profile_begin")
+
+    def profile_end(self):
+        """(groups[4], ms[4]) indexed by kind."""
+        g, ms = (C.c_int64 * 4)(), (C.c_double * 4)()
+        check(lib().tl_profile_end(self.h, g, ms), "tl_profile_end")
+        return list(g), list(ms)
+
     def stats(self) -> dict:
         s = _lib.TlStats()
         check(lib().tl_stats_get(self.h, C.byref(s)), "tl_stats_get")

@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libtl.so")
 
 TL_OK, TL_EINVAL, TL_ENOMEM, TL_ESTATE, TL_EKV, TL_ECUDA, TL_ETIMEOUT, TL_EDEVICE = 0, -1, -2, -3, -4, -5, -6, -7
 TL_FMT_INT4, TL_FMT_BF16 = 0, 1
+TL_PROF_NONE, TL_PROF_ATTN, TL_PROF_PROJ, TL_PROF_HEAD = 0, 1, 2, 3
 
 
 class TlConfig(C.Structure):
@@ -53,6 +54,11 @@ SIGNATURES = {
     "tl_decode": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p]),
     "tl_generate": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_int32, C.c_void_p,
                               C.c_void_p]),
+    "tl_lane_state_bytes": (C.c_int, [C.c_void_p, C.POINTER(C.c_size_t)]),
+    "tl_lane_state_save": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "tl_lane_state_load": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "tl_profile_begin": (C.c_int, [C.c_void_p, C.c_int32]),
+    "tl_profile_end": (C.c_int, [C.c_void_p, C.POINTER(C.c_int64), C.POINTER(C.c_double)]),
     "tl_stats_get": (C.c_int, [C.c_void_p, C.POINTER(TlStats)]),
     "tl_strerror": (C.c_char_p, [C.c_int]),
     "tl_last_cuda_error": (C.c_char_p, []),

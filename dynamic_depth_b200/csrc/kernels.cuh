@@ -238,83 +238,104 @@ __device__ __forceinline__ void dot_chunk(const float* __restrict__ xs, int K, i
 }
 
 template <int FMT, int R, int EPI>
-__global__ void __launch_bounds__(GEMV_WARPS * 32)
-gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o) {
-  extern __shared__ float4 smem4[];
-  float* xs = reinterpret_cast<float*>(smem4);
-  __shared__ float best_v[GEMV_WARPS][R];
-  __shared__ int best_i[GEMV_WARPS][R];
+__device__ __forceinline__ void gemv_rows(const float* __restrict__ xs, int r0, int rows, const MatView& W,
+                                          const MatView& W2, const ProjOut& o, float (*best_v)[8],
+                                          int (*best_i)[8]) {
   const int K = W.K, N = W.N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * GEMV_WARPS + warp;
-  const int rows = n_rows[0];
   const int nch = K / 32;
-  for (int r0 = 0; r0 < rows; r0 += R) {
+  float acc[R], acc2[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = acc2[r] = 0.f;
+  if (n < N) {
+    for (int c = lane; c < nch; c += 32) {
+      float w[32], sc;
+      load_chunk<FMT>(W, n, c, w, sc);
+      dot_chunk<R>(xs, K, c, w, sc, acc);
+      if constexpr (EPI == EPI_SWIGLU) {
+        load_chunk<FMT>(W2, n, c, w, sc);
+        dot_chunk<R>(xs, K, c, w, sc, acc2);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    acc[r] = warp_sum(acc[r]);
+    if constexpr (EPI == EPI_SWIGLU) acc2[r] = warp_sum(acc2[r]);
+  }
+  if constexpr (EPI == EPI_ARGMAX) {
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        best_v[warp][r] = (n < N) ? acc[r] : -INFINITY;
+        best_i[warp][r] = (n < N) ? n : 0x7fffffff;
+      }
+    }
+    if (n < N && o.logits && lane < R && r0 + lane < rows) {
+      float v = acc[0];
+#pragma unroll
+      for (int r = 1; r < R; ++r) if (lane == r) v = acc[r];
+      o.logits[(int64_t)o.lmap[r0 + lane] * o.ldo + n] = v;
+    }
     __syncthreads();
-    for (int f = threadIdx.x; f < R * K / 4; f += blockDim.x) {
+    if (threadIdx.x < R && r0 + threadIdx.x < rows) {
+      const int r = threadIdx.x;
+      float bv = best_v[0][r];
+      int bi = best_i[0][r];
+      for (int ww = 1; ww < GEMV_WARPS; ++ww)
+        if (better(best_v[ww][r], best_i[ww][r], bv, bi)) { bv = best_v[ww][r]; bi = best_i[ww][r]; }
+      o.part_val[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bv;
+      o.part_idx[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bi;
+    }
+  } else if (n < N && lane < R && r0 + lane < rows) {
+    float v = acc[0], v2 = acc2[0];
+#pragma unroll
+    for (int r = 1; r < R; ++r)
+      if (lane == r) { v = acc[r]; v2 = acc2[r]; }
+    const int r = r0 + lane;
+    if constexpr (EPI == EPI_STORE) {
+      o.out[(int64_t)r * o.ldo + n] = v;
+    } else if constexpr (EPI == EPI_SWIGLU) {
+      o.out[(int64_t)r * o.ldo + n] = silu_f(v) * v2;
+    } else {
+      const int hr = o.map ? o.map[r] : r;
+      o.h[(int64_t)hr * N + n] += v;
+    }
+  }
+}
+
+// Rows are taken 8 at a time (fewer for the last chunk, dispatched to a body
+// compiled for that count).  With skip_above > 0 the kernel does nothing when
+// the row count exceeds it (the tiled GEMM launched beside it takes those).
+template <int FMT, int EPI>
+__global__ void __launch_bounds__(GEMV_WARPS * 32)
+gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
+            int skip_above) {
+  extern __shared__ float4 smem4[];
+  float* xs = reinterpret_cast<float*>(smem4);
+  __shared__ float best_v[GEMV_WARPS][8];
+  __shared__ int best_i[GEMV_WARPS][8];
+  const int K = W.K;
+  const int rows = n_rows[0];
+  if (skip_above > 0 && rows > skip_above) return;
+  for (int r0 = 0; r0 < rows; r0 += 8) {
+    const int nr = min(8, rows - r0);
+    __syncthreads();
+    for (int f = threadIdx.x; f < nr * K / 4; f += blockDim.x) {
       const int r = f / (K / 4), fi = f % (K / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r0 + r < rows) v = reinterpret_cast<const float4*>(X + (int64_t)(r0 + r) * K)[fi];
-      smem4[r * (K / 4) + swz_slot(fi)] = v;
+      smem4[r * (K / 4) + swz_slot(fi)] = reinterpret_cast<const float4*>(X + (int64_t)(r0 + r) * K)[fi];
     }
     __syncthreads();
-    float acc[R], acc2[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = acc2[r] = 0.f;
-    if (n < N) {
-      for (int c = lane; c < nch; c += 32) {
-        float w[32], sc;
-        load_chunk<FMT>(W, n, c, w, sc);
-        dot_chunk<R>(xs, K, c, w, sc, acc);
-        if constexpr (EPI == EPI_SWIGLU) {
-          load_chunk<FMT>(W2, n, c, w, sc);
-          dot_chunk<R>(xs, K, c, w, sc, acc2);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      acc[r] = warp_sum(acc[r]);
-      if constexpr (EPI == EPI_SWIGLU) acc2[r] = warp_sum(acc2[r]);
-    }
-    if constexpr (EPI == EPI_ARGMAX) {
-      if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          best_v[warp][r] = (n < N) ? acc[r] : -INFINITY;
-          best_i[warp][r] = (n < N) ? n : 0x7fffffff;
-        }
-      }
-      if (n < N && o.logits && lane < R && r0 + lane < rows) {
-        float v = acc[0];
-#pragma unroll
-        for (int r = 1; r < R; ++r) if (lane == r) v = acc[r];
-        o.logits[(int64_t)o.lmap[r0 + lane] * o.ldo + n] = v;
-      }
-      __syncthreads();
-      if (threadIdx.x < R && r0 + threadIdx.x < rows) {
-        const int r = threadIdx.x;
-        float bv = best_v[0][r];
-        int bi = best_i[0][r];
-        for (int ww = 1; ww < GEMV_WARPS; ++ww)
-          if (better(best_v[ww][r], best_i[ww][r], bv, bi)) { bv = best_v[ww][r]; bi = best_i[ww][r]; }
-        o.part_val[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bv;
-        o.part_idx[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bi;
-      }
-    } else if (n < N && lane < R && r0 + lane < rows) {
-      float v = acc[0], v2 = acc2[0];
-#pragma unroll
-      for (int r = 1; r < R; ++r)
-        if (lane == r) { v = acc[r]; v2 = acc2[r]; }
-      const int r = r0 + lane;
-      if constexpr (EPI == EPI_STORE) {
-        o.out[(int64_t)r * o.ldo + n] = v;
-      } else if constexpr (EPI == EPI_SWIGLU) {
-        o.out[(int64_t)r * o.ldo + n] = silu_f(v) * v2;
-      } else {
-        const int hr = o.map ? o.map[r] : r;
-        o.h[(int64_t)hr * N + n] += v;
-      }
+    switch (nr) {
+      case 1: gemv_rows<FMT, 1, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 2: gemv_rows<FMT, 2, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 3: gemv_rows<FMT, 3, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 4: gemv_rows<FMT, 4, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 5: gemv_rows<FMT, 5, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 6: gemv_rows<FMT, 6, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 7: gemv_rows<FMT, 7, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      default: gemv_rows<FMT, 8, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
     }
   }
 }
@@ -358,13 +379,14 @@ __device__ __forceinline__ void load_w_tile(const MatView& W, int n0, int k0, fl
 
 template <int FMT, int EPI>
 __global__ void __launch_bounds__(256)
-gemm_simt_kernel(const float* __restrict__ A, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o) {
+gemm_simt_kernel(const float* __restrict__ A, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
+                 int skip_at_or_below) {
   __shared__ float As[SG_BK][SG_BM + 4];
   __shared__ float Ws[SG_BK][SG_BN + 4];
   __shared__ float Ws2[(EPI == EPI_SWIGLU) ? SG_BK : 1][SG_BN + 4];
   const int M = n_rows[0];
   const int m0 = blockIdx.y * SG_BM, n0 = blockIdx.x * SG_BN;
-  if (m0 >= M) return;
+  if (m0 >= M || M <= skip_at_or_below) return;
   const int K = W.K, N = W.N;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4] = {}, acc2[4][4] = {};
@@ -569,6 +591,148 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows
     float v = 0.f;
     for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
     o[(int64_t)r * d + h * HD + i] = v / Lsum;
+  }
+}
+
+// --------------------------------------------------- prefill attention ----
+//
+// Causal attention for a block of consecutive prompt rows of one lane: CTA
+// (qb, h) takes query rows r in [64 qb, 64 qb + 64) (positions rows.pos[r],
+// consecutive) and walks key blocks of 64 positions from 0 up to its last
+// query position, staging K and V once per block in shared memory (fp32) and
+// keeping a running max / sum per query row.  256 threads: for the scores
+// thread (ty, tx) owns rows 4ty..4ty+3 and keys 4tx..4tx+3; for the output it
+// owns the same rows and dims tx*HD/16 .. +HD/16.
+template <int HD>
+__global__ void __launch_bounds__(256)
+attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows, KVGeom g, int slot,
+                    int32_t* __restrict__ status) {
+  constexpr int BQ = 64, BK = 64, DPT = HD / 16;
+  extern __shared__ float4 smem_pf[];
+  float* Qs = reinterpret_cast<float*>(smem_pf);  // [HD][BQ]  (pre-scaled)
+  float* Ks = Qs + HD * BQ;                        // [HD][BK]
+  float* Vs = Ks + HD * BK;                        // [BK][HD]
+  float* Ps = Vs + BK * HD;                        // [BQ][BK + 1]
+  const int n = rows.n[0];
+  const int r0 = blockIdx.x * BQ, h = blockIdx.y;
+  if (r0 >= n) return;
+  const int ln = rows.lane[r0];
+  const int d = g.H * HD;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int nq = min(BQ, n - r0);
+  const int pos_first = rows.pos[r0];
+  const int pos_last = pos_first + nq - 1;
+  const float scale = rsqrtf((float)HD);
+  for (int i = threadIdx.x; i < BQ * HD; i += 256) {
+    const int r = i / HD, dd = i % HD;
+    Qs[dd * BQ + r] = (r < nq) ? q[(int64_t)(r0 + r) * d + h * HD + dd] * scale : 0.f;
+  }
+  float m[4], l[4], acc[4][DPT];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < DPT; ++j) acc[i][j] = 0.f;
+  }
+  const int nkb = pos_last / BK + 1;
+  for (int kb = 0; kb < nkb; ++kb) {
+    const int k0 = kb * BK;
+    __syncthreads();
+    // stage K (transposed) and V for key positions k0 .. k0+63 (<= pos_last)
+    for (int i = threadIdx.x; i < BK * (HD / 8); i += 256) {
+      const int kr = i / (HD / 8), c8 = i % (HD / 8);
+      const int kp = k0 + kr;
+      float kv[8], vv[8];
+      const __half* kptr = (kp <= pos_last) ? kv_k_ptr(g, ln, slot, kp, h, status) : nullptr;
+      if (kptr) {
+        const uint4 ku = *reinterpret_cast<const uint4*>(kptr + c8 * 8);
+        const uint4 vu = *reinterpret_cast<const uint4*>(kptr + (int64_t)g.H * g.page_tokens * HD + c8 * 8);
+        const __half2* kh = reinterpret_cast<const __half2*>(&ku);
+        const __half2* vh = reinterpret_cast<const __half2*>(&vu);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 a = __half22float2(kh[e]), b = __half22float2(vh[e]);
+          kv[2 * e] = a.x; kv[2 * e + 1] = a.y; vv[2 * e] = b.x; vv[2 * e + 1] = b.y;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kv[e] = vv[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        Ks[(c8 * 8 + e) * BK + kr] = kv[e];
+        Vs[kr * HD + c8 * 8 + e] = vv[e];
+      }
+    }
+    __syncthreads();
+    // scores
+    float sc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sc[i][j] = 0.f;
+#pragma unroll 8
+    for (int dd = 0; dd < HD; ++dd) {
+      const float4 a = *reinterpret_cast<const float4*>(&Qs[dd * BQ + ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Ks[dd * BK + tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc[i][j] = fmaf(av[i], bv[j], sc[i][j]);
+    }
+    // causal mask, online softmax per row (the 16 threads of a row group share it)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int qp = pos_first + ty * 4 + i;
+      float mb = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int kp = k0 + tx * 4 + j;
+        if (kp > qp) sc[i][j] = -INFINITY;
+        mb = fmaxf(mb, sc[i][j]);
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+      const float mn = fmaxf(m[i], mb);
+      float ps = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float pv = (sc[i][j] == -INFINITY) ? 0.f : expf(sc[i][j] - mn);
+        Ps[(ty * 4 + i) * (BK + 1) + tx * 4 + j] = pv;
+        ps += pv;
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      const float corr = (m[i] == -INFINITY) ? 0.f : expf(m[i] - mn);
+      l[i] = l[i] * corr + ps;
+      m[i] = mn;
+#pragma unroll
+      for (int j = 0; j < DPT; ++j) acc[i][j] *= corr;
+    }
+    __syncthreads();
+    // output: acc[r][dims] += P[r][k] V[k][dims]
+#pragma unroll 4
+    for (int k = 0; k < BK; ++k) {
+      float vv[DPT];
+#pragma unroll
+      for (int j = 0; j < DPT; ++j) vv[j] = Vs[k * HD + tx * DPT + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float pk = Ps[(ty * 4 + i) * (BK + 1) + k];
+#pragma unroll
+        for (int j = 0; j < DPT; ++j) acc[i][j] = fmaf(pk, vv[j], acc[i][j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty * 4 + i;
+    if (r >= nq) continue;
+    const float inv = 1.f / l[i];
+#pragma unroll
+    for (int j = 0; j < DPT; ++j) o[(int64_t)(r0 + r) * d + h * HD + tx * DPT + j] = acc[i][j] * inv;
   }
 }
 

@@ -4,6 +4,7 @@
 // waits are the lagged "lanes still alive" polls of tl_decode and the explicit
 // synchronisations of tl_generate / tl_stats_get.
 #include <cstdio>
+#include <array>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -176,9 +177,16 @@ struct tl_ctx {
   int32_t* pinned_alive = nullptr;    // ring of alive counts
   cudaEvent_t alive_ev[4];
   int64_t steps = 0, prefill_tokens = 0, launches = 0;
+  // profiling ring (tl_profile_begin / tl_profile_end)
+  int prof_mask = 0;
+  std::vector<std::array<cudaEvent_t, 2>> prof_ev;
+  std::vector<int> prof_kind_of;
+  int64_t prof_head = 0, prof_tail = 0, prof_groups[4] = {0, 0, 0, 0};
+  double prof_ms[4] = {0, 0, 0, 0};
 };
 
 static constexpr int kAliveRing = 4;
+static constexpr int kProfRing = 4096;
 
 namespace {
 
@@ -189,11 +197,42 @@ int launch_err(tl_ctx* c) {
   return check_cuda(cudaGetLastError());
 }
 
-template <int FMT, int R, int EPI>
+// Per-kind device time: event pairs around every launch group of a profiled
+// kind, kept in a ring; the host folds in the oldest pair only when the ring is
+// full, so timing adds no wait until thousands of groups are in flight.
+int prof_fold_oldest(tl_ctx* c) {
+  const int i = (int)(c->prof_tail % kProfRing);
+  TL_CUDA(cudaEventSynchronize(c->prof_ev[i][1]));
+  float ms = 0.f;
+  TL_CUDA(cudaEventElapsedTime(&ms, c->prof_ev[i][0], c->prof_ev[i][1]));
+  c->prof_ms[c->prof_kind_of[i]] += ms;
+  c->prof_tail++;
+  return TL_OK;
+}
+
+bool prof_on(tl_ctx* c, int kind) { return kind > 0 && kind < 4 && ((c->prof_mask >> kind) & 1); }
+
+int prof_start(tl_ctx* c, int kind) {
+  if (!prof_on(c, kind)) return TL_OK;
+  if (c->prof_head - c->prof_tail == kProfRing) TL_TRY(prof_fold_oldest(c));
+  const int i = (int)(c->prof_head % kProfRing);
+  c->prof_kind_of[i] = kind;
+  return check_cuda(cudaEventRecord(c->prof_ev[i][0], c->stream));
+}
+
+int prof_stop(tl_ctx* c, int kind) {
+  if (!prof_on(c, kind)) return TL_OK;
+  TL_CUDA(cudaEventRecord(c->prof_ev[c->prof_head % kProfRing][1], c->stream));
+  c->prof_head++;
+  c->prof_groups[kind]++;
+  return TL_OK;
+}
+
+template <int FMT, int EPI>
 int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView& W, const MatView& W2,
-                const ProjOut& o) {
-  const size_t smem = (size_t)R * W.K * 4;
-  auto kern = gemv_kernel<FMT, R, EPI>;
+                const ProjOut& o, int skip_above) {
+  const size_t smem = (size_t)8 * W.K * 4;
+  auto kern = gemv_kernel<FMT, EPI>;
   static bool attr_done = false;  // once per instantiation
   if (!attr_done) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
@@ -201,67 +240,97 @@ int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView&
   }
   if (smem > 200 * 1024) return TL_EINVAL;
   const unsigned grid = (unsigned)((W.N + GEMV_WARPS - 1) / GEMV_WARPS);
-  kern<<<grid, GEMV_WARPS * 32, smem, c->stream>>>(X, n_rows, W, W2, o);
+  kern<<<grid, GEMV_WARPS * 32, smem, c->stream>>>(X, n_rows, W, W2, o, skip_above);
   return launch_err(c);
 }
 
 template <int FMT, int EPI>
-int gemv_pick_r(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView& W2,
-                const ProjOut& o) {
-  if (max_rows <= 1) return gemv_launch<FMT, 1, EPI>(c, X, n, W, W2, o);
-  if (max_rows <= 2) return gemv_launch<FMT, 2, EPI>(c, X, n, W, W2, o);
-  if (max_rows <= 4) return gemv_launch<FMT, 4, EPI>(c, X, n, W, W2, o);
-  return gemv_launch<FMT, 8, EPI>(c, X, n, W, W2, o);
-}
-
-template <int FMT, int EPI>
 int gemm_launch(tl_ctx* c, int max_rows, const float* A, const int32_t* n, const MatView& W, const MatView& W2,
-                const ProjOut& o) {
+                const ProjOut& o, int skip_at_or_below) {
   dim3 grid((W.N + SG_BN - 1) / SG_BN, (max_rows + SG_BM - 1) / SG_BM);
-  gemm_simt_kernel<FMT, EPI><<<grid, 256, 0, c->stream>>>(A, n, W, W2, o);
+  gemm_simt_kernel<FMT, EPI><<<grid, 256, 0, c->stream>>>(A, n, W, W2, o, skip_at_or_below);
   return launch_err(c);
 }
 
 constexpr int kGemvMaxRows = 8;
 
+// Projection over the device-side row count: the GEMV takes up to 8 rows; when
+// more rows are possible a tiled GEMM is launched beside it and exactly one of
+// the two does the work.  The head (EPI_ARGMAX) always uses the GEMV, which
+// loops over its rows 8 at a time, so its partial-result count is fixed.
 template <int EPI>
 int proj_epi(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView& W2,
              ProjOut o) {
-  const bool gemv = max_rows <= kGemvMaxRows;
-  if (EPI == EPI_ARGMAX)
-    o.n_parts = gemv ? (W.N + GEMV_WARPS - 1) / GEMV_WARPS : (W.N + SG_BN - 1) / SG_BN;
-  if (W.fmt == TL_FMT_INT4)
-    return gemv ? gemv_pick_r<TL_FMT_INT4, EPI>(c, max_rows, X, n, W, W2, o)
-                : gemm_launch<TL_FMT_INT4, EPI>(c, max_rows, X, n, W, W2, o);
-  return gemv ? gemv_pick_r<TL_FMT_BF16, EPI>(c, max_rows, X, n, W, W2, o)
-              : gemm_launch<TL_FMT_BF16, EPI>(c, max_rows, X, n, W, W2, o);
+  const bool gemv_only = EPI == EPI_ARGMAX || max_rows <= kGemvMaxRows;
+  if (EPI == EPI_ARGMAX) o.n_parts = (W.N + GEMV_WARPS - 1) / GEMV_WARPS;
+  if (W.fmt == TL_FMT_INT4) {
+    TL_TRY((gemv_launch<TL_FMT_INT4, EPI>(c, X, n, W, W2, o, gemv_only ? 0 : kGemvMaxRows)));
+    if (!gemv_only) TL_TRY((gemm_launch<TL_FMT_INT4, EPI>(c, max_rows, X, n, W, W2, o, kGemvMaxRows)));
+  } else {
+    TL_TRY((gemv_launch<TL_FMT_BF16, EPI>(c, X, n, W, W2, o, gemv_only ? 0 : kGemvMaxRows)));
+    if (!gemv_only) TL_TRY((gemm_launch<TL_FMT_BF16, EPI>(c, max_rows, X, n, W, W2, o, kGemvMaxRows)));
+  }
+  return TL_OK;
 }
 
 int proj(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView* W2,
-         const ProjOut& o) {
+         const ProjOut& o, int prof_kind = TL_PROF_PROJ) {
   const MatView& w2 = W2 ? *W2 : W;
+  TL_TRY(prof_start(c, prof_kind));
+  int st;
   switch (o.epi) {
-    case EPI_STORE: return proj_epi<EPI_STORE>(c, max_rows, X, n, W, w2, o);
-    case EPI_RESID: return proj_epi<EPI_RESID>(c, max_rows, X, n, W, w2, o);
-    case EPI_SWIGLU: return proj_epi<EPI_SWIGLU>(c, max_rows, X, n, W, w2, o);
-    default: return proj_epi<EPI_ARGMAX>(c, max_rows, X, n, W, w2, o);
+    case EPI_STORE: st = proj_epi<EPI_STORE>(c, max_rows, X, n, W, w2, o); break;
+    case EPI_RESID: st = proj_epi<EPI_RESID>(c, max_rows, X, n, W, w2, o); break;
+    case EPI_SWIGLU: st = proj_epi<EPI_SWIGLU>(c, max_rows, X, n, W, w2, o); break;
+    default: st = proj_epi<EPI_ARGMAX>(c, max_rows, X, n, W, w2, o); break;
   }
+  TL_TRY(st);
+  return prof_stop(c, prof_kind);
 }
 
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
+  TL_TRY(prof_start(c, TL_PROF_ATTN));
   dim3 grid(max_rows, c->cfg.n_heads);
   switch (c->hd) {
     case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
     case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
     default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
   }
+  TL_TRY(launch_err(c));
+  return prof_stop(c, TL_PROF_ATTN);
+}
+
+// Causal attention over a prompt block (rows of one lane, consecutive positions).
+template <int HD>
+int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
+  const size_t smem = (size_t)(3 * HD * 64 + 64 * 65) * 4;
+  static bool attr_done = false;
+  if (!attr_done) {
+    TL_CUDA(cudaFuncSetAttribute(attn_prefill_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr_done = true;
+  }
+  dim3 grid((max_rows + 63) / 64, c->cfg.n_heads);
+  attn_prefill_kernel<HD><<<grid, 256, smem, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot, c->status);
   return launch_err(c);
+}
+
+int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
+  TL_TRY(prof_start(c, TL_PROF_ATTN));
+  int st;
+  switch (c->hd) {
+    case 32: st = attn_prefill_launch_hd<32>(c, max_rows, rows, slot); break;
+    case 64: st = attn_prefill_launch_hd<64>(c, max_rows, rows, slot); break;
+    default: st = attn_prefill_launch_hd<128>(c, max_rows, rows, slot); break;
+  }
+  TL_TRY(st);
+  return prof_stop(c, TL_PROF_ATTN);
 }
 
 // One transformer block on the rows of `rows`; hidden rows live in hbuf
 // (indexed through map, or by row when map is null).
+// prompt = rows are consecutive positions of one lane (tiled causal attention).
 int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int32_t* map, const BlockW& w,
-              int slot_base, int slot_stride, float* h_in) {
+              int slot_base, int slot_stride, float* h_in, bool prompt = false) {
   const int d = c->cfg.d, F = c->cfg.ffn;
   const float eps = c->cfg.rms_eps;
   rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in);
@@ -274,7 +343,10 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   rope_kv_kernel<<<max_rows, d / 2, 0, c->stream>>>(c->act_qkv, c->act_q, rows, c->kv, c->rope, slot_base,
                                                      slot_stride, nullptr, c->status);
   TL_TRY(launch_err(c));
-  TL_TRY(attn_launch(c, max_rows, rows, slot_base, slot_stride));
+  if (prompt)
+    TL_TRY(attn_prefill_launch(c, max_rows, rows, slot_base));
+  else
+    TL_TRY(attn_launch(c, max_rows, rows, slot_base, slot_stride));
   ProjOut r{};
   r.epi = EPI_RESID;
   r.h = hbuf;
@@ -334,7 +406,7 @@ int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax
   o.ldo = c->cfg.vocab;
   o.part_val = c->part_val;
   o.part_idx = c->part_idx;
-  TL_TRY(proj(c, max_rows, c->act_a, B.n, c->head, nullptr, o));
+  TL_TRY(proj(c, max_rows, c->act_a, B.n, c->head, nullptr, o, TL_PROF_HEAD));
   const int n_parts = max_rows <= kGemvMaxRows ? (c->cfg.vocab + GEMV_WARPS - 1) / GEMV_WARPS
                                                : (c->cfg.vocab + SG_BN - 1) / SG_BN;
   head_finalize_kernel<<<max_rows, 256, 0, c->stream>>>(B, c->lanes, c->part_val, c->part_idx, n_parts, mode, argmax,
@@ -528,6 +600,10 @@ extern "C" int tl_destroy(tl_ctx* c) {
   if (!c) return TL_EINVAL;
   cudaStreamSynchronize(c->stream);
   for (int i = 0; i < kAliveRing; ++i) cudaEventDestroy(c->alive_ev[i]);
+  for (auto& e : c->prof_ev) {
+    cudaEventDestroy(e[0]);
+    cudaEventDestroy(e[1]);
+  }
   if (c->pinned_alive) cudaFreeHost(c->pinned_alive);
   delete c;
   return TL_OK;
@@ -619,10 +695,10 @@ extern "C" int tl_prefill(tl_ctx* c, int32_t lane, const int32_t* host_tokens, i
   TL_TRY(launch_err(c));
   embed_rows_kernel<<<Tn, 256, 0, c->stream>>>(c->embed, c->tok_stage, Tn, cfg.d, c->hrows, c->status);
   TL_TRY(launch_err(c));
-  for (int b = 0; b < P; ++b) TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->pre[b], b, 0, nullptr));
+  for (int b = 0; b < P; ++b) TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->pre[b], b, 0, nullptr, true));
   for (int l = 0; l < L; ++l)
     for (int m = 0; m < Lb; ++m)
-      TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr));
+      TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr, true));
   prefill_finish_kernel<<<1, 256, 0, c->stream>>>(c->lanes, lane, Tn, T - 1, L, c->hrows, c->h, cfg.d);
   TL_TRY(launch_err(c));
   if (dev_hidden_out)
@@ -725,5 +801,57 @@ extern "C" int tl_stats_get(tl_ctx* c, tl_stats* out) {
   out->kernel_launches = c->launches;
   out->device_status = st;
   out->kv_pages_used = c->lay.n_pages - (int32_t)c->free_pages.size();
+  return TL_OK;
+}
+
+extern "C" int tl_lane_state_bytes(tl_ctx* c, size_t* out) {
+  if (!c || !out) return TL_EINVAL;
+  *out = (size_t)c->cfg.max_lanes * (sizeof(LaneState) + (size_t)c->cfg.d * 4);
+  return TL_OK;
+}
+
+extern "C" int tl_lane_state_save(tl_ctx* c, void* dev_dst) {
+  if (!c || !dev_dst) return TL_EINVAL;
+  const size_t a = (size_t)c->cfg.max_lanes * sizeof(LaneState), b = (size_t)c->cfg.max_lanes * c->cfg.d * 4;
+  TL_CUDA(cudaMemcpyAsync(dev_dst, c->lanes, a, cudaMemcpyDeviceToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync((char*)dev_dst + a, c->h, b, cudaMemcpyDeviceToDevice, c->stream));
+  return TL_OK;
+}
+
+extern "C" int tl_lane_state_load(tl_ctx* c, const void* dev_src) {
+  if (!c || !dev_src) return TL_EINVAL;
+  const size_t a = (size_t)c->cfg.max_lanes * sizeof(LaneState), b = (size_t)c->cfg.max_lanes * c->cfg.d * 4;
+  TL_CUDA(cudaMemcpyAsync(c->lanes, dev_src, a, cudaMemcpyDeviceToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->h, (const char*)dev_src + a, b, cudaMemcpyDeviceToDevice, c->stream));
+  return TL_OK;
+}
+
+extern "C" int tl_profile_begin(tl_ctx* c, int32_t kind_mask) {
+  if (!c || (kind_mask & ~0xE)) return TL_EINVAL;
+  if (c->prof_ev.empty()) {
+    c->prof_ev.resize(kProfRing);
+    c->prof_kind_of.assign(kProfRing, 0);
+    for (auto& e : c->prof_ev) {
+      TL_CUDA(cudaEventCreate(&e[0]));
+      TL_CUDA(cudaEventCreate(&e[1]));
+    }
+  }
+  c->prof_mask = kind_mask;
+  c->prof_head = c->prof_tail = 0;
+  for (int k = 0; k < 4; ++k) {
+    c->prof_groups[k] = 0;
+    c->prof_ms[k] = 0.0;
+  }
+  return TL_OK;
+}
+
+extern "C" int tl_profile_end(tl_ctx* c, int64_t* groups, double* total_ms) {
+  if (!c) return TL_EINVAL;
+  while (c->prof_tail < c->prof_head) TL_TRY(prof_fold_oldest(c));
+  for (int k = 0; k < 4; ++k) {
+    if (groups) groups[k] = c->prof_groups[k];
+    if (total_ms) total_ms[k] = c->prof_ms[k];
+  }
+  c->prof_mask = 0;
   return TL_OK;
 }

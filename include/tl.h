@@ -241,6 +241,42 @@ int tl_generate(tl_ctx* ctx, const int32_t* host_prompts, int32_t n_lanes, int32
                 const int32_t* host_per_lane_L, int32_t n_new, int32_t* host_tokens_out,
                 int32_t* host_depths_out);
 
+/* ------------------------------------------------- lane-state checkpoint -- */
+
+/* Bytes of a lane-state snapshot: the scheduling state and the fp32 hidden row
+ * of every lane (max_lanes * (48 + 4 d)).  The KV cache is not part of it: a
+ * decode started from a restored snapshot rewrites every position past the
+ * saved ones before reading it, and positions at or before them are never
+ * written by decode. */
+int tl_lane_state_bytes(tl_ctx* ctx, size_t* out_bytes);
+
+/* Copy the lane states into dev_dst (device, tl_lane_state_bytes bytes),
+ * enqueued on the context's stream. */
+int tl_lane_state_save(tl_ctx* ctx, void* dev_dst);
+
+/* Restore lane states saved by tl_lane_state_save on this context. */
+int tl_lane_state_load(tl_ctx* ctx, const void* dev_src);
+
+/* ------------------------------------------------------------ profiling -- */
+
+typedef enum tl_prof_kind {
+    TL_PROF_NONE = 0,
+    TL_PROF_ATTN = 1,   /* per-iteration attention launches                  */
+    TL_PROF_PROJ = 2,   /* block projections (QKV, O, gate/up, down)         */
+    TL_PROF_HEAD = 3    /* head projection + argmax partials                 */
+} tl_prof_kind;
+
+/* Time every launch group of the kinds in kind_mask (bit k = tl_prof_kind k)
+ * with CUDA events on the context's stream until tl_profile_end.  A group is
+ * one attention launch, or the one or two kernels of one projection.  Cost:
+ * two event records per group; the host waits only when 4096 groups are
+ * outstanding.  TL_EINVAL for bits outside kinds 1..3. */
+int tl_profile_begin(tl_ctx* ctx, int32_t kind_mask);
+
+/* Stop timing.  out_groups / out_total_ms (nullable) receive 4 entries indexed
+ * by tl_prof_kind: groups timed and their summed device time in ms. */
+int tl_profile_end(tl_ctx* ctx, int64_t* out_groups, double* out_total_ms);
+
 /* -------------------------------------------------------------- misc -- */
 
 /* Counters; also reads back and clears the device status word (synchronises
