@@ -122,6 +122,11 @@ __device__ __forceinline__ float nib_to_f(uint32_t w, int sh) {
 
 __device__ __forceinline__ float bf16_bits_to_f(uint32_t b) { return __uint_as_float(b << 16); }
 
+// Nibble holding element e (0..7) of an 8-element word in the device INT4
+// layout: element 2i in nibble i, element 2i+1 in nibble i + 4 (the loader
+// repacks the blob's plain order into this one).
+__device__ __forceinline__ constexpr int nib_pos(int e) { return (e & 1) ? (e >> 1) + 4 : (e >> 1); }
+
 __device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
 
 // Address of (slot, lane, pos) K row for head h; V follows at + H*P*hd.

@@ -129,11 +129,13 @@ __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, in
 
 // --------------------------------------------------------------- norms ----
 
-// out[r] = RMSNorm(h[map ? map[r] : r]) * g, fp32.  One CTA per row.  When
-// h_in is given, also copies the source row there (indexed like h).
+// out[r] = RMSNorm(h[map ? map[r] : r]) * g, fp32 (and an fp16 copy for the
+// tensor-core projections when out16 is given).  One CTA per row.  When h_in is
+// given, also copies the source row there (indexed like h).
 __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* __restrict__ map,
                                     const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
-                                    float eps, float* __restrict__ out, float* __restrict__ h_in) {
+                                    float eps, float* __restrict__ out, float* __restrict__ h_in,
+                                    __half* __restrict__ out16) {
   __shared__ float red[32];
   const int r = blockIdx.x;
   if (r >= n_rows[0]) return;
@@ -145,7 +147,9 @@ __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* 
   const float inv = rsqrtf(ss / (float)d + eps);
   for (int k = threadIdx.x; k < d; k += blockDim.x) {
     const float v = x[k];
-    out[(int64_t)r * d + k] = v * inv * g[k];
+    const float y = v * inv * g[k];
+    out[(int64_t)r * d + k] = y;
+    if (out16) out16[(int64_t)r * d + k] = __float2half_rn(y);
     if (h_in) h_in[(int64_t)src * d + k] = v;
   }
 }
@@ -155,13 +159,13 @@ __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* 
 // h[dst] = dequantised embedding row of token; one CTA per row.
 __device__ __forceinline__ void embed_row(const MatView& E, int tok, float* __restrict__ dst, int d) {
   if (E.fmt == TL_FMT_INT4) {
-    const uint8_t* q = E.q + (int64_t)tok * (d / 2);
+    const uint32_t* q = reinterpret_cast<const uint32_t*>(E.q + (int64_t)tok * (d / 2));
     const __half* s = E.s + (int64_t)tok * (d / E.group);
-    for (int k = 2 * threadIdx.x; k < d; k += 2 * blockDim.x) {
-      const uint32_t b = q[k / 2];
-      const float sc = __half2float(s[k / E.group]);
-      dst[k] = nib_to_f(b, 0) * sc;
-      dst[k + 1] = nib_to_f(b, 4) * sc;
+    for (int wi = threadIdx.x; wi < d / 8; wi += blockDim.x) {
+      const uint32_t w = q[wi];
+      const float sc = __half2float(s[(8 * wi) / E.group]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dst[8 * wi + e] = nib_to_f(w, 4 * nib_pos(e)) * sc;
     }
   } else {
     const uint16_t* p = E.bf + (int64_t)tok * d;
@@ -201,7 +205,7 @@ __device__ __forceinline__ void load_chunk(const MatView& W, int n, int c, float
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) w[8 * j + e] = nib_to_f(u[j], 4 * e);
+      for (int e = 0; e < 8; ++e) w[8 * j + e] = nib_to_f(u[j], 4 * nib_pos(e));
   } else {
     const uint4* p = reinterpret_cast<const uint4*>(W.bf + (int64_t)n * W.K + c * 32);
     sc = 1.f;
@@ -340,138 +344,6 @@ gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, Mat
   }
 }
 
-// ---------------------------------------------------- tiled GEMM (many rows) ----
-//
-// C[m][n] = sum_k A[m][k] * W[n][k] on CUDA cores: 64 x 64 tiles, K steps of
-// 32, 256 threads with 4 x 4 outputs each; W tiles are dequantised to fp32 in
-// shared memory (INT4: (u - 8) * scale, exact in fp32).
-
-constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 32;
-
-template <int FMT>
-__device__ __forceinline__ void load_w_tile(const MatView& W, int n0, int k0, float (*Ws)[SG_BN + 4]) {
-  // 256 threads: feature f = t / 4 (64 features), quarter qk = t % 4 covers 8 k values.
-  const int t = threadIdx.x, f = t >> 2, qk = t & 3;
-  const int n = n0 + f;
-  float w[8];
-  if (n < W.N) {
-    if constexpr (FMT == TL_FMT_INT4) {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(W.q + (int64_t)n * (W.K / 2) + (k0 + 8 * qk) / 2);
-      const float sc = __half2float(W.s[(int64_t)n * (W.K / W.group) + (k0 + 8 * qk) / W.group]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = nib_to_f(u, 4 * e) * sc;
-    } else {
-      const uint4 v = *reinterpret_cast<const uint4*>(W.bf + (int64_t)n * W.K + k0 + 8 * qk);
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w[2 * e] = __uint_as_float(u[e] << 16);
-        w[2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = 0.f;
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) Ws[8 * qk + e][f] = w[e];
-}
-
-template <int FMT, int EPI>
-__global__ void __launch_bounds__(256)
-gemm_simt_kernel(const float* __restrict__ A, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
-                 int skip_at_or_below) {
-  __shared__ float As[SG_BK][SG_BM + 4];
-  __shared__ float Ws[SG_BK][SG_BN + 4];
-  __shared__ float Ws2[(EPI == EPI_SWIGLU) ? SG_BK : 1][SG_BN + 4];
-  const int M = n_rows[0];
-  const int m0 = blockIdx.y * SG_BM, n0 = blockIdx.x * SG_BN;
-  if (m0 >= M || M <= skip_at_or_below) return;
-  const int K = W.K, N = W.N;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {}, acc2[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += SG_BK) {
-    // A tile: 64 rows x 32 k; thread t loads two float4 (row t/4 and t/4+... ) stored transposed.
-    for (int f = threadIdx.x; f < SG_BM * SG_BK / 4; f += 256) {
-      const int r = f / (SG_BK / 4), kq = f % (SG_BK / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (m0 + r < M) v = *reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * K + k0 + 4 * kq);
-      As[4 * kq][r] = v.x;
-      As[4 * kq + 1][r] = v.y;
-      As[4 * kq + 2][r] = v.z;
-      As[4 * kq + 3][r] = v.w;
-    }
-    load_w_tile<FMT>(W, n0, k0, Ws);
-    if constexpr (EPI == EPI_SWIGLU) load_w_tile<FMT>(W2, n0, k0, Ws2);
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < SG_BK; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Ws[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-      if constexpr (EPI == EPI_SWIGLU) {
-        const float4 b2 = *reinterpret_cast<const float4*>(&Ws2[kk][tx * 4]);
-        const float bv2[4] = {b2.x, b2.y, b2.z, b2.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc2[i][j] = fmaf(av[i], bv2[j], acc2[i][j]);
-      }
-    }
-    __syncthreads();
-  }
-  if constexpr (EPI == EPI_ARGMAX) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = m0 + ty * 4 + i;
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = n0 + tx * 4 + j;
-        if (n < N) {
-          if (better(acc[i][j], n, bv, bi)) { bv = acc[i][j]; bi = n; }
-          if (o.logits && m < M) o.logits[(int64_t)o.lmap[m] * o.ldo + n] = acc[i][j];
-        }
-      }
-#pragma unroll
-      for (int off = 1; off < 16; off <<= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-      }
-      if (tx == 0 && m < M) {
-        o.part_val[(int64_t)m * o.n_parts + blockIdx.x] = bv;
-        o.part_idx[(int64_t)m * o.n_parts + blockIdx.x] = bi;
-      }
-    }
-    return;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = m0 + ty * 4 + i;
-      if (m >= M) continue;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = n0 + tx * 4 + j;
-        if (n >= N) continue;
-        if constexpr (EPI == EPI_STORE) {
-          o.out[(int64_t)m * o.ldo + n] = acc[i][j];
-        } else if constexpr (EPI == EPI_SWIGLU) {
-          o.out[(int64_t)m * o.ldo + n] = silu_f(acc[i][j]) * acc2[i][j];
-        } else {
-          const int hr = o.map ? o.map[m] : m;
-          o.h[(int64_t)hr * N + n] += acc[i][j];
-        }
-      }
-    }
-  }
-}
-
 // --------------------------------------------------------- RoPE + KV ----
 
 // q_out[r] = RoPE(q), and K = RoPE(k), V = v appended (fp16) to the page of
@@ -516,8 +388,8 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
 // block never straddles a page.
 template <int HD>
 __global__ void __launch_bounds__(128)
-attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows, KVGeom g, int slot_base,
-                   int slot_stride, const int32_t* __restrict__ map_lane, int32_t* __restrict__ status) {
+attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows, KVGeom g,
+                   int slot_base, int slot_stride, const int32_t* __restrict__ map_lane, int32_t* __restrict__ status) {
   constexpr int DPL = HD / 32;  // output dims per lane
   __shared__ float qs[HD];
   __shared__ float wm[4], wl[4];
@@ -591,6 +463,7 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows
     float v = 0.f;
     for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
     o[(int64_t)r * d + h * HD + i] = v / Lsum;
+    o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lsum);
   }
 }
 
@@ -605,8 +478,8 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows
 // owns the same rows and dims tx*HD/16 .. +HD/16.
 template <int HD>
 __global__ void __launch_bounds__(256)
-attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, Rows rows, KVGeom g, int slot,
-                    int32_t* __restrict__ status) {
+attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
+                    KVGeom g, int slot, int32_t* __restrict__ status) {
   constexpr int BQ = 64, BK = 64, DPT = HD / 16;
   extern __shared__ float4 smem_pf[];
   float* Qs = reinterpret_cast<float*>(smem_pf);  // [HD][BQ]  (pre-scaled)
@@ -732,7 +605,10 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, Rows row
     if (r >= nq) continue;
     const float inv = 1.f / l[i];
 #pragma unroll
-    for (int j = 0; j < DPT; ++j) o[(int64_t)(r0 + r) * d + h * HD + tx * DPT + j] = acc[i][j] * inv;
+    for (int j = 0; j < DPT; ++j) {
+      o[(int64_t)(r0 + r) * d + h * HD + tx * DPT + j] = acc[i][j] * inv;
+      o16[(int64_t)(r0 + r) * d + h * HD + tx * DPT + j] = __float2half_rn(acc[i][j] * inv);
+    }
   }
 }
 

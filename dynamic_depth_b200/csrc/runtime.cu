@@ -9,9 +9,12 @@
 #include <string>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.cuh"
+#include "tc_gemm.cuh"
 
 namespace tl {
 
@@ -82,13 +85,54 @@ static size_t blob_bytes(const tl_config* c) {
   return s;
 }
 
+// ------------------------------------------------- tensor-core tiling ----
+
+constexpr int kGemvMaxRows = 8;  // row counts the CUDA-core GEMV takes; more go to the tensor cores
+
+static int tc_nt(int max_rows) { return max_rows <= 64 ? 64 : (max_rows <= 128 ? 128 : 256); }
+
+// Split of the K loop so that the grid fills the 148 SMs (two CTAs per SM fit
+// for the smaller tiles).  Every split keeps >= 2 k-blocks and its INT4 scale
+// groups within TC_SC_MAX.
+static int tc_splits(int N, int K, int max_rows, int nmat, int fmt, int group) {
+  const int nt = tc_nt(max_rows);
+  const int m_tiles = (N + 127) / 128, n_tiles = (max_rows + nt - 1) / nt;
+  const int kb = K / 64;
+  const int slots = (nmat == 1 && nt == 64) ? 296 : 148;
+  int best = 1;
+  for (int s = 1; s <= 16; ++s) {
+    if (kb % s) continue;
+    const int per = kb / s;
+    if (per < 2 && s > 1) break;
+    if (fmt == TL_FMT_INT4 && (per * 64) / group + 1 > TC_SC_MAX) continue;
+    if ((int64_t)m_tiles * n_tiles * s <= slots) best = s;
+  }
+  if (fmt == TL_FMT_INT4)
+    while ((kb / best) * 64 / group + 1 > TC_SC_MAX && best < kb) {
+      int nb = best + 1;
+      while (kb % nb) ++nb;
+      best = nb;
+    }
+  return best;
+}
+
+static size_t tc_scratch_bytes(int N, int K, int max_rows, int nmat, int fmt, int group) {
+  if (max_rows <= kGemvMaxRows) return 0;
+  const int nt = tc_nt(max_rows);
+  const int S = tc_splits(N, K, max_rows, nmat, fmt, group);
+  if (S == 1) return 0;
+  const size_t tiles = (size_t)((N + 127) / 128) * ((max_rows + nt - 1) / nt);
+  return tiles * S * nmat * nt * 128 * 4;
+}
+
 // Offsets of every workspace region (computed identically by tl_workspace_bytes and tl_create).
 struct Layout {
   int n_slots, pages_per_seq, n_pages, max_rows, n_parts, max_prefill;
-  size_t page_elems;
+  size_t page_elems, tc_scratch_size;
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[4], act_a, act_qkv, act_q, act_o, act_u,
-      part_val, part_idx, tok_stage, L_stage, mask_stage, out_tok, out_dep, status, counters, alive, total;
+      act_a16, act_o16, act_u16, tc_scratch, tc_counters, part_val, part_idx, tok_stage, L_stage, mask_stage,
+      out_tok, out_dep, status, counters, alive, total;
 };
 
 static Layout make_layout(const tl_config* c) {
@@ -122,6 +166,25 @@ static Layout make_layout(const tl_config* c) {
   L.act_q = take(R * d * 4);
   L.act_o = take(R * d * 4);
   L.act_u = take(R * F * 4);
+  L.act_a16 = take(R * d * 2);
+  L.act_o16 = take(R * d * 2);
+  L.act_u16 = take(R * F * 2);
+  size_t scratch = 0;
+  const int top = c->max_lanes > L.max_prefill ? c->max_lanes : L.max_prefill;
+  for (int b = 0; b < 2; ++b) {
+    const int fmt = b == 0 ? c->fmt_pre : c->fmt_loop;
+    if (b == 0 && c->n_pre == 0) continue;
+    for (int mr = kGemvMaxRows + 1; mr <= top; ++mr) {
+      const size_t v[4] = {tc_scratch_bytes(3 * c->d, c->d, mr, 1, fmt, c->group),
+                           tc_scratch_bytes(c->d, c->d, mr, 1, fmt, c->group),
+                           tc_scratch_bytes(c->ffn, c->d, mr, 2, fmt, c->group),
+                           tc_scratch_bytes(c->d, c->ffn, mr, 1, fmt, c->group)};
+      for (size_t x : v) scratch = x > scratch ? x : scratch;
+    }
+  }
+  L.tc_scratch_size = scratch;
+  L.tc_scratch = take(scratch ? scratch : 256);
+  L.tc_counters = take(4096 * 4);
   L.part_val = take(lanes * L.n_parts * 4);
   L.part_idx = take(lanes * L.n_parts * 4);
   L.tok_stage = take(R * 4);
@@ -139,6 +202,7 @@ static Layout make_layout(const tl_config* c) {
 struct BlockW {
   MatView wqkv, wo, wg, wu, wd;
   const float *g1, *g2;
+  CUtensorMap mqkv, mo, mg, mu, md;  // TMA maps of the raw weight tiles
 };
 
 }  // namespace tl
@@ -163,6 +227,10 @@ struct tl_ctx {
   float *h, *h_in, *hrows;
   Rows rows[4];  // 0 loop, 1 boundary, 2 entered, 3 prefill / mask
   float *act_a, *act_qkv, *act_q, *act_o, *act_u;
+  __half *act_a16, *act_o16, *act_u16;
+  float* tc_scratch;
+  int32_t* tc_counters;
+  CUtensorMap xmap[3][3];  // [a16, o16, u16][NT 64, 128, 256]
   float* part_val;
   int32_t* part_idx;
   int32_t *tok_stage, *L_stage, *out_tok, *out_dep, *status, *alive;
@@ -244,47 +312,100 @@ int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView&
   return launch_err(c);
 }
 
-template <int FMT, int EPI>
-int gemm_launch(tl_ctx* c, int max_rows, const float* A, const int32_t* n, const MatView& W, const MatView& W2,
-                const ProjOut& o, int skip_at_or_below) {
-  dim3 grid((W.N + SG_BN - 1) / SG_BN, (max_rows + SG_BM - 1) / SG_BM);
-  gemm_simt_kernel<FMT, EPI><<<grid, 256, 0, c->stream>>>(A, n, W, W2, o, skip_at_or_below);
+template <int NT, int NMAT, int FMT, int EPI>
+int tc_launch_t(tl_ctx* c, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+                const TcParams& p, dim3 grid) {
+  using Cf = TcCfg<NT, NMAT, FMT>;
+  auto kern = tc_gemm_kernel<NT, NMAT, FMT, EPI>;
+  static bool attr_done = false;  // once per instantiation
+  if (!attr_done) {
+    TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
+    attr_done = true;
+  }
+  kern<<<grid, 256, Cf::SMEM, c->stream>>>(mw, mw2, mx, p);
   return launch_err(c);
 }
 
-constexpr int kGemvMaxRows = 8;
-
-// Projection over the device-side row count: the GEMV takes up to 8 rows; when
-// more rows are possible a tiled GEMM is launched beside it and exactly one of
-// the two does the work.  The head (EPI_ARGMAX) always uses the GEMV, which
-// loops over its rows 8 at a time, so its partial-result count is fixed.
-template <int EPI>
-int proj_epi(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView& W2,
-             ProjOut o) {
-  const bool gemv_only = EPI == EPI_ARGMAX || max_rows <= kGemvMaxRows;
-  if (EPI == EPI_ARGMAX) o.n_parts = (W.N + GEMV_WARPS - 1) / GEMV_WARPS;
-  if (W.fmt == TL_FMT_INT4) {
-    TL_TRY((gemv_launch<TL_FMT_INT4, EPI>(c, X, n, W, W2, o, gemv_only ? 0 : kGemvMaxRows)));
-    if (!gemv_only) TL_TRY((gemm_launch<TL_FMT_INT4, EPI>(c, max_rows, X, n, W, W2, o, kGemvMaxRows)));
-  } else {
-    TL_TRY((gemv_launch<TL_FMT_BF16, EPI>(c, X, n, W, W2, o, gemv_only ? 0 : kGemvMaxRows)));
-    if (!gemv_only) TL_TRY((gemm_launch<TL_FMT_BF16, EPI>(c, max_rows, X, n, W, W2, o, kGemvMaxRows)));
-  }
-  return TL_OK;
+template <int NMAT, int FMT, int EPI>
+int tc_launch_nt(tl_ctx* c, int nt, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+                 const TcParams& p, dim3 grid) {
+  if (nt == 64) return tc_launch_t<64, NMAT, FMT, EPI>(c, mw, mw2, mx, p, grid);
+  if (nt == 128) return tc_launch_t<128, NMAT, FMT, EPI>(c, mw, mw2, mx, p, grid);
+  return tc_launch_t<256, NMAT, FMT, EPI>(c, mw, mw2, mx, p, grid);
 }
 
-int proj(tl_ctx* c, int max_rows, const float* X, const int32_t* n, const MatView& W, const MatView* W2,
-         const ProjOut& o, int prof_kind = TL_PROF_PROJ) {
+// Tensor-core projection reading the fp16 copy `xsel` of the activations
+// (0: norm output, 1: attention output, 2: SwiGLU output).
+int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& W, const CUtensorMap& mw,
+            const MatView* W2, const CUtensorMap* mw2, const ProjOut& o, __half* out16, int skip) {
+  const int nmat = W2 ? 2 : 1;
+  const int nt = tc_nt(max_rows);
+  const int S = tc_splits(W.N, W.K, max_rows, nmat, W.fmt, W.group);
+  dim3 grid((W.N + 127) / 128, (max_rows + nt - 1) / nt, S);
+  if ((size_t)grid.x * grid.y > 4096) return TL_EINVAL;
+  if (S > 1 && (size_t)grid.x * grid.y * S * nmat * nt * 128 * 4 > c->lay.tc_scratch_size) return TL_ENOMEM;
+  TcParams p{};
+  p.n_rows = n;
+  p.skip_at_or_below = skip;
+  p.N = W.N;
+  p.K = W.K;
+  p.group = W.group;
+  p.kb_per_split = (W.K / 64) / S;
+  p.scales = W.s;
+  p.scales2 = W2 ? W2->s : nullptr;
+  p.o = o;
+  p.out16 = out16;
+  p.scratch = c->tc_scratch;
+  p.counters = c->tc_counters;
+  p.status = c->status;
+  const CUtensorMap& mx = c->xmap[xsel][nt == 64 ? 0 : (nt == 128 ? 1 : 2)];
+  const CUtensorMap& m2 = mw2 ? *mw2 : mw;
+  if (W.fmt == TL_FMT_INT4) {
+    if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, TL_FMT_INT4, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);
+    if (o.epi == EPI_RESID) return tc_launch_nt<1, TL_FMT_INT4, EPI_RESID>(c, nt, mw, m2, mx, p, grid);
+    return tc_launch_nt<1, TL_FMT_INT4, EPI_STORE>(c, nt, mw, m2, mx, p, grid);
+  }
+  if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, TL_FMT_BF16, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);
+  if (o.epi == EPI_RESID) return tc_launch_nt<1, TL_FMT_BF16, EPI_RESID>(c, nt, mw, m2, mx, p, grid);
+  return tc_launch_nt<1, TL_FMT_BF16, EPI_STORE>(c, nt, mw, m2, mx, p, grid);
+}
+
+// Projection over the device-side row count: the CUDA-core GEMV takes up to 8
+// rows (exact fp32 weights and activations); larger counts go to the tensor
+// cores.  When the host only knows an upper bound both are launched and the
+// one that does not apply returns at once; when it knows the exact count
+// (`exact`, prompts) only the right one is launched.  The head (EPI_ARGMAX)
+// always uses the GEMV, which loops over its rows 8 at a time.
+int proj(tl_ctx* c, int max_rows, bool exact, const float* X, int xsel, const int32_t* n, const MatView& W,
+         const CUtensorMap* mw, const MatView* W2, const CUtensorMap* mw2, ProjOut o, __half* out16,
+         int prof_kind = TL_PROF_PROJ) {
   const MatView& w2 = W2 ? *W2 : W;
   TL_TRY(prof_start(c, prof_kind));
-  int st;
-  switch (o.epi) {
-    case EPI_STORE: st = proj_epi<EPI_STORE>(c, max_rows, X, n, W, w2, o); break;
-    case EPI_RESID: st = proj_epi<EPI_RESID>(c, max_rows, X, n, W, w2, o); break;
-    case EPI_SWIGLU: st = proj_epi<EPI_SWIGLU>(c, max_rows, X, n, W, w2, o); break;
-    default: st = proj_epi<EPI_ARGMAX>(c, max_rows, X, n, W, w2, o); break;
+  const bool argmax = o.epi == EPI_ARGMAX;
+  const bool use_tc = !argmax && max_rows > kGemvMaxRows;
+  const bool use_gemv = argmax || !use_tc || !exact;
+  if (argmax) o.n_parts = (W.N + GEMV_WARPS - 1) / GEMV_WARPS;
+  if (use_gemv) {
+    const int skip = use_tc ? kGemvMaxRows : 0;
+    int st;
+    if (W.fmt == TL_FMT_INT4) {
+      switch (o.epi) {
+        case EPI_STORE: st = gemv_launch<TL_FMT_INT4, EPI_STORE>(c, X, n, W, w2, o, skip); break;
+        case EPI_RESID: st = gemv_launch<TL_FMT_INT4, EPI_RESID>(c, X, n, W, w2, o, skip); break;
+        case EPI_SWIGLU: st = gemv_launch<TL_FMT_INT4, EPI_SWIGLU>(c, X, n, W, w2, o, skip); break;
+        default: st = gemv_launch<TL_FMT_INT4, EPI_ARGMAX>(c, X, n, W, w2, o, skip); break;
+      }
+    } else {
+      switch (o.epi) {
+        case EPI_STORE: st = gemv_launch<TL_FMT_BF16, EPI_STORE>(c, X, n, W, w2, o, skip); break;
+        case EPI_RESID: st = gemv_launch<TL_FMT_BF16, EPI_RESID>(c, X, n, W, w2, o, skip); break;
+        case EPI_SWIGLU: st = gemv_launch<TL_FMT_BF16, EPI_SWIGLU>(c, X, n, W, w2, o, skip); break;
+        default: st = gemv_launch<TL_FMT_BF16, EPI_ARGMAX>(c, X, n, W, w2, o, skip); break;
+      }
+    }
+    TL_TRY(st);
   }
-  TL_TRY(st);
+  if (use_tc) TL_TRY(tc_proj(c, max_rows, xsel, n, W, *mw, W2, mw2, o, out16, exact ? 0 : kGemvMaxRows));
   return prof_stop(c, prof_kind);
 }
 
@@ -292,9 +413,9 @@ int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int sl
   TL_TRY(prof_start(c, TL_PROF_ATTN));
   dim3 grid(max_rows, c->cfg.n_heads);
   switch (c->hd) {
-    case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
-    case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
-    default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+    case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+    case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+    default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
   }
   TL_TRY(launch_err(c));
   return prof_stop(c, TL_PROF_ATTN);
@@ -310,7 +431,8 @@ int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot) 
     attr_done = true;
   }
   dim3 grid((max_rows + 63) / 64, c->cfg.n_heads);
-  attn_prefill_kernel<HD><<<grid, 256, smem, c->stream>>>(c->act_q, c->act_o, rows, c->kv, slot, c->status);
+  attn_prefill_kernel<HD><<<grid, 256, smem, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot,
+                                                            c->status);
   return launch_err(c);
 }
 
@@ -333,13 +455,13 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
               int slot_base, int slot_stride, float* h_in, bool prompt = false) {
   const int d = c->cfg.d, F = c->cfg.ffn;
   const float eps = c->cfg.rms_eps;
-  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in);
+  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in, c->act_a16);
   TL_TRY(launch_err(c));
   ProjOut o{};
   o.epi = EPI_STORE;
   o.out = c->act_qkv;
   o.ldo = 3 * d;
-  TL_TRY(proj(c, max_rows, c->act_a, rows.n, w.wqkv, nullptr, o));
+  TL_TRY(proj(c, max_rows, prompt, c->act_a, 0, rows.n, w.wqkv, &w.mqkv, nullptr, nullptr, o, nullptr));
   rope_kv_kernel<<<max_rows, d / 2, 0, c->stream>>>(c->act_qkv, c->act_q, rows, c->kv, c->rope, slot_base,
                                                      slot_stride, nullptr, c->status);
   TL_TRY(launch_err(c));
@@ -351,15 +473,16 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   r.epi = EPI_RESID;
   r.h = hbuf;
   r.map = map;
-  TL_TRY(proj(c, max_rows, c->act_o, rows.n, w.wo, nullptr, r));
-  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr);
+  TL_TRY(proj(c, max_rows, prompt, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
+  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr,
+                                                       c->act_a16);
   TL_TRY(launch_err(c));
-  ProjOut s{};
-  s.epi = EPI_SWIGLU;
-  s.out = c->act_u;
-  s.ldo = F;
-  TL_TRY(proj(c, max_rows, c->act_a, rows.n, w.wg, &w.wu, s));
-  return proj(c, max_rows, c->act_u, rows.n, w.wd, nullptr, r);
+  ProjOut sw{};
+  sw.epi = EPI_SWIGLU;
+  sw.out = c->act_u;
+  sw.ldo = F;
+  TL_TRY(proj(c, max_rows, prompt, c->act_a, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16));
+  return proj(c, max_rows, prompt, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr);
 }
 
 // Row table `which` from lanes 0..n_consider-1 (all lanes when n_consider <= 0).
@@ -397,7 +520,7 @@ int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax
                int32_t* dep_out, int n_new) {
   const Rows& B = c->rows[1];
   rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(c->h, B.lane, B.n, c->cfg.d, c->g_final, c->cfg.rms_eps,
-                                                       c->act_a, nullptr);
+                                                       c->act_a, nullptr, nullptr);
   TL_TRY(launch_err(c));
   ProjOut o{};
   o.epi = EPI_ARGMAX;
@@ -406,9 +529,8 @@ int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax
   o.ldo = c->cfg.vocab;
   o.part_val = c->part_val;
   o.part_idx = c->part_idx;
-  TL_TRY(proj(c, max_rows, c->act_a, B.n, c->head, nullptr, o, TL_PROF_HEAD));
-  const int n_parts = max_rows <= kGemvMaxRows ? (c->cfg.vocab + GEMV_WARPS - 1) / GEMV_WARPS
-                                               : (c->cfg.vocab + SG_BN - 1) / SG_BN;
+  TL_TRY(proj(c, max_rows, false, c->act_a, 0, B.n, c->head, nullptr, nullptr, nullptr, o, nullptr, TL_PROF_HEAD));
+  const int n_parts = (c->cfg.vocab + GEMV_WARPS - 1) / GEMV_WARPS;
   head_finalize_kernel<<<max_rows, 256, 0, c->stream>>>(B, c->lanes, c->part_val, c->part_idx, n_parts, mode, argmax,
                                                         tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
                                                         c->cfg.max_seq, c->status, &c->counters[1]);
@@ -427,6 +549,69 @@ void release_lane_pages(tl_ctx* c, int lane) {
     t[i] = -1;
   }
   c->lane_L[lane] = 0;
+}
+
+// --------------------------------------------------------- tensor maps ----
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major 2D map: `inner` elements per row, `outer` rows, row pitch in bytes.
+int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = tensor_map_encoder();
+  if (!fn) {
+    g_cuda_err = "cuTensorMapEncodeTiled entry point unavailable";
+    return TL_ECUDA;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_cuda_err = "cuTensorMapEncodeTiled failed";
+    return TL_ECUDA;
+  }
+  return TL_OK;
+}
+
+// Raw weight tiles: INT4 128 rows x 32 bytes, BF16 128 rows x 64 elements; unswizzled.
+int encode_weight_map(CUtensorMap* m, const MatView& W) {
+  if (W.fmt == TL_FMT_INT4)
+    return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.q, (uint64_t)W.K / 2, (uint64_t)W.N, (uint64_t)W.K / 2, 32,
+                     128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, W.bf, (uint64_t)W.K, (uint64_t)W.N, (uint64_t)W.K * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int encode_all_maps(tl_ctx* c) {
+  for (auto* v : {&c->pre, &c->loop})
+    for (BlockW& b : *v) {
+      TL_TRY(encode_weight_map(&b.mqkv, b.wqkv));
+      TL_TRY(encode_weight_map(&b.mo, b.wo));
+      TL_TRY(encode_weight_map(&b.mg, b.wg));
+      TL_TRY(encode_weight_map(&b.mu, b.wu));
+      TL_TRY(encode_weight_map(&b.md, b.wd));
+    }
+  const __half* xs[3] = {c->act_a16, c->act_o16, c->act_u16};
+  const int ks[3] = {c->cfg.d, c->cfg.d, c->cfg.ffn};
+  const int nts[3] = {64, 128, 256};
+  for (int x = 0; x < 3; ++x)
+    for (int i = 0; i < 3; ++i)
+      TL_TRY(encode_2d(&c->xmap[x][i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[x], (uint64_t)ks[x],
+                       (uint64_t)c->lay.max_rows, (uint64_t)ks[x] * 2, 64, nts[i], CU_TENSOR_MAP_SWIZZLE_128B));
+  return TL_OK;
 }
 
 }  // namespace
@@ -551,6 +736,11 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->act_q = (float*)(w + lay.act_q);
   c->act_o = (float*)(w + lay.act_o);
   c->act_u = (float*)(w + lay.act_u);
+  c->act_a16 = (__half*)(w + lay.act_a16);
+  c->act_o16 = (__half*)(w + lay.act_o16);
+  c->act_u16 = (__half*)(w + lay.act_u16);
+  c->tc_scratch = (float*)(w + lay.tc_scratch);
+  c->tc_counters = (int32_t*)(w + lay.tc_counters);
   c->part_val = (float*)(w + lay.part_val);
   c->part_idx = (int32_t*)(w + lay.part_idx);
   c->tok_stage = (int32_t*)(w + lay.tok_stage);
@@ -580,6 +770,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     if ((st = check_cuda(cudaMemsetAsync(w + lay.page_table, 0xFF, per_lane * cfg->max_lanes * 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->status, 0, 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->counters, 0, 32, c->stream))) != TL_OK) break;
+    if ((st = check_cuda(cudaMemsetAsync(c->tc_counters, 0, 4096 * 4, c->stream))) != TL_OK) break;
+    if ((st = encode_all_maps(c)) != TL_OK) break;
     for (int i = 0; i < 4; ++i)
       if ((st = check_cuda(cudaMemsetAsync(c->rows[i].n, 0, 4, c->stream))) != TL_OK) break;
     if (st != TL_OK) break;
@@ -631,6 +823,17 @@ extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
   }
   const size_t gb = (size_t)(2 * (cfg->n_pre + cfg->n_loop_layers) + 1) * cfg->d * 4;
   TL_CUDA(cudaMemcpyAsync(c->ws + c->lay.gains, b + off, gb, cudaMemcpyHostToDevice, c->stream));
+  // INT4 matrices into the device nibble order
+  std::vector<const MatView*> mats = {&c->embed, &c->head};
+  for (auto* v : {&c->pre, &c->loop})
+    for (const BlockW& bw : *v)
+      for (const MatView* m : {&bw.wqkv, &bw.wo, &bw.wg, &bw.wu, &bw.wd}) mats.push_back(m);
+  for (const MatView* m : mats) {
+    if (m->fmt != TL_FMT_INT4) continue;
+    const int64_t words = (int64_t)m->N * m->K / 8;
+    int4_repack_kernel<<<(unsigned)((words + 255) / 256), 256, 0, c->stream>>>((uint32_t*)m->q, words);
+    TL_TRY(launch_err(c));
+  }
   TL_CUDA(cudaStreamSynchronize(c->stream));
   c->loaded = true;
   return TL_OK;

@@ -1,0 +1,407 @@
+// W4A16 / BF16 projection on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Y[rows, N] = X[rows, K] * W[N, K]^T computed as its transpose: the weight
+// tile is the 128-row M operand and the activation rows are the N operand
+// (NT = 64, 128 or 256 rows), so decode batches of a few dozen lanes still fill
+// an M=128 instruction while the kernel streams each weight byte once.
+//
+// Per CTA (256 threads): warp 0 issues TMA loads of the raw weight tile (INT4
+// nibbles or BF16, unswizzled) and of the fp16 activation tile (SWIZZLE_128B)
+// into a ring of stages; warps 4-7 convert the raw weight tile to fp16 in the
+// canonical K-major SWIZZLE_128B layout (INT4: (u - 8) * scale rounded once to
+// fp16) and later run the epilogue; warp 1 issues tcgen05.mma (K = 16 per
+// instruction, 4 per 64-wide k-block) into a TMEM accumulator and commits each
+// stage back to the producer; warp 2 owns the TMEM allocation.  Split-K CTAs
+// write fp32 partials to scratch and the last CTA of a tile (arrival counter)
+// sums them in split order and applies the epilogue, so results do not depend
+// on CTA timing.  Every mbarrier wait is bounded (~1.5 s of %globaltimer);
+// on expiry the CTA records ST_TIMEOUT in the status word and unwinds.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace tl {
+
+constexpr int ST_TIMEOUT = 1 << 6;
+
+struct TcParams {
+  const int32_t* n_rows;   // device scalar
+  int32_t skip_at_or_below;
+  int32_t N, K, group;
+  int32_t kb_per_split;    // 64-wide k-blocks per split
+  const __half* scales;    // INT4: [N][K/group]
+  const __half* scales2;   // second matrix (gate/up pair)
+  ProjOut o;
+  __half* out16;           // fp16 copy of EPI_STORE / EPI_SWIGLU rows (ld = o.ldo), nullable
+  float* scratch;          // split-K partials
+  int32_t* counters;       // per-tile arrivals, zero between launches
+  int32_t* status;
+};
+
+constexpr int TC_SC_MAX = 33;  // scale groups per CTA row
+
+template <int NT, int NMAT, int FMT>
+struct TcCfg {
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = NT * 64 * 2;
+  static constexpr int RAW_BYTES = (FMT == TL_FMT_INT4) ? 128 * 32 : 128 * 128;
+  static constexpr int SC_BYTES = (FMT == TL_FMT_INT4) ? NMAT * 128 * TC_SC_MAX * 2 : 0;
+  static constexpr int stage_bytes = NMAT * (A_BYTES + RAW_BYTES) + B_BYTES;
+  static constexpr int fixed = SC_BYTES + 256 + 1024;
+  // the 64-row single-matrix tile (decode batches) keeps 3 stages so two CTAs share an SM
+  static constexpr int CAP = (NT == 64 && NMAT == 1) ? 3 : 4;
+  static constexpr int STAGES = ((220 * 1024 - fixed) / stage_bytes) >= CAP ? CAP : ((220 * 1024 - fixed) / stage_bytes);
+  static constexpr int SMEM = STAGES * stage_bytes + fixed;
+  static constexpr int TMEM_COLS = (NMAT * NT <= 32) ? 32 : NMAT * NT;
+  static_assert(STAGES >= 2, "tile does not fit in shared memory");
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag) {
+  uint64_t start = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 31) == 31) {
+      if (*abort_flag) return false;
+      const uint64_t now = gtimer();
+      if (start == 0) {
+        start = now;
+      } else if (now - start > 1500000000ull) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// K-major, SWIZZLE_128B canonical layout: 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+template <int NT>
+__device__ __forceinline__ constexpr uint32_t umma_idesc_f16() {
+  // D fp32, A/B fp16, both K-major, N = NT, M = 128
+  return (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// INT4 device layout: in each 32-bit word of 8 consecutive k, element 2i is
+// nibble i and element 2i+1 is nibble i + 4 (see the load-time repack), so
+// (w >> 4i) & 0x000F000F is the pair (2i, 2i+1) as two 16-bit lanes.
+__device__ __forceinline__ uint4 int4_word_to_half8(uint32_t w, __half2 s2) {
+  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t bits = ((w >> (4 * i)) & 0x000F000Fu) | 0x64006400u;  // (1024 + u) in each half
+    __half2 h = *reinterpret_cast<const __half2*>(&bits);
+    h = __hmul2(__hsub2(h, off), s2);  // (u - 8) exact, then one rounding of (u - 8) * s
+    out[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__device__ __forceinline__ uint4 bf16x8_to_half8(uint4 v) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(in[i] << 16), __uint_as_float(in[i] & 0xFFFF0000u));
+    out[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+template <int EPI>
+__device__ __forceinline__ void tc_store(const TcParams& p, int row, int m, float v, float v2) {
+  const ProjOut& o = p.o;
+  if constexpr (EPI == EPI_STORE) {
+    o.out[(int64_t)row * o.ldo + m] = v;
+    if (p.out16) p.out16[(int64_t)row * o.ldo + m] = __float2half_rn(v);
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    const float u = silu_f(v) * v2;
+    o.out[(int64_t)row * o.ldo + m] = u;
+    if (p.out16) p.out16[(int64_t)row * o.ldo + m] = __float2half_rn(u);
+  } else {
+    const int hr = o.map ? o.map[row] : row;
+    o.h[(int64_t)hr * p.N + m] += v;
+  }
+}
+
+template <int NT, int NMAT, int FMT, int EPI>
+__global__ void __launch_bounds__(256, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapW2,
+               const __grid_constant__ CUtensorMap mapX, TcParams p) {
+  using C = TcCfg<NT, NMAT, FMT>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = base;                                          // [STAGES][NMAT][A_BYTES]
+  uint8_t* sB = sA + STAGES * NMAT * C::A_BYTES;               // [STAGES][B_BYTES]
+  uint8_t* sRaw = sB + STAGES * C::B_BYTES;                    // [STAGES][NMAT][RAW_BYTES]
+  __half* sSc = reinterpret_cast<__half*>(sRaw + STAGES * NMAT * C::RAW_BYTES);  // [NMAT][128][TC_SC_MAX]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sSc) + C::SC_BYTES);
+  uint64_t* full = bars;                // TMA landed (raw W + X)
+  uint64_t* afull = bars + STAGES;      // fp16 weight tile converted
+  uint64_t* empty = bars + 2 * STAGES;  // MMAs of the stage finished
+  uint64_t* accfull = bars + 3 * STAGES;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 3 * STAGES + 1);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+  volatile int32_t* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows = p.n_rows[0];
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * NT;
+  if (rows <= p.skip_at_or_below || n0 >= rows) return;
+  const int nkb = p.kb_per_split, kb0 = blockIdx.z * nkb;
+  const int S = gridDim.z;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&afull[s]), 4);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(accfull), 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32((const void*)tmem_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if constexpr (FMT == TL_FMT_INT4) {
+    if (warp >= 4) {
+      const int t = threadIdx.x - 128;
+      const int g = p.group;
+      const int gfirst = (kb0 * 64) / g;
+      const int glast = ((kb0 + nkb) * 64 - 1) / g;
+      for (int mat = 0; mat < NMAT; ++mat) {
+        const __half* sc = mat == 0 ? p.scales : p.scales2;
+        const int64_t rowoff = (int64_t)(m0 + t) * (p.K / g);
+        for (int j = 0; j <= glast - gfirst && j < TC_SC_MAX; ++j)
+          sSc[(mat * 128 + t) * TC_SC_MAX + j] = (m0 + t < p.N) ? sc[rowoff + gfirst + j] : __float2half(0.f);
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES, r = i / STAGES;
+        if (r > 0 && !mbar_wait(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) break;
+        const uint32_t fb = smem_u32(&full[s]);
+        mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
+        const int kb = kb0 + i;
+        const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
+        tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
+        if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+        tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
+        issued = i + 1;
+      }
+      if (*abort_flag) {  // let copies already in flight land before the CTA leaves
+        for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
+          volatile int32_t never = 0;
+          mbar_wait(smem_u32(&full[i % STAGES]), (i / STAGES) & 1, &never);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_f16<NT>();
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES, r = i / STAGES;
+        if (!mbar_wait(smem_u32(&afull[s]), r & 1, abort_flag)) break;
+        if (!mbar_wait(smem_u32(&full[s]), r & 1, abort_flag)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bdesc = umma_desc(b_addr + kk * 32);
+#pragma unroll
+          for (int mat = 0; mat < NMAT; ++mat) {
+            const uint64_t adesc = umma_desc(smem_u32(sA + (s * NMAT + mat) * C::A_BYTES) + kk * 32);
+            umma_f16(tmem + mat * NT, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(smem_u32(&empty[s]));
+      }
+      umma_commit(smem_u32(accfull));
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------- convert + epilogue
+    const int t = threadIdx.x - 128;  // weight row within the tile == TMEM lane
+    const int q = warp - 4;
+    const int gfirst = (FMT == TL_FMT_INT4) ? (kb0 * 64) / p.group : 0;
+    bool ok = true;
+    for (int i = 0; i < nkb && ok; ++i) {
+      const int s = i % STAGES, r = i / STAGES;
+      if (!mbar_wait(smem_u32(&full[s]), r & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+      for (int mat = 0; mat < NMAT; ++mat) {
+        uint8_t* arow = sA + (s * NMAT + mat) * C::A_BYTES + t * 128;
+        const uint8_t* raw = sRaw + (s * NMAT + mat) * C::RAW_BYTES;
+        if constexpr (FMT == TL_FMT_INT4) {
+          const uint4 w0 = *reinterpret_cast<const uint4*>(raw + t * 32);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(raw + t * 32 + 16);
+          const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          const int kbase = (kb0 + i) * 64;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const __half sc = sSc[(mat * 128 + t) * TC_SC_MAX + (kbase + 8 * c) / p.group - gfirst];
+            const uint4 h = int4_word_to_half8(w[c], __halves2half2(sc, sc));
+            *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = h;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(raw + t * 128 + c * 16);
+            *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = bf16x8_to_half8(v);
+          }
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
+    }
+    if (ok && mbar_wait(smem_u32(accfull), 0, abort_flag)) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const int m = m0 + t;
+      const int ncols = min(NT, rows - n0);
+      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+      const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+      for (int j = 0; j < ncols; j += 8) {
+        float v[8], v2[8];
+        tmem_ld8(tl + j, v);
+        if constexpr (NMAT == 2) tmem_ld8(tl + NT + j, v2);
+        if (S == 1) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (j + e < ncols && m < p.N) tc_store<EPI>(p, n0 + j + e, m, v[e], NMAT == 2 ? v2[e] : 0.f);
+        } else {
+          float* part = p.scratch + ((int64_t)(tile * S + blockIdx.z) * NMAT) * NT * 128;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            part[(j + e) * 128 + t] = v[e];
+            if constexpr (NMAT == 2) part[NT * 128 + (j + e) * 128 + t] = v2[e];
+          }
+        }
+      }
+      if (S > 1) {
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (t == 0) *last_flag = (atomicAdd(&p.counters[tile], 1) == S - 1) ? 1 : 0;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*last_flag) {
+          __threadfence();
+          for (int j = 0; j < ncols; ++j) {
+            float a = 0.f, b = 0.f;
+            for (int z = 0; z < S; ++z) {
+              const float* part = p.scratch + ((int64_t)(tile * S + z) * NMAT) * NT * 128;
+              a += __ldcg(part + j * 128 + t);
+              if constexpr (NMAT == 2) b += __ldcg(part + NT * 128 + j * 128 + t);
+            }
+            if (m < p.N) tc_store<EPI>(p, n0 + j, m, a, b);
+          }
+          if (t == 0) p.counters[tile] = 0;
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, ST_TIMEOUT);
+  if (warp == 2) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// Load-time repack of an INT4 matrix (standard packing: element e of each
+// 8-element word in nibble e) into the device layout used above and by the
+// CUDA-core kernels (element 2i in nibble i, 2i+1 in nibble i + 4).  In place.
+__global__ void int4_repack_kernel(uint32_t* __restrict__ w, int64_t n_words) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_words) return;
+  const uint32_t x = w[i];
+  uint32_t y = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    y |= ((x >> (4 * e)) & 0xFu) << (4 * nib_pos(e));
+  }
+  w[i] = y;
+}
+
+}  // namespace tl

@@ -150,3 +150,44 @@ def test_m407_decode_logits_teacher_forced(L):
         assert_logits_close(lg[0, t], ref[0].logits[t], f"L={L} token {t}")
         if M.top2_margin(ref[0].logits[t]) > MARGIN:
             assert am[0, t] == ref[0].tokens[t]
+
+
+# ------------------------------------------- wide batches (tensor-core path) ----
+
+def test_tiny_wide_batch_tensor_core_decode():
+    # 12 lanes: more rows than the CUDA-core GEMV takes, so loop steps run on tcgen05
+    W = oracle_weights("tiny", 7)
+    P = S.prompts(12, 16, 512, seed=71)
+    Ls = [2, 3, 4, 5] * 3
+    m = gpu_model("tiny", 7, max_lanes=12, max_seq=32, L_max=8)
+    ref, lg, am, dep = teacher_forced(m, W, P, Ls, 4)
+    status_clean(m)
+    for i in range(12):
+        assert dep[i].tolist() == ref[i].depths.tolist()
+        for t in range(4):
+            assert_logits_close(lg[i, t], ref[i].logits[t], f"lane {i} token {t}")
+
+
+def test_tiny_wide_batch_generate_matches_oracle():
+    W = oracle_weights("tiny")
+    P = S.prompts(16, 20, 512, seed=72)
+    Ls = [1, 2, 3, 4, 5, 6, 7, 8] * 2
+    m = gpu_model("tiny", None, max_lanes=16, max_seq=40, L_max=8)
+    tok, dep = m.generate(P, Ls, 8)
+    status_clean(m)
+    for i in range(16):
+        r = D.generate_lane(W, P[i], Ls[i], 8)
+        assert dep[i].tolist() == r.depths.tolist()
+        _check_tokens(r.tokens, r.logits, tok[i])
+
+
+def test_m407_wide_decode_logits():
+    W = oracle_weights("m407")
+    P = S.prompts(16, 24, S.M407.vocab, seed=73)
+    Ls = [3] * 16
+    m = gpu_model("m407", None, max_lanes=16, max_seq=32, L_max=4)
+    ref, lg, am, dep = teacher_forced(m, W, P, Ls, 3)
+    status_clean(m)
+    for i in range(16):
+        for t in range(3):
+            assert_logits_close(lg[i, t], ref[i].logits[t], f"lane {i} token {t}")
