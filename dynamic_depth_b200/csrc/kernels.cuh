@@ -131,11 +131,13 @@ __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, in
 
 // out[r] = RMSNorm(h[map ? map[r] : r]) * g, fp32 (and an fp16 copy for the
 // tensor-core projections when out16 is given).  One CTA per row.  When h_in is
-// given, also copies the source row there (indexed like h).
+// given, also copies the source row there (indexed like h); when zero_rows is
+// given, clears row r of that [rows][zero_cols] accumulator, which the next
+// (split-K) projection adds into.
 __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* __restrict__ map,
                                     const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
                                     float eps, float* __restrict__ out, float* __restrict__ h_in,
-                                    __half* __restrict__ out16) {
+                                    __half* __restrict__ out16, float* __restrict__ zero_rows, int zero_cols) {
   __shared__ float red[32];
   const int r = blockIdx.x;
   if (r >= n_rows[0]) return;
@@ -152,6 +154,8 @@ __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* 
     if (out16) out16[(int64_t)r * d + k] = __float2half_rn(y);
     if (h_in) h_in[(int64_t)src * d + k] = v;
   }
+  if (zero_rows)
+    for (int k = threadIdx.x; k < zero_cols; k += blockDim.x) zero_rows[(int64_t)r * zero_cols + k] = 0.f;
 }
 
 // ------------------------------------------------------------ embedding ----
@@ -196,23 +200,38 @@ constexpr int GEMV_WARPS = 8;
 
 __device__ __forceinline__ int swz_slot(int f) { return (f & ~7) | ((f & 7) ^ ((f >> 3) & 7)); }
 
+// Raw bytes of one 32-element chunk of a weight row: INT4 16 bytes, BF16 64.
 template <int FMT>
-__device__ __forceinline__ void load_chunk(const MatView& W, int n, int c, float (&w)[32], float& sc) {
+struct Chunk {
+  uint4 v[FMT == TL_FMT_INT4 ? 1 : 4];
+  float sc;
+};
+
+template <int FMT>
+__device__ __forceinline__ void load_chunk_raw(const MatView& W, int n, int c, Chunk<FMT>& ch) {
   if constexpr (FMT == TL_FMT_INT4) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(W.q + (int64_t)n * (W.K / 2) + c * 16));
-    sc = __half2float(W.s[(int64_t)n * (W.K / W.group) + (c * 32) / W.group]);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    ch.v[0] = __ldg(reinterpret_cast<const uint4*>(W.q + (int64_t)n * (W.K / 2) + c * 16));
+    ch.sc = __half2float(W.s[(int64_t)n * (W.K / W.group) + (c * 32) / W.group]);
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(W.bf + (int64_t)n * W.K + c * 32);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ch.v[j] = __ldg(p + j);
+    ch.sc = 1.f;
+  }
+}
+
+template <int FMT>
+__device__ __forceinline__ void unpack_chunk(const Chunk<FMT>& ch, float (&w)[32]) {
+  if constexpr (FMT == TL_FMT_INT4) {
+    const uint32_t u[4] = {ch.v[0].x, ch.v[0].y, ch.v[0].z, ch.v[0].w};
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int e = 0; e < 8; ++e) w[8 * j + e] = nib_to_f(u[j], 4 * nib_pos(e));
   } else {
-    const uint4* p = reinterpret_cast<const uint4*>(W.bf + (int64_t)n * W.K + c * 32);
-    sc = 1.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint4 v = __ldg(p + j);
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+      const uint32_t u[4] = {ch.v[j].x, ch.v[j].y, ch.v[j].z, ch.v[j].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         w[8 * j + 2 * e] = __uint_as_float(u[e] << 16);
@@ -241,46 +260,77 @@ __device__ __forceinline__ void dot_chunk(const float* __restrict__ xs, int K, i
   }
 }
 
-template <int FMT, int R, int EPI>
+// One warp owns RPW consecutive output features (for EPI_SWIGLU: gate row n
+// and up row n, RPW = 1); a lane loads the raw chunks of all of them before
+// using any, so a warp keeps RPW (x2) 16-byte loads in flight per lane.
+template <int FMT, int R, int EPI, int RPW>
 __device__ __forceinline__ void gemv_rows(const float* __restrict__ xs, int r0, int rows, const MatView& W,
                                           const MatView& W2, const ProjOut& o, float (*best_v)[8],
                                           int (*best_i)[8]) {
   const int K = W.K, N = W.N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = blockIdx.x * GEMV_WARPS + warp;
+  const int nbase = (blockIdx.x * GEMV_WARPS + warp) * RPW;
   const int nch = K / 32;
-  float acc[R], acc2[R];
+  float acc[RPW][R], acc2[R];
 #pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = acc2[r] = 0.f;
-  if (n < N) {
-    for (int c = lane; c < nch; c += 32) {
-      float w[32], sc;
-      load_chunk<FMT>(W, n, c, w, sc);
-      dot_chunk<R>(xs, K, c, w, sc, acc);
-      if constexpr (EPI == EPI_SWIGLU) {
-        load_chunk<FMT>(W2, n, c, w, sc);
-        dot_chunk<R>(xs, K, c, w, sc, acc2);
+  for (int f = 0; f < RPW; ++f)
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[f][r] = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc2[r] = 0.f;
+  for (int c = lane; c < nch; c += 32) {
+    Chunk<FMT> ch[RPW];
+#pragma unroll
+    for (int f = 0; f < RPW; ++f)
+      if (nbase + f < N) load_chunk_raw<FMT>(W, nbase + f, c, ch[f]);
+    Chunk<FMT> ch2;
+    if constexpr (EPI == EPI_SWIGLU)
+      if (nbase < N) load_chunk_raw<FMT>(W2, nbase, c, ch2);
+#pragma unroll
+    for (int f = 0; f < RPW; ++f) {
+      if (nbase + f < N) {
+        float w[32];
+        unpack_chunk<FMT>(ch[f], w);
+        dot_chunk<R>(xs, K, c, w, ch[f].sc, acc[f]);
+      }
+    }
+    if constexpr (EPI == EPI_SWIGLU) {
+      if (nbase < N) {
+        float w[32];
+        unpack_chunk<FMT>(ch2, w);
+        dot_chunk<R>(xs, K, c, w, ch2.sc, acc2);
       }
     }
   }
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    acc[r] = warp_sum(acc[r]);
-    if constexpr (EPI == EPI_SWIGLU) acc2[r] = warp_sum(acc2[r]);
+  for (int f = 0; f < RPW; ++f)
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[f][r] = warp_sum(acc[f][r]);
+  if constexpr (EPI == EPI_SWIGLU) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc2[r] = warp_sum(acc2[r]);
   }
   if constexpr (EPI == EPI_ARGMAX) {
     if (lane == 0) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        best_v[warp][r] = (n < N) ? acc[r] : -INFINITY;
-        best_i[warp][r] = (n < N) ? n : 0x7fffffff;
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int f = 0; f < RPW; ++f)
+          if (nbase + f < N && better(acc[f][r], nbase + f, bv, bi)) { bv = acc[f][r]; bi = nbase + f; }
+        best_v[warp][r] = bv;
+        best_i[warp][r] = bi;
       }
     }
-    if (n < N && o.logits && lane < R && r0 + lane < rows) {
-      float v = acc[0];
+    if (o.logits && lane < R && r0 + lane < rows) {
 #pragma unroll
-      for (int r = 1; r < R; ++r) if (lane == r) v = acc[r];
-      o.logits[(int64_t)o.lmap[r0 + lane] * o.ldo + n] = v;
+      for (int f = 0; f < RPW; ++f) {
+        float v = acc[f][0];
+#pragma unroll
+        for (int r = 1; r < R; ++r) if (lane == r) v = acc[f][r];
+        if (nbase + f < N) o.logits[(int64_t)o.lmap[r0 + lane] * o.ldo + nbase + f] = v;
+      }
     }
     __syncthreads();
     if (threadIdx.x < R && r0 + threadIdx.x < rows) {
@@ -292,27 +342,33 @@ __device__ __forceinline__ void gemv_rows(const float* __restrict__ xs, int r0, 
       o.part_val[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bv;
       o.part_idx[(int64_t)(r0 + r) * o.n_parts + blockIdx.x] = bi;
     }
-  } else if (n < N && lane < R && r0 + lane < rows) {
-    float v = acc[0], v2 = acc2[0];
-#pragma unroll
-    for (int r = 1; r < R; ++r)
-      if (lane == r) { v = acc[r]; v2 = acc2[r]; }
+  } else if (lane < R && r0 + lane < rows) {
     const int r = r0 + lane;
-    if constexpr (EPI == EPI_STORE) {
-      o.out[(int64_t)r * o.ldo + n] = v;
-    } else if constexpr (EPI == EPI_SWIGLU) {
-      o.out[(int64_t)r * o.ldo + n] = silu_f(v) * v2;
-    } else {
-      const int hr = o.map ? o.map[r] : r;
-      o.h[(int64_t)hr * N + n] += v;
+#pragma unroll
+    for (int f = 0; f < RPW; ++f) {
+      const int n = nbase + f;
+      if (n >= N) continue;
+      float v = acc[f][0], v2 = acc2[0];
+#pragma unroll
+      for (int rr = 1; rr < R; ++rr)
+        if (lane == rr) { v = acc[f][rr]; v2 = acc2[rr]; }
+      if constexpr (EPI == EPI_STORE) {
+        o.out[(int64_t)r * o.ldo + n] = v;
+      } else if constexpr (EPI == EPI_SWIGLU) {
+        o.out[(int64_t)r * o.ldo + n] = silu_f(v) * v2;
+      } else {
+        const int hr = o.map ? o.map[r] : r;
+        o.h[(int64_t)hr * N + n] += v;
+      }
     }
   }
 }
 
 // Rows are taken 8 at a time (fewer for the last chunk, dispatched to a body
 // compiled for that count).  With skip_above > 0 the kernel does nothing when
-// the row count exceeds it (the tiled GEMM launched beside it takes those).
-template <int FMT, int EPI>
+// the row count exceeds it (the tensor-core kernel launched beside it takes
+// those).  A CTA covers GEMV_WARPS * RPW output features.
+template <int FMT, int EPI, int RPW>
 __global__ void __launch_bounds__(GEMV_WARPS * 32)
 gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
             int skip_above) {
@@ -332,14 +388,14 @@ gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, Mat
     }
     __syncthreads();
     switch (nr) {
-      case 1: gemv_rows<FMT, 1, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      case 2: gemv_rows<FMT, 2, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      case 3: gemv_rows<FMT, 3, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      case 4: gemv_rows<FMT, 4, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      case 5: gemv_rows<FMT, 5, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      case 6: gemv_rows<FMT, 6, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      case 7: gemv_rows<FMT, 7, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
-      default: gemv_rows<FMT, 8, EPI>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 1: gemv_rows<FMT, 1, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 2: gemv_rows<FMT, 2, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 3: gemv_rows<FMT, 3, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 4: gemv_rows<FMT, 4, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 5: gemv_rows<FMT, 5, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 6: gemv_rows<FMT, 6, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      case 7: gemv_rows<FMT, 7, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
+      default: gemv_rows<FMT, 8, EPI, RPW>(xs, r0, rows, W, W2, o, best_v, best_i); break;
     }
   }
 }
@@ -381,35 +437,45 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
 // ------------------------------------------------------------- attention ----
 //
 // o[r][h] = softmax(q k^T / sqrt(hd)) v over positions 0..pos of the row's
-// (lane, slot) cache.  One CTA of 4 warps per (row, head); warp w takes key
-// blocks w, w+4, ... of 32 keys (one key per lane for the scores, then every
-// lane owns hd/32 output dimensions for the value sum); running max and sum are
-// kept per warp and merged at the end.  Requires kv_page_tokens >= 32 so a key
-// block never straddles a page.
+// (lane, slot) cache.  One CTA of 4 warps per (row, head, split): the key
+// blocks of 32 positions are divided into S contiguous ranges, S chosen on the
+// device from the live row count so that few rows still spread over the SMs
+// (S <= gridDim.z).  Inside a CTA warp w takes blocks w, w+4, ...: one key per
+// lane for the scores, then every lane owns hd/32 output dimensions for the
+// value sum (all 32 value loads of a block issued together); running max and
+// sum are merged across warps, and across splits by the last CTA of the
+// (row, head) to finish, in split order.  Requires kv_page_tokens >= 32.
 template <int HD>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows, KVGeom g,
-                   int slot_base, int slot_stride, const int32_t* __restrict__ map_lane, int32_t* __restrict__ status) {
+                   int slot_base, int slot_stride, float* __restrict__ part, int32_t* __restrict__ counters,
+                   int32_t* __restrict__ status) {
   constexpr int DPL = HD / 32;  // output dims per lane
   __shared__ float qs[HD];
   __shared__ float wm[4], wl[4];
   __shared__ float wacc[4][HD];
-  const int r = blockIdx.x, h = blockIdx.y;
-  if (r >= rows.n[0]) return;
+  __shared__ int last_s;
+  const int r = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
+  const int n = rows.n[0];
+  if (r >= n) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = g.H * HD;
   const int pos = rows.pos[r];
-  const int ln = map_lane ? map_lane[r] : rows.lane[r];
+  const int ln = rows.lane[r];
   const int slot = slot_base + rows.iter[r] * slot_stride;
+  const int ctx = pos + 1;
+  const int nblk = (ctx + 31) / 32;
+  int S = (4 * 148 + n * g.H - 1) / (n * g.H);
+  S = min(min(S, (int)gridDim.z), nblk);
+  if (z >= S) return;
+  const int b0 = (z * nblk) / S, b1 = ((z + 1) * nblk) / S;
   const float scale = rsqrtf((float)HD);
   for (int i = threadIdx.x; i < HD; i += blockDim.x) qs[i] = q[(int64_t)r * d + h * HD + i] * scale;
   __syncthreads();
-  const int ctx = pos + 1;
-  const int nblk = (ctx + 31) / 32;
   float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  for (int kb = warp; kb < nblk; kb += 4) {
+  for (int kb = b0 + warp; kb < b1; kb += 4) {
     const __half* kbase = kv_k_ptr(g, ln, slot, kb * 32, h, status);
     if (!kbase) break;
     const __half* vbase = kbase + (int64_t)g.H * g.page_tokens * HD;
@@ -417,11 +483,13 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* _
     float s = -INFINITY;
     if (j < ctx) {
       const uint4* kr = reinterpret_cast<const uint4*>(kbase + (int64_t)lane * HD);
+      uint4 kv[HD / 8];
+#pragma unroll
+      for (int c = 0; c < HD / 8; ++c) kv[c] = kr[c];
       float dot = 0.f;
 #pragma unroll
       for (int c = 0; c < HD / 8; ++c) {
-        const uint4 v = kr[c];
-        const __half2* hv = reinterpret_cast<const __half2*>(&v);
+        const __half2* hv = reinterpret_cast<const __half2*>(&kv[c]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __half22float2(hv[e]);
@@ -440,11 +508,21 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* _
     for (int e = 0; e < DPL; ++e) acc[e] *= corr;
     m = mn;
     const int nk = min(32, ctx - kb * 32);
-    for (int jj = 0; jj < nk; ++jj) {
-      const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const __half* vr = vbase + (int64_t)jj * HD + lane * DPL;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pj, __half2float(vr[e]), acc[e]);
+    for (int half = 0; half < 2; ++half) {
+      float vv[16][DPL];
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const __half* vr = vbase + (int64_t)(16 * half + jj) * HD + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) vv[jj][e] = (16 * half + jj < nk) ? __half2float(vr[e]) : 0.f;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const float pj = __shfl_sync(0xffffffffu, p, 16 * half + jj);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pj, vv[jj][e], acc[e]);
+      }
     }
   }
   if (lane == 0) { wm[warp] = m; wl[warp] = l; }
@@ -459,12 +537,47 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* _
     f[w] = (wm[w] == -INFINITY) ? 0.f : expf(wm[w] - M);
     Lsum += wl[w] * f[w];
   }
+  if (S == 1) {
+    for (int i = threadIdx.x; i < HD; i += blockDim.x) {
+      float v = 0.f;
+      for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
+      o[(int64_t)r * d + h * HD + i] = v / Lsum;
+      o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lsum);
+    }
+    return;
+  }
+  // split partial: (max, sum, unnormalised output) for this key range
+  float* mine = part + (((int64_t)r * g.H + h) * gridDim.z + z) * (HD + 2);
   for (int i = threadIdx.x; i < HD; i += blockDim.x) {
     float v = 0.f;
     for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
-    o[(int64_t)r * d + h * HD + i] = v / Lsum;
-    o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lsum);
+    mine[2 + i] = v;
   }
+  if (threadIdx.x == 0) { mine[0] = M; mine[1] = Lsum; }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = (atomicAdd(&counters[r * g.H + h], 1) == S - 1);
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  const float* base = part + ((int64_t)r * g.H + h) * gridDim.z * (HD + 2);
+  float Mx = -INFINITY;
+  for (int zz = 0; zz < S; ++zz) Mx = fmaxf(Mx, __ldcg(base + zz * (HD + 2)));
+  float Lt = 0.f;
+  for (int zz = 0; zz < S; ++zz) {
+    const float mz = __ldcg(base + zz * (HD + 2));
+    Lt += __ldcg(base + zz * (HD + 2) + 1) * ((mz == -INFINITY) ? 0.f : expf(mz - Mx));
+  }
+  for (int i = threadIdx.x; i < HD; i += blockDim.x) {
+    float v = 0.f;
+    for (int zz = 0; zz < S; ++zz) {
+      const float mz = __ldcg(base + zz * (HD + 2));
+      v += __ldcg(base + zz * (HD + 2) + 2 + i) * ((mz == -INFINITY) ? 0.f : expf(mz - Mx));
+    }
+    o[(int64_t)r * d + h * HD + i] = v / Lt;
+    o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lt);
+  }
+  if (threadIdx.x == 0) counters[r * g.H + h] = 0;
 }
 
 // --------------------------------------------------- prefill attention ----

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "host_util.h"
+#include "gemv_stream.cuh"
 #include "kernels.cuh"
 #include "tc_gemm.cuh"
 
@@ -88,50 +89,82 @@ static size_t blob_bytes(const tl_config* c) {
 // ------------------------------------------------- tensor-core tiling ----
 
 constexpr int kGemvMaxRows = 8;  // row counts the CUDA-core GEMV takes; more go to the tensor cores
+// head GEMV: output features per warp (its registers hold that many raw chunks
+// and 8 row accumulators each)
+constexpr int head_rpw(int fmt) { return fmt == TL_FMT_INT4 ? 4 : 2; }
+constexpr int kAttnSplits = 8;   // largest split of the context in decode attention
 
 static int tc_nt(int max_rows) { return max_rows <= 64 ? 64 : (max_rows <= 128 ? 128 : 256); }
 
-// Split of the K loop so that the grid fills the 148 SMs (two CTAs per SM fit
-// for the smaller tiles).  Every split keeps >= 2 k-blocks and its INT4 scale
-// groups within TC_SC_MAX.
+template <int NMAT, int FMT>
+static bool tc_split_ok(int nt) {
+  return nt == 64 ? TcCfg<64, NMAT, FMT>::SPLIT_OK
+                  : (nt == 128 ? TcCfg<128, NMAT, FMT>::SPLIT_OK : TcCfg<256, NMAT, FMT>::SPLIT_OK);
+}
+
+// Split of the K loop (the cluster size, <= 8) so that the grid fills the 148
+// SMs (two CTAs per SM fit for the 64-row single-matrix tile).  Every split
+// keeps >= 2 k-blocks and its INT4 scale groups within TC_SC_MAX.
 static int tc_splits(int N, int K, int max_rows, int nmat, int fmt, int group) {
   const int nt = tc_nt(max_rows);
+  const bool ok = nmat == 1 ? (fmt == TL_FMT_INT4 ? tc_split_ok<1, TL_FMT_INT4>(nt) : tc_split_ok<1, TL_FMT_BF16>(nt))
+                            : (fmt == TL_FMT_INT4 ? tc_split_ok<2, TL_FMT_INT4>(nt) : tc_split_ok<2, TL_FMT_BF16>(nt));
   const int m_tiles = (N + 127) / 128, n_tiles = (max_rows + nt - 1) / nt;
   const int kb = K / 64;
   const int slots = (nmat == 1 && nt == 64) ? 296 : 148;
   int best = 1;
-  for (int s = 1; s <= 16; ++s) {
-    if (kb % s) continue;
-    const int per = kb / s;
-    if (per < 2 && s > 1) break;
-    if (fmt == TL_FMT_INT4 && (per * 64) / group + 1 > TC_SC_MAX) continue;
+  for (int s = 2; s <= 8 && ok; ++s) {
+    if (kb % s || kb / s < 2) continue;
     if ((int64_t)m_tiles * n_tiles * s <= slots) best = s;
   }
-  if (fmt == TL_FMT_INT4)
-    while ((kb / best) * 64 / group + 1 > TC_SC_MAX && best < kb) {
-      int nb = best + 1;
-      while (kb % nb) ++nb;
-      best = nb;
-    }
   return best;
 }
 
-static size_t tc_scratch_bytes(int N, int K, int max_rows, int nmat, int fmt, int group) {
-  if (max_rows <= kGemvMaxRows) return 0;
-  const int nt = tc_nt(max_rows);
-  const int S = tc_splits(N, K, max_rows, nmat, fmt, group);
-  if (S == 1) return 0;
-  const size_t tiles = (size_t)((N + 127) / 128) * ((max_rows + nt - 1) / nt);
-  return tiles * S * nmat * nt * 128 * 4;
+// ------------------------------------------------ streamed GEMV geometry ----
+
+struct GsChoice {
+  bool ok;
+  GsPlan pl;
+  int smem, grid;
+};
+
+// Blocks of fb output features (>= 8, a multiple of 8, ~16 KB of weights) and
+// as many ring stages as fit beside the 8-row activation tile.
+static GsChoice gs_plan(int fmt, int N, int K, int group, int nmat, int n_sms) {
+  GsChoice c{};
+  const int row = fmt == TL_FMT_INT4 ? K / 2 : 2 * K;
+  const int sc = fmt == TL_FMT_INT4 ? (K / group) * 2 : 0;
+  int fb = (16384 / (row + sc)) / 8 * 8;
+  if (fb < 8) fb = 8;
+  const int stage = (fb * (row + sc) + 127) / 128 * 128;
+  const int xs = 8 * K * 4;
+  const int cap = 220 * 1024;
+  int stages = (cap - xs - 512) / (nmat * stage);
+  if (stages > 8) stages = 8;
+  if (stages < 2) return c;
+  if (((int64_t)(N % fb) * sc) % 16) return c;  // the last block's scales must be a 16-byte multiple
+  c.pl.fb = fb;
+  c.pl.stages = stages;
+  c.pl.stage_bytes = stage;
+  c.pl.row_bytes = row;
+  c.pl.sc_row_bytes = sc;
+  c.pl.xs_offset = stages * nmat * stage;
+  c.pl.bar_offset = c.pl.xs_offset + xs;
+  c.smem = c.pl.bar_offset + 2 * stages * 8 + 16;
+  const int nblocks = (N + fb - 1) / fb;
+  c.grid = nblocks < n_sms ? nblocks : n_sms;
+  c.ok = true;
+  return c;
 }
 
 // Offsets of every workspace region (computed identically by tl_workspace_bytes and tl_create).
 struct Layout {
   int n_slots, pages_per_seq, n_pages, max_rows, n_parts, max_prefill;
-  size_t page_elems, tc_scratch_size;
+  size_t page_elems;
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[4], act_a, act_qkv, act_q, act_o, act_u,
-      act_a16, act_o16, act_u16, tc_scratch, tc_counters, part_val, part_idx, tok_stage, L_stage, mask_stage,
+      act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
+      mask_stage,
       out_tok, out_dep, status, counters, alive, total;
 };
 
@@ -144,7 +177,8 @@ static Layout make_layout(const tl_config* c) {
   L.n_pages = c->kv_pool_pages ? c->kv_pool_pages : c->max_lanes * L.n_slots * L.pages_per_seq;
   L.page_elems = (size_t)2 * c->n_heads * c->kv_page_tokens * hd;
   L.max_rows = c->max_lanes > L.max_prefill ? c->max_lanes : L.max_prefill;
-  L.n_parts = (c->vocab + GEMV_WARPS - 1) / GEMV_WARPS;
+  L.n_parts = (c->vocab + GEMV_WARPS * 2 - 1) / (GEMV_WARPS * 2);  // the smallest head_rpw
+  if (L.n_parts < 1024) L.n_parts = 1024;                            // streamed GEMV: one per SM
   size_t o = 0;
   for (const auto& m : mat_specs(c)) {
     L.mat_off.push_back(o);
@@ -169,22 +203,8 @@ static Layout make_layout(const tl_config* c) {
   L.act_a16 = take(R * d * 2);
   L.act_o16 = take(R * d * 2);
   L.act_u16 = take(R * F * 2);
-  size_t scratch = 0;
-  const int top = c->max_lanes > L.max_prefill ? c->max_lanes : L.max_prefill;
-  for (int b = 0; b < 2; ++b) {
-    const int fmt = b == 0 ? c->fmt_pre : c->fmt_loop;
-    if (b == 0 && c->n_pre == 0) continue;
-    for (int mr = kGemvMaxRows + 1; mr <= top; ++mr) {
-      const size_t v[4] = {tc_scratch_bytes(3 * c->d, c->d, mr, 1, fmt, c->group),
-                           tc_scratch_bytes(c->d, c->d, mr, 1, fmt, c->group),
-                           tc_scratch_bytes(c->ffn, c->d, mr, 2, fmt, c->group),
-                           tc_scratch_bytes(c->d, c->ffn, mr, 1, fmt, c->group)};
-      for (size_t x : v) scratch = x > scratch ? x : scratch;
-    }
-  }
-  L.tc_scratch_size = scratch;
-  L.tc_scratch = take(scratch ? scratch : 256);
-  L.tc_counters = take(4096 * 4);
+  L.attn_part = take(lanes * c->n_heads * kAttnSplits * (hd + 2) * 4);
+  L.attn_counters = take(lanes * c->n_heads * 4);
   L.part_val = take(lanes * L.n_parts * 4);
   L.part_idx = take(lanes * L.n_parts * 4);
   L.tok_stage = take(R * 4);
@@ -228,8 +248,8 @@ struct tl_ctx {
   Rows rows[4];  // 0 loop, 1 boundary, 2 entered, 3 prefill / mask
   float *act_a, *act_qkv, *act_q, *act_o, *act_u;
   __half *act_a16, *act_o16, *act_u16;
-  float* tc_scratch;
-  int32_t* tc_counters;
+  float* attn_part;
+  int32_t* attn_counters;
   CUtensorMap xmap[3][3];  // [a16, o16, u16][NT 64, 128, 256]
   float* part_val;
   int32_t* part_idx;
@@ -237,6 +257,15 @@ struct tl_ctx {
   uint8_t* mask_stage;
   unsigned long long* counters;  // 0 lane iterations, 1 tokens
   EEParams ee{0.0, 2, 0, 1, 0};
+  int n_sms = 148;
+  int head_parts = 0;  // partial results per row written by the head projection
+  // CUDA graph of one decode tick (captured on cap_stream, replayed on stream)
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t tick_exec = nullptr;
+  int tick_lanes = 0, tick_new = 0;
+  int32_t *tick_tok = nullptr, *tick_dep = nullptr;
+  EEParams tick_ee{};
+  int64_t tick_launches = 0;
   // host state
   std::vector<int32_t> h_page_table;  // [lanes][slots][pages]
   std::vector<int32_t> refcount;      // per page
@@ -296,20 +325,47 @@ int prof_stop(tl_ctx* c, int kind) {
   return TL_OK;
 }
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int RPW = 1>
 int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView& W, const MatView& W2,
                 const ProjOut& o, int skip_above) {
   const size_t smem = (size_t)8 * W.K * 4;
-  auto kern = gemv_kernel<FMT, EPI>;
+  auto kern = gemv_kernel<FMT, EPI, RPW>;
   static bool attr_done = false;  // once per instantiation
   if (!attr_done) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
     attr_done = true;
   }
   if (smem > 200 * 1024) return TL_EINVAL;
-  const unsigned grid = (unsigned)((W.N + GEMV_WARPS - 1) / GEMV_WARPS);
+  const unsigned grid = (unsigned)((W.N + GEMV_WARPS * RPW - 1) / (GEMV_WARPS * RPW));
   kern<<<grid, GEMV_WARPS * 32, smem, c->stream>>>(X, n_rows, W, W2, o, skip_above);
   return launch_err(c);
+}
+
+template <int FMT, int EPI>
+int gemv_stream_launch(tl_ctx* c, const GsChoice& g, const float* X, const int32_t* n_rows, const MatView& W,
+                       const MatView& W2, const ProjOut& o, int skip_above) {
+  auto kern = gemv_stream_kernel<FMT, EPI>;
+  static int attr_smem = 0;  // per instantiation: largest opt-in requested so far
+  if (g.smem > attr_smem) {
+    TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem));
+    attr_smem = g.smem;
+  }
+  kern<<<g.grid, GS_THREADS, g.smem, c->stream>>>(X, n_rows, W, W2, o, skip_above, g.pl, c->status);
+  return launch_err(c);
+}
+
+// Few-row projection: the streamed GEMV where its ring fits, else the
+// register-blocked CUDA-core GEMV.
+template <int FMT, int EPI, int RPW>
+int small_rows_proj(tl_ctx* c, const float* X, const int32_t* n, const MatView& W, const MatView& W2, ProjOut o,
+                    int skip) {
+  const GsChoice g = gs_plan(FMT, W.N, W.K, W.group, EPI == EPI_SWIGLU ? 2 : 1, c->n_sms);
+  if (g.ok) {
+    if (EPI == EPI_ARGMAX) o.n_parts = g.grid;
+    return gemv_stream_launch<FMT, EPI>(c, g, X, n, W, W2, o, skip);
+  }
+  if (EPI == EPI_ARGMAX) o.n_parts = (W.N + GEMV_WARPS * RPW - 1) / (GEMV_WARPS * RPW);
+  return gemv_launch<FMT, EPI, RPW>(c, X, n, W, W2, o, skip);
 }
 
 template <int NT, int NMAT, int FMT, int EPI>
@@ -322,7 +378,19 @@ int tc_launch_t(tl_ctx* c, const CUtensorMap& mw, const CUtensorMap& mw2, const 
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
     attr_done = true;
   }
-  kern<<<grid, 256, Cf::SMEM, c->stream>>>(mw, mw2, mx, p);
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = grid;
+  lc.blockDim = dim3(256, 1, 1);
+  lc.dynamicSmemBytes = Cf::SMEM;
+  lc.stream = c->stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;  // the split-K CTAs of a tile share a cluster
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = grid.z;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  TL_CUDA(cudaLaunchKernelEx(&lc, kern, mw, mw2, mx, p));
   return launch_err(c);
 }
 
@@ -342,8 +410,6 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   const int nt = tc_nt(max_rows);
   const int S = tc_splits(W.N, W.K, max_rows, nmat, W.fmt, W.group);
   dim3 grid((W.N + 127) / 128, (max_rows + nt - 1) / nt, S);
-  if ((size_t)grid.x * grid.y > 4096) return TL_EINVAL;
-  if (S > 1 && (size_t)grid.x * grid.y * S * nmat * nt * 128 * 4 > c->lay.tc_scratch_size) return TL_ENOMEM;
   TcParams p{};
   p.n_rows = n;
   p.skip_at_or_below = skip;
@@ -355,8 +421,6 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   p.scales2 = W2 ? W2->s : nullptr;
   p.o = o;
   p.out16 = out16;
-  p.scratch = c->tc_scratch;
-  p.counters = c->tc_counters;
   p.status = c->status;
   const CUtensorMap& mx = c->xmap[xsel][nt == 64 ? 0 : (nt == 128 ? 1 : 2)];
   const CUtensorMap& m2 = mw2 ? *mw2 : mw;
@@ -384,23 +448,22 @@ int proj(tl_ctx* c, int max_rows, bool exact, const float* X, int xsel, const in
   const bool argmax = o.epi == EPI_ARGMAX;
   const bool use_tc = !argmax && max_rows > kGemvMaxRows;
   const bool use_gemv = argmax || !use_tc || !exact;
-  if (argmax) o.n_parts = (W.N + GEMV_WARPS - 1) / GEMV_WARPS;
   if (use_gemv) {
     const int skip = use_tc ? kGemvMaxRows : 0;
     int st;
     if (W.fmt == TL_FMT_INT4) {
       switch (o.epi) {
-        case EPI_STORE: st = gemv_launch<TL_FMT_INT4, EPI_STORE>(c, X, n, W, w2, o, skip); break;
-        case EPI_RESID: st = gemv_launch<TL_FMT_INT4, EPI_RESID>(c, X, n, W, w2, o, skip); break;
-        case EPI_SWIGLU: st = gemv_launch<TL_FMT_INT4, EPI_SWIGLU>(c, X, n, W, w2, o, skip); break;
-        default: st = gemv_launch<TL_FMT_INT4, EPI_ARGMAX>(c, X, n, W, w2, o, skip); break;
+        case EPI_STORE: st = small_rows_proj<TL_FMT_INT4, EPI_STORE, 1>(c, X, n, W, w2, o, skip); break;
+        case EPI_RESID: st = small_rows_proj<TL_FMT_INT4, EPI_RESID, 1>(c, X, n, W, w2, o, skip); break;
+        case EPI_SWIGLU: st = small_rows_proj<TL_FMT_INT4, EPI_SWIGLU, 1>(c, X, n, W, w2, o, skip); break;
+        default: st = small_rows_proj<TL_FMT_INT4, EPI_ARGMAX, head_rpw(TL_FMT_INT4)>(c, X, n, W, w2, o, skip); break;
       }
     } else {
       switch (o.epi) {
-        case EPI_STORE: st = gemv_launch<TL_FMT_BF16, EPI_STORE>(c, X, n, W, w2, o, skip); break;
-        case EPI_RESID: st = gemv_launch<TL_FMT_BF16, EPI_RESID>(c, X, n, W, w2, o, skip); break;
-        case EPI_SWIGLU: st = gemv_launch<TL_FMT_BF16, EPI_SWIGLU>(c, X, n, W, w2, o, skip); break;
-        default: st = gemv_launch<TL_FMT_BF16, EPI_ARGMAX>(c, X, n, W, w2, o, skip); break;
+        case EPI_STORE: st = small_rows_proj<TL_FMT_BF16, EPI_STORE, 1>(c, X, n, W, w2, o, skip); break;
+        case EPI_RESID: st = small_rows_proj<TL_FMT_BF16, EPI_RESID, 1>(c, X, n, W, w2, o, skip); break;
+        case EPI_SWIGLU: st = small_rows_proj<TL_FMT_BF16, EPI_SWIGLU, 1>(c, X, n, W, w2, o, skip); break;
+        default: st = small_rows_proj<TL_FMT_BF16, EPI_ARGMAX, head_rpw(TL_FMT_BF16)>(c, X, n, W, w2, o, skip); break;
       }
     }
     TL_TRY(st);
@@ -411,11 +474,15 @@ int proj(tl_ctx* c, int max_rows, bool exact, const float* X, int xsel, const in
 
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
   TL_TRY(prof_start(c, TL_PROF_ATTN));
-  dim3 grid(max_rows, c->cfg.n_heads);
+  // splits beyond what max_rows * heads needs to fill the GPU are never used
+  int ks = (4 * 148 + max_rows * c->cfg.n_heads - 1) / (max_rows * c->cfg.n_heads);
+  ks = ks < 1 ? 1 : (ks > kAttnSplits ? kAttnSplits : ks);
+  if (max_rows > 1) ks = kAttnSplits < 4 ? kAttnSplits : (ks < 4 ? 4 : ks);
+  dim3 grid(max_rows, c->cfg.n_heads, ks);
   switch (c->hd) {
-    case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
-    case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
-    default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, nullptr, c->status); break;
+    case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
+    case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
+    default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
   }
   TL_TRY(launch_err(c));
   return prof_stop(c, TL_PROF_ATTN);
@@ -455,7 +522,8 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
               int slot_base, int slot_stride, float* h_in, bool prompt = false) {
   const int d = c->cfg.d, F = c->cfg.ffn;
   const float eps = c->cfg.rms_eps;
-  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in, c->act_a16);
+  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in, c->act_a16,
+                                                       nullptr, 0);
   TL_TRY(launch_err(c));
   ProjOut o{};
   o.epi = EPI_STORE;
@@ -475,7 +543,7 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   r.map = map;
   TL_TRY(proj(c, max_rows, prompt, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
   rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr,
-                                                       c->act_a16);
+                                                       c->act_a16, nullptr, 0);
   TL_TRY(launch_err(c));
   ProjOut sw{};
   sw.epi = EPI_SWIGLU;
@@ -520,7 +588,7 @@ int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax
                int32_t* dep_out, int n_new) {
   const Rows& B = c->rows[1];
   rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(c->h, B.lane, B.n, c->cfg.d, c->g_final, c->cfg.rms_eps,
-                                                       c->act_a, nullptr, nullptr);
+                                                       c->act_a, nullptr, nullptr, nullptr, 0);
   TL_TRY(launch_err(c));
   ProjOut o{};
   o.epi = EPI_ARGMAX;
@@ -530,7 +598,7 @@ int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax
   o.part_val = c->part_val;
   o.part_idx = c->part_idx;
   TL_TRY(proj(c, max_rows, false, c->act_a, 0, B.n, c->head, nullptr, nullptr, nullptr, o, nullptr, TL_PROF_HEAD));
-  const int n_parts = (c->cfg.vocab + GEMV_WARPS - 1) / GEMV_WARPS;
+  const int n_parts = c->head_parts;
   head_finalize_kernel<<<max_rows, 256, 0, c->stream>>>(B, c->lanes, c->part_val, c->part_idx, n_parts, mode, argmax,
                                                         tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
                                                         c->cfg.max_seq, c->status, &c->counters[1]);
@@ -739,8 +807,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->act_a16 = (__half*)(w + lay.act_a16);
   c->act_o16 = (__half*)(w + lay.act_o16);
   c->act_u16 = (__half*)(w + lay.act_u16);
-  c->tc_scratch = (float*)(w + lay.tc_scratch);
-  c->tc_counters = (int32_t*)(w + lay.tc_counters);
+  c->attn_part = (float*)(w + lay.attn_part);
+  c->attn_counters = (int32_t*)(w + lay.attn_counters);
   c->part_val = (float*)(w + lay.part_val);
   c->part_idx = (int32_t*)(w + lay.part_idx);
   c->tok_stage = (int32_t*)(w + lay.tok_stage);
@@ -751,6 +819,14 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->status = (int32_t*)(w + lay.status);
   c->counters = (unsigned long long*)(w + lay.counters);
   c->alive = (int32_t*)(w + lay.alive);
+  {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+      c->n_sms = sms;
+    const GsChoice g = gs_plan(c->head.fmt, c->head.N, c->head.K, c->head.group, 1, c->n_sms);
+    const int rpw = head_rpw(c->head.fmt);
+    c->head_parts = g.ok ? g.grid : (c->head.N + GEMV_WARPS * rpw - 1) / (GEMV_WARPS * rpw);
+  }
   // host-side page allocator
   const size_t per_lane = (size_t)lay.n_slots * lay.pages_per_seq;
   c->h_page_table.assign(per_lane * cfg->max_lanes, -1);
@@ -770,7 +846,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     if ((st = check_cuda(cudaMemsetAsync(w + lay.page_table, 0xFF, per_lane * cfg->max_lanes * 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->status, 0, 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->counters, 0, 32, c->stream))) != TL_OK) break;
-    if ((st = check_cuda(cudaMemsetAsync(c->tc_counters, 0, 4096 * 4, c->stream))) != TL_OK) break;
+    if ((st = check_cuda(cudaMemsetAsync(c->attn_counters, 0, (size_t)cfg->max_lanes * cfg->n_heads * 4, c->stream))) != TL_OK) break;
     if ((st = encode_all_maps(c)) != TL_OK) break;
     for (int i = 0; i < 4; ++i)
       if ((st = check_cuda(cudaMemsetAsync(c->rows[i].n, 0, 4, c->stream))) != TL_OK) break;
@@ -778,6 +854,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     if ((st = check_cuda(cudaHostAlloc((void**)&c->pinned_alive, kAliveRing * sizeof(int32_t), cudaHostAllocDefault))) != TL_OK) break;
     for (int i = 0; i < kAliveRing; ++i)
       if ((st = check_cuda(cudaEventCreateWithFlags(&c->alive_ev[i], cudaEventDisableTiming))) != TL_OK) break;
+    if (st != TL_OK) break;
+    if ((st = check_cuda(cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking))) != TL_OK) break;
   } while (0);
   if (st != TL_OK) {
     if (c->pinned_alive) cudaFreeHost(c->pinned_alive);
@@ -791,6 +869,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
 extern "C" int tl_destroy(tl_ctx* c) {
   if (!c) return TL_EINVAL;
   cudaStreamSynchronize(c->stream);
+  if (c->tick_exec) cudaGraphExecDestroy(c->tick_exec);
+  if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
   for (int i = 0; i < kAliveRing; ++i) cudaEventDestroy(c->alive_ev[i]);
   for (auto& e : c->prof_ev) {
     cudaEventDestroy(e[0]);
@@ -933,28 +1013,85 @@ extern "C" int tl_embed_next(tl_ctx* c, const uint8_t* dev_mask, const int32_t* 
   return pre_blocks_for_entered(c, c->cfg.max_lanes);
 }
 
+// One decode tick: boundary stage (head, tokens, embedding, pre blocks) for
+// lanes whose loop finished, then one loop iteration for lanes in their loop.
+static int enqueue_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
+  TL_TRY(build_rows(c, 1, SEL_BOUNDARY, nullptr, nullptr, nullptr, c->alive, n_lanes));
+  TL_TRY(head_stage(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new));
+  TL_TRY(build_rows(c, 0, SEL_LOOP, nullptr, nullptr, nullptr, nullptr, n_lanes));
+  return loop_iteration(c, n_lanes, nullptr);
+}
+
+static bool same_ee(const EEParams& a, const EEParams& b) {
+  return a.tau == b.tau && a.min_L == b.min_L && a.patience == b.patience && a.peek_every == b.peek_every &&
+         a.enabled == b.enabled;
+}
+
+// The tick as a CUDA graph: every kernel reads its row count from device
+// memory, so one capture serves every tick of a decode with the same lanes,
+// token budget, outputs and early-exit parameters.
+static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
+  if (c->tick_exec && c->tick_lanes == n_lanes && c->tick_new == n_new && c->tick_tok == tok_out &&
+      c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee))
+    return TL_OK;
+  if (c->tick_exec) {
+    cudaGraphExecDestroy(c->tick_exec);
+    c->tick_exec = nullptr;
+  }
+  const int64_t l0 = c->launches, s0 = c->steps;
+  cudaStream_t saved = c->stream;
+  TL_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
+  c->stream = c->cap_stream;
+  const int st = enqueue_tick(c, n_lanes, n_new, tok_out, dep_out);
+  c->stream = saved;
+  cudaGraph_t g = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
+  const int64_t per_tick = c->launches - l0;
+  c->launches = l0;
+  c->steps = s0;
+  if (st != TL_OK) {
+    if (g) cudaGraphDestroy(g);
+    return st;
+  }
+  TL_CUDA(e);
+  const cudaError_t ei = cudaGraphInstantiate(&c->tick_exec, g, 0);
+  cudaGraphDestroy(g);
+  TL_CUDA(ei);
+  c->tick_lanes = n_lanes;
+  c->tick_new = n_new;
+  c->tick_tok = tok_out;
+  c->tick_dep = dep_out;
+  c->tick_ee = c->ee;
+  c->tick_launches = per_tick;
+  return TL_OK;
+}
+
 static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
   decode_init_kernel<<<(n_lanes + 255) / 256, 256, 0, c->stream>>>(c->lanes, n_lanes, c->L_stage, n_new, c->status);
   TL_TRY(launch_err(c));
+  // per-kind event profiling needs individual launches; otherwise replay a captured tick
+  const bool graphs = c->prof_mask == 0;
+  if (graphs) TL_TRY(tick_graph(c, n_lanes, n_new, tok_out, dep_out));
   // upper bound on ticks: every token runs at most L_max iterations, plus the first
   const int64_t max_ticks = (int64_t)n_new * (c->cfg.L_max + 1) + 4;
-  int64_t polled = 0;
   for (int64_t t = 0; t < max_ticks; ++t) {
     // lagged poll: tick t - (ring-1) must be known before launching tick t
     if (t >= kAliveRing - 1) {
       const int64_t q = t - (kAliveRing - 1);
       TL_CUDA(cudaEventSynchronize(c->alive_ev[q % kAliveRing]));
-      polled = q;
       if (c->pinned_alive[q % kAliveRing] == 0) break;
     }
-    TL_TRY(build_rows(c, 1, SEL_BOUNDARY, nullptr, nullptr, nullptr, c->alive, n_lanes));
+    if (graphs) {
+      TL_CUDA(cudaGraphLaunch(c->tick_exec, c->stream));
+      c->launches += c->tick_launches;
+      c->steps++;
+    } else {
+      TL_TRY(enqueue_tick(c, n_lanes, n_new, tok_out, dep_out));
+    }
+    // the alive count was written by the tick's first kernel
     TL_CUDA(cudaMemcpyAsync(&c->pinned_alive[t % kAliveRing], c->alive, 4, cudaMemcpyDeviceToHost, c->stream));
     TL_CUDA(cudaEventRecord(c->alive_ev[t % kAliveRing], c->stream));
-    TL_TRY(head_stage(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new));
-    TL_TRY(build_rows(c, 0, SEL_LOOP, nullptr, nullptr, nullptr, nullptr, n_lanes));
-    TL_TRY(loop_iteration(c, n_lanes, nullptr));
   }
-  (void)polled;
   return TL_OK;
 }
 

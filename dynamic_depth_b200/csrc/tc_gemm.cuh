@@ -12,20 +12,23 @@
 // fp16) and later run the epilogue; warp 1 issues tcgen05.mma (K = 16 per
 // instruction, 4 per 64-wide k-block) into a TMEM accumulator and commits each
 // stage back to the producer; warp 2 owns the TMEM allocation.  Split-K CTAs
-// write fp32 partials to scratch and the last CTA of a tile (arrival counter)
-// sums them in split order and applies the epilogue, so results do not depend
-// on CTA timing.  Every mbarrier wait is bounded (~1.5 s of %globaltimer);
-// on expiry the CTA records ST_TIMEOUT in the status word and unwinds.
+// of one output tile form a thread-block cluster: each parks its fp32 partial
+// tile in its own shared memory, and after a cluster barrier CTA z reduces the
+// z-th slice of the tile's rows over the cluster's shared memory in split
+// order (deterministic, no global scratch) and applies the epilogue (store,
+// residual add, or silu(gate) * up).  Every mbarrier wait is bounded (~1.5 s
+// of %globaltimer); on expiry the CTA records ST_TIMEOUT in the status word and
+// still reaches both cluster barriers.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace tl {
-
-constexpr int ST_TIMEOUT = 1 << 6;
 
 struct TcParams {
   const int32_t* n_rows;   // device scalar
@@ -34,10 +37,8 @@ struct TcParams {
   int32_t kb_per_split;    // 64-wide k-blocks per split
   const __half* scales;    // INT4: [N][K/group]
   const __half* scales2;   // second matrix (gate/up pair)
-  ProjOut o;
-  __half* out16;           // fp16 copy of EPI_STORE / EPI_SWIGLU rows (ld = o.ldo), nullable
-  float* scratch;          // split-K partials
-  int32_t* counters;       // per-tile arrivals, zero between launches
+  ProjOut o;               // EPI_STORE / EPI_SWIGLU: o.out [rows][ldo]; EPI_RESID: o.h / o.map
+  __half* out16;           // fp16 copy of the EPI_SWIGLU output (the next projection's operand)
   int32_t* status;
 };
 
@@ -56,59 +57,10 @@ struct TcCfg {
   static constexpr int STAGES = ((220 * 1024 - fixed) / stage_bytes) >= CAP ? CAP : ((220 * 1024 - fixed) / stage_bytes);
   static constexpr int SMEM = STAGES * stage_bytes + fixed;
   static constexpr int TMEM_COLS = (NMAT * NT <= 32) ? 32 : NMAT * NT;
+  // split-K parks a [NMAT][NT][128] fp32 partial tile in the stage buffers
+  static constexpr bool SPLIT_OK = NMAT * NT * 128 * 4 <= STAGES * stage_bytes;
   static_assert(STAGES >= 2, "tile does not fit in shared memory");
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort_flag) {
-  uint64_t start = 0;
-  for (uint32_t it = 0;; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred P;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
-        "selp.b32 %0, 1, 0, P;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((it & 31) == 31) {
-      if (*abort_flag) return false;
-      const uint64_t now = gtimer();
-      if (start == 0) {
-        start = now;
-      } else if (now - start > 1500000000ull) {
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
 
 // K-major, SWIZZLE_128B canonical layout: 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
@@ -173,12 +125,12 @@ __device__ __forceinline__ uint4 bf16x8_to_half8(uint4 v) {
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// Final value of one output element.
 template <int EPI>
-__device__ __forceinline__ void tc_store(const TcParams& p, int row, int m, float v, float v2) {
+__device__ __forceinline__ void tc_emit(const TcParams& p, int row, int m, float v, float v2) {
   const ProjOut& o = p.o;
   if constexpr (EPI == EPI_STORE) {
     o.out[(int64_t)row * o.ldo + m] = v;
-    if (p.out16) p.out16[(int64_t)row * o.ldo + m] = __float2half_rn(v);
   } else if constexpr (EPI == EPI_SWIGLU) {
     const float u = silu_f(v) * v2;
     o.out[(int64_t)row * o.ldo + m] = u;
@@ -208,14 +160,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
   uint64_t* accfull = bars + 3 * STAGES;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 3 * STAGES + 1);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
-  volatile int32_t* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = p.n_rows[0];
   const int m0 = blockIdx.x * 128, n0 = blockIdx.y * NT;
   if (rows <= p.skip_at_or_below || n0 >= rows) return;
   const int nkb = p.kb_per_split, kb0 = blockIdx.z * nkb;
-  const int S = gridDim.z;
+  const int S = gridDim.z;                      // split-K CTAs of this tile = cluster size
+  const int ncols = min(NT, rows - n0);
+  float* red = reinterpret_cast<float*>(sA);    // [NMAT][NT][128] partial tile after the main loop
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -225,7 +178,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     }
     mbar_init(smem_u32(accfull), 1);
     *abort_flag = 0;
-    *last_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 2) {
@@ -233,20 +185,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
                  "r"((uint32_t)C::TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  if constexpr (FMT == TL_FMT_INT4) {
-    if (warp >= 4) {
-      const int t = threadIdx.x - 128;
-      const int g = p.group;
-      const int gfirst = (kb0 * 64) / g;
-      const int glast = ((kb0 + nkb) * 64 - 1) / g;
-      for (int mat = 0; mat < NMAT; ++mat) {
-        const __half* sc = mat == 0 ? p.scales : p.scales2;
-        const int64_t rowoff = (int64_t)(m0 + t) * (p.K / g);
-        for (int j = 0; j <= glast - gfirst && j < TC_SC_MAX; ++j)
-          sSc[(mat * 128 + t) * TC_SC_MAX + j] = (m0 + t < p.N) ? sc[rowoff + gfirst + j] : __float2half(0.f);
-      }
-    }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -304,6 +242,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     const int t = threadIdx.x - 128;  // weight row within the tile == TMEM lane
     const int q = warp - 4;
     const int gfirst = (FMT == TL_FMT_INT4) ? (kb0 * 64) / p.group : 0;
+    if constexpr (FMT == TL_FMT_INT4) {
+      // this row's group scales for the CTA's K range (while the first TMA is in flight)
+      const int glast = ((kb0 + nkb) * 64 - 1) / p.group;
+      for (int mat = 0; mat < NMAT; ++mat) {
+        const __half* sc = mat == 0 ? p.scales : p.scales2;
+        const int64_t rowoff = (int64_t)(m0 + t) * (p.K / p.group);
+        for (int j = 0; j <= glast - gfirst && j < TC_SC_MAX; ++j)
+          sSc[(mat * 128 + t) * TC_SC_MAX + j] = (m0 + t < p.N) ? sc[rowoff + gfirst + j] : __float2half(0.f);
+      }
+    }
     bool ok = true;
     for (int i = 0; i < nkb && ok; ++i) {
       const int s = i % STAGES, r = i / STAGES;
@@ -338,46 +286,45 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     if (ok && mbar_wait(smem_u32(accfull), 0, abort_flag)) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int m = m0 + t;
-      const int ncols = min(NT, rows - n0);
-      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
       const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
       for (int j = 0; j < ncols; j += 8) {
         float v[8], v2[8];
         tmem_ld8(tl + j, v);
         if constexpr (NMAT == 2) tmem_ld8(tl + NT + j, v2);
         if (S == 1) {
+          if (m < p.N) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (j + e < ncols && m < p.N) tc_store<EPI>(p, n0 + j + e, m, v[e], NMAT == 2 ? v2[e] : 0.f);
+            for (int e = 0; e < 8; ++e)
+              if (j + e < ncols) tc_emit<EPI>(p, n0 + j + e, m, v[e], NMAT == 2 ? v2[e] : 0.f);
+          }
         } else {
-          float* part = p.scratch + ((int64_t)(tile * S + blockIdx.z) * NMAT) * NT * 128;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            part[(j + e) * 128 + t] = v[e];
-            if constexpr (NMAT == 2) part[NT * 128 + (j + e) * 128 + t] = v2[e];
+            red[(j + e) * 128 + t] = v[e];
+            if constexpr (NMAT == 2) red[(NT + j + e) * 128 + t] = v2[e];
           }
-        }
-      }
-      if (S > 1) {
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (t == 0) *last_flag = (atomicAdd(&p.counters[tile], 1) == S - 1) ? 1 : 0;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (*last_flag) {
-          __threadfence();
-          for (int j = 0; j < ncols; ++j) {
-            float a = 0.f, b = 0.f;
-            for (int z = 0; z < S; ++z) {
-              const float* part = p.scratch + ((int64_t)(tile * S + z) * NMAT) * NT * 128;
-              a += __ldcg(part + j * 128 + t);
-              if constexpr (NMAT == 2) b += __ldcg(part + NT * 128 + j * 128 + t);
-            }
-            if (m < p.N) tc_store<EPI>(p, n0 + j, m, a, b);
-          }
-          if (t == 0) p.counters[tile] = 0;
         }
       }
     }
+  }
+  if (S > 1) {
+    // split-K: reduce this CTA's slice of rows over the cluster's partial tiles
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int z = blockIdx.z;
+    const int f0 = (z * 128) / S, nf = ((z + 1) * 128) / S - f0;
+    for (int i = threadIdx.x; i < nf * ncols; i += blockDim.x) {
+      const int tt = f0 + i % nf, j = i / nf;
+      float a = 0.f, b = 0.f;
+      for (int zz = 0; zz < S; ++zz) {
+        const float* rz = cluster.map_shared_rank(red, zz);
+        a += rz[j * 128 + tt];
+        if constexpr (NMAT == 2) b += rz[(NT + j) * 128 + tt];
+      }
+      if (m0 + tt < p.N) tc_emit<EPI>(p, n0 + j, m0 + tt, a, b);
+    }
+    cluster.sync();
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
