@@ -277,6 +277,38 @@ int tl_profile_begin(tl_ctx* ctx, int32_t kind_mask);
  * by tl_prof_kind: groups timed and their summed device time in ms. */
 int tl_profile_end(tl_ctx* ctx, int64_t* out_groups, double* out_total_ms);
 
+/* ------------------------------------------------ allocation-free head -- */
+
+/* Greedy LM head for callers that cannot allocate device memory.  The pages
+ * have no counterpart for this call: it exists because some callers cannot
+ * allocate device memory at the time they need the head (a serving loop that
+ * reserved all its memory at start-up and forbids allocation afterwards, a
+ * host framework whose allocator owns every cudaMalloc, or code that runs
+ * while a stream is being captured, where cudaMalloc is not allowed), and
+ * tl_head_logits needs the scratch space of a tl_create workspace.
+ *
+ * Computes, for r < rows: logits[r] = RMSNorm(h[r]; g_final, rms_eps) W^T and
+ * argmax[r] = the lowest id among the largest logits.  Enqueued on
+ * cuda_stream; calls no cudaMalloc / cudaFree and no allocating routine.
+ *   dev_h: fp32 [rows][d] hidden rows (before the final norm);
+ *   dev_g_final: fp32 [d];
+ *   dev_head_packed: INT4 head [V][d/2] in the weight blob's packing (element
+ *     2i in the low nibble of byte i), 16-byte aligned;
+ *   dev_head_scales: fp16 bits [V][d/group];
+ *   dev_logits: NULL or fp32 [rows][V]; dev_argmax: int32 [rows].
+ * Its scratch is one fixed array in device global memory defined by the
+ * library (about 1.5 MB, held on every GPU that loads the library until the
+ * process exits): rows <= 64, d <= 4096 and V <= 262144, else TL_ENOMEM with
+ * nothing enqueued.  Every call shares that array and it keeps the last
+ * call's contents (each call writes all it reads); calls whose kernels
+ * overlap on the GPU (unordered streams) race on it.  The first call on a
+ * device looks up the array's device address with that device current; make
+ * that first call before any stream capture begins.  TL_EINVAL on NULL inputs
+ * or d, group not multiples of 32 / group not dividing d. */
+int tl_head_argmax_static(const float* dev_h, int32_t rows, const float* dev_g_final, float rms_eps,
+                          const uint8_t* dev_head_packed, const uint16_t* dev_head_scales, int32_t V,
+                          int32_t d, int32_t group, float* dev_logits, int32_t* dev_argmax, void* cuda_stream);
+
 /* -------------------------------------------------------------- misc -- */
 
 /* Counters; also reads back and clears the device status word (synchronises
