@@ -43,8 +43,10 @@ WORKLOAD = "m407_cdb64"
 
 
 def workload_config(wl):
-    return {"workload": "407M-class looped LM, 64 lanes x (512-token prompt + 128 greedy tokens), "
-                        "per-lane L ~ clamp(Poisson(8), 2, 32), rel-L2 early exit tau 0.1 / min_L 2 / patience 2",
+    return {"workload": f"407M-class looped LM, {wl.n_lanes} lanes x ({wl.prompt_len}-token prompt + {wl.n_new} "
+                        "greedy tokens), per-lane L ~ clamp(Poisson(8), 2, 32), rel-L2 early exit tau 0.1 / min_L 2 / "
+                        "patience 2" + ("" if (wl.n_lanes, wl.prompt_len, wl.n_new) == (64, 512, 128)
+                                        else " [reduced case]"),
             "model": "vocab 50257, d 1024, 16x64 heads, SwiGLU 4096, 2 pre + 1 loop block, INT4 g128",
             "lanes": wl.n_lanes, "prompt_len": wl.prompt_len, "new_tokens": wl.n_new,
             "per_lane_L": list(wl.per_lane_L), "weights": "random N(0,0.02) seed 0",
@@ -148,6 +150,22 @@ def head_weight_bytes(sh) -> int:
     return sh.vocab * sh.d // 2 + sh.vocab * (sh.d // sh.group) * 2
 
 
+def workload_from_args(args):
+    """The benchmark workload, or a reduced case of it (profiling captures) when
+    --lanes / --prompt-len / --new-tokens are given."""
+    import dataclasses
+    wl = S.workload(WORKLOAD)
+    kw = {}
+    if args.lanes:
+        kw["n_lanes"] = args.lanes
+        kw["per_lane_L"] = tuple(wl.per_lane_L[i % len(wl.per_lane_L)] for i in range(args.lanes))
+    if args.prompt_len:
+        kw["prompt_len"] = args.prompt_len
+    if args.new_tokens:
+        kw["n_new"] = args.new_tokens
+    return dataclasses.replace(wl, **kw) if kw else wl
+
+
 # -------------------------------------------------------------------- ours --
 
 def run_ours(args, rank, world, local_rank):
@@ -157,13 +175,15 @@ def run_ours(args, rank, world, local_rank):
 
     dev = f"cuda:{local_rank}"
     torch.cuda.set_device(dev)
-    wl = S.workload(WORKLOAD)
+    wl = workload_from_args(args)
     sh = wl.shape
     cfg = T.config_from_shape(sh, max_lanes=wl.n_lanes, max_seq=wl.prompt_len + wl.n_new, L_max=32,
                               max_prefill_tokens=wl.prompt_len)
     m = T.LoopedLM(cfg, dev)
     m.load_weights(Wt.build_blob(cfg, S.master_weights(sh), S.gains(sh), dev))
     m.set_early_exit(wl.ee_tau, wl.ee_min_L, wl.ee_patience, wl.ee_peek_every)
+    if args.eager:
+        m.set_graphs(False)
     P = S.prompts(wl.n_lanes, wl.prompt_len, sh.vocab)
     Ls = np.array(wl.per_lane_L, dtype=np.int32)
 
@@ -192,11 +212,13 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id(dev)) as clk:
+        torch.cuda.nvtx.range_push("timed")
         ev0.record(stream)
         for _ in range(args.steps):
             step()
         ev1.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     if world > 1:
         torch.distributed.barrier()
     st1 = m.stats()
@@ -279,6 +301,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
         "ms_per_step_profiled_pass": round(ms_profiled / args.steps, 3),
+        "launch_mode": "eager" if args.eager else "cuda graph per tick (conditional nodes)",
         "scaling": "weak", "vs_baseline": None, "dtype": "fp32 accumulate; INT4 weights; fp16 KV",
         "data": "synthetic (seeded random weights and token ids)",
         "config": dict(workload_config(wl), parallelism=f"replicas x{world} (lanes independent, no collective)"),
@@ -353,6 +376,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-mask", type=int, default=0b1110)
+    ap.add_argument("--eager", action="store_true", help="launch every kernel of a tick individually "
+                    "(for profilers that cannot look inside graphs with conditional nodes)")
+    ap.add_argument("--lanes", type=int, default=0, help="reduced case: lanes (profiling captures only)")
+    ap.add_argument("--prompt-len", type=int, default=0, help="reduced case: prompt tokens")
+    ap.add_argument("--new-tokens", type=int, default=0, help="reduced case: generated tokens")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

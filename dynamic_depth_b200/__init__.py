@@ -121,6 +121,9 @@ class LoopedLM:
               "tl_generate")
         return tok, dep
 
+    def set_graphs(self, enabled: bool):
+        check(lib().tl_set_graphs(self.h, 1 if enabled else 0), "tl_set_graphs")
+
     def lane_state_save(self):
         """Snapshot of every lane's scheduling state and hidden row (a device tensor)."""
         n = C.c_size_t()

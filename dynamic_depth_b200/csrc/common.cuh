@@ -73,6 +73,14 @@ struct KVGeom {
 
 __device__ __forceinline__ void set_status(int32_t* st, int32_t bit) { atomicOr(st, bit); }
 
+// Programmatic dependent launch: a kernel lets the next kernel of the stream
+// start its independent prologue at once (launch_dependents), and waits for
+// the previous kernel's completion and memory (wait) before it touches
+// anything that kernel or an earlier one wrote.  Both are no-ops when the
+// launch did not ask for programmatic serialization.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -118,6 +118,28 @@ __device__ __forceinline__ void gs_consume(const uint8_t* __restrict__ stage, in
   }
 }
 
+// Producer: request weight block b (and its scales) into stage s.
+template <int FMT, int NMAT>
+__device__ __forceinline__ void gs_issue(const MatView& W, const MatView& W2, const GsPlan& pl, uint8_t* ring,
+                                         uint64_t* full, int s, int rd, int b) {
+  (void)rd;
+  const int N = W.N;
+  const int nrow = min(pl.fb, N - b * pl.fb);
+  const uint32_t wbytes = (uint32_t)nrow * pl.row_bytes, sbytes = (uint32_t)nrow * pl.sc_row_bytes;
+  const uint32_t fb = smem_u32(&full[s]);
+  mbar_expect_tx(fb, NMAT * (wbytes + sbytes));
+#pragma unroll
+  for (int mat = 0; mat < NMAT; ++mat) {
+    const MatView& M = mat == 0 ? W : W2;
+    uint8_t* dst = ring + (size_t)(s * NMAT + mat) * pl.stage_bytes;
+    const uint8_t* src = (FMT == TL_FMT_INT4) ? M.q : reinterpret_cast<const uint8_t*>(M.bf);
+    bulk_load(smem_u32(dst), src + (size_t)b * pl.fb * pl.row_bytes, wbytes, fb);
+    if (FMT == TL_FMT_INT4)
+      bulk_load(smem_u32(dst + (size_t)pl.fb * pl.row_bytes),
+                reinterpret_cast<const uint8_t*>(M.s) + (size_t)b * pl.fb * pl.sc_row_bytes, sbytes, fb);
+  }
+}
+
 template <int FMT, int EPI>
 __global__ void __launch_bounds__(GS_THREADS, 1)
 gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
@@ -132,11 +154,10 @@ gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_ro
   __shared__ float best_v[GS_CONSUMERS][8];
   __shared__ int best_i[GS_CONSUMERS][8];
 
-  const int rows = n_rows[0];
-  if ((skip_above > 0 && rows > skip_above) || rows <= 0) return;
   const int K = W.K, N = W.N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblocks = (N + pl.fb - 1) / pl.fb;
+  pdl_launch_dependents();
   if ((int)blockIdx.x >= nblocks) return;
   const int my_blocks = (nblocks - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   if (threadIdx.x == 0) {
@@ -148,6 +169,21 @@ gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_ro
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // Weights depend on no earlier kernel: when this launch certainly runs (no
+  // row-count skip), the first blocks are requested before waiting for the
+  // previous kernel.
+  const int pre = (skip_above == 0) ? min(my_blocks, pl.stages) : 0;
+  if (warp == GS_CONSUMERS && lane == 0)
+    for (int i = 0; i < pre; ++i) gs_issue<FMT, NMAT>(W, W2, pl, ring, full, i, i, blockIdx.x + i * gridDim.x);
+  pdl_wait();
+  const int rows = n_rows[0];
+  if ((skip_above > 0 && rows > skip_above) || rows <= 0) {
+    if (warp == GS_CONSUMERS && lane == 0) {  // let the early copies land before leaving
+      volatile int32_t never = 0;
+      for (int i = 0; i < pre; ++i) mbar_wait(smem_u32(&full[i]), 0, &never);
+    }
+    return;
+  }
   int it = 0;  // pipeline position, continued across row chunks
   for (int r0 = 0; r0 < rows; r0 += 8) {
     const int nr = min(8, rows - r0);
@@ -162,22 +198,9 @@ gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_ro
       if (lane == 0) {
         for (int i = 0; i < my_blocks; ++i) {
           const int g = it + i, s = g % pl.stages, rd = g / pl.stages;
+          if (g < pre) continue;  // requested before the dependency wait
           if (rd > 0 && !mbar_wait(smem_u32(&empty[s]), (rd - 1) & 1, abort_flag)) break;
-          const int b = blockIdx.x + i * gridDim.x;
-          const int nrow = min(pl.fb, N - b * pl.fb);
-          const uint32_t wbytes = (uint32_t)nrow * pl.row_bytes, sbytes = (uint32_t)nrow * pl.sc_row_bytes;
-          const uint32_t fb = smem_u32(&full[s]);
-          mbar_expect_tx(fb, NMAT * (wbytes + sbytes));
-#pragma unroll
-          for (int mat = 0; mat < NMAT; ++mat) {
-            const MatView& M = mat == 0 ? W : W2;
-            uint8_t* dst = ring + (size_t)(s * NMAT + mat) * pl.stage_bytes;
-            const uint8_t* src = (FMT == TL_FMT_INT4) ? M.q : reinterpret_cast<const uint8_t*>(M.bf);
-            bulk_load(smem_u32(dst), src + (size_t)b * pl.fb * pl.row_bytes, wbytes, fb);
-            if (FMT == TL_FMT_INT4)
-              bulk_load(smem_u32(dst + (size_t)pl.fb * pl.row_bytes),
-                        reinterpret_cast<const uint8_t*>(M.s) + (size_t)b * pl.fb * pl.sc_row_bytes, sbytes, fb);
-          }
+          gs_issue<FMT, NMAT>(W, W2, pl, ring, full, s, rd, blockIdx.x + i * gridDim.x);
         }
       }
     } else {
@@ -214,6 +237,7 @@ gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_ro
     it += my_blocks;
     __syncthreads();
     if constexpr (EPI == EPI_ARGMAX) {
+      if (blockIdx.x == 0 && threadIdx.x == 0 && o.n_parts_dev) o.n_parts_dev[0] = o.n_parts;
       if (threadIdx.x < nr) {
         const int r = threadIdx.x;
         float v = best_v[0][r];

@@ -38,6 +38,7 @@ struct ProjOut {
   float* part_val;
   int32_t* part_idx;
   int32_t n_parts;
+  int32_t* n_parts_dev;  // EPI_ARGMAX: the kernel that did the work stores n_parts here
 };
 
 // Orders (value, index) pairs: larger value first, lower index on ties.
@@ -55,10 +56,20 @@ enum RowSel : int32_t { SEL_LOOP = 0, SEL_BOUNDARY = 1, SEL_ENTERED = 2, SEL_MAS
 // optional per-lane L request: a request above the lane's cap sets ST_EKV and
 // keeps the lane out; a request at or below the iterations already done
 // finishes the lane's loop without running.
+// Conditional graph nodes driven by a row table (cond_mode): 1 = IF (rows > 0);
+// 2 = SWITCH over (rows <= 8 -> body 0, CUDA-core GEMV variant; rows > 8 ->
+// body 1, tensor-core variant; no rows -> no body).  body_kernels[v] is the
+// number of kernels body v launches; it is added to *kernel_count.
+enum CondMode : int32_t { COND_NONE = 0, COND_IF = 1, COND_SWITCH = 2 };
+
 __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, int32_t sel,
                                   const uint8_t* __restrict__ mask, const int32_t* __restrict__ per_lane_L,
                                   Rows rows, uint8_t* __restrict__ exit_mask_out, int32_t* __restrict__ alive,
-                                  int32_t* __restrict__ status) {
+                                  int32_t* __restrict__ status, cudaGraphConditionalHandle cond, int32_t cond_mode,
+                                  int32_t gemv_max_rows, const int32_t* __restrict__ body_kernels,
+                                  unsigned long long* __restrict__ kernel_count) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int32_t warp_cnt[32];
   __shared__ int32_t alive_cnt;
   const int i = threadIdx.x;
@@ -122,8 +133,17 @@ __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, in
     rows.iter[r] = lanes[i].iter;
   }
   if (i == 0) {
-    rows.n[0] = warp_cnt[31];
+    const int n = warp_cnt[31];
+    rows.n[0] = n;
     if (alive) alive[0] = alive_cnt;
+    if (cond_mode == COND_IF) {
+      cudaGraphSetConditional(cond, n > 0 ? 1u : 0u);
+      if (n > 0) atomicAdd(kernel_count, (unsigned long long)body_kernels[0]);
+    } else if (cond_mode == COND_SWITCH) {
+      const unsigned v = n == 0 ? 2u : (n <= gemv_max_rows ? 0u : 1u);
+      cudaGraphSetConditional(cond, v);
+      if (v < 2) atomicAdd(kernel_count, (unsigned long long)body_kernels[v]);
+    }
   }
 }
 
@@ -138,6 +158,8 @@ __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* 
                                     const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
                                     float eps, float* __restrict__ out, float* __restrict__ h_in,
                                     __half* __restrict__ out16, float* __restrict__ zero_rows, int zero_cols) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float red[32];
   const int r = blockIdx.x;
   if (r >= n_rows[0]) return;
@@ -179,6 +201,8 @@ __device__ __forceinline__ void embed_row(const MatView& E, int tok, float* __re
 
 __global__ void embed_rows_kernel(MatView E, const int32_t* __restrict__ tokens, int n, int d,
                                   float* __restrict__ h, int32_t* __restrict__ status) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int r = blockIdx.x;
   if (r >= n) return;
   int tok = tokens[r];
@@ -372,6 +396,8 @@ template <int FMT, int EPI, int RPW>
 __global__ void __launch_bounds__(GEMV_WARPS * 32)
 gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
             int skip_above) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ float4 smem4[];
   float* xs = reinterpret_cast<float*>(smem4);
   __shared__ float best_v[GEMV_WARPS][8];
@@ -408,6 +434,8 @@ gemv_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, Mat
 __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict__ q_out, Rows rows, KVGeom g,
                                const float2* __restrict__ rope_cs, int slot_base, int slot_stride,
                                const int32_t* __restrict__ map_lane, int32_t* __restrict__ status) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int r = blockIdx.x;
   if (r >= rows.n[0]) return;
   const int d = g.H * g.hd, half = g.hd / 2;
@@ -450,6 +478,8 @@ __global__ void __launch_bounds__(128)
 attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows, KVGeom g,
                    int slot_base, int slot_stride, float* __restrict__ part, int32_t* __restrict__ counters,
                    int32_t* __restrict__ status) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int DPL = HD / 32;  // output dims per lane
   __shared__ float qs[HD];
   __shared__ float wm[4], wl[4];
@@ -480,6 +510,25 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* _
     if (!kbase) break;
     const __half* vbase = kbase + (int64_t)g.H * g.page_tokens * HD;
     const int j = kb * 32 + lane;
+    const int nk = min(32, ctx - kb * 32);
+    // the block's values, loaded together with its keys (neither depends on the scores)
+    constexpr int VW = DPL >= 2 ? DPL / 2 : 1;  // 32-bit words of values per lane per key
+    uint32_t vraw[32][VW];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) {
+      if (jj < nk) {
+        if constexpr (DPL >= 2) {
+#pragma unroll
+          for (int e = 0; e < VW; ++e)
+            vraw[jj][e] = reinterpret_cast<const uint32_t*>(vbase + (int64_t)jj * HD + lane * DPL)[e];
+        } else {
+          vraw[jj][0] = __half_as_ushort(vbase[(int64_t)jj * HD + lane]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < VW; ++e) vraw[jj][e] = 0u;
+      }
+    }
     float s = -INFINITY;
     if (j < ctx) {
       const uint4* kr = reinterpret_cast<const uint4*>(kbase + (int64_t)lane * HD);
@@ -507,21 +556,18 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* _
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[e] *= corr;
     m = mn;
-    const int nk = min(32, ctx - kb * 32);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float vv[16][DPL];
+    for (int jj = 0; jj < 32; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+      if constexpr (DPL >= 2) {
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const __half* vr = vbase + (int64_t)(16 * half + jj) * HD + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) vv[jj][e] = (16 * half + jj < nk) ? __half2float(vr[e]) : 0.f;
-      }
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const float pj = __shfl_sync(0xffffffffu, p, 16 * half + jj);
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pj, vv[jj][e], acc[e]);
+        for (int e = 0; e < VW; ++e) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vraw[jj][e]));
+          acc[2 * e] = fmaf(pj, f.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(pj, f.y, acc[2 * e + 1]);
+        }
+      } else {
+        acc[0] = fmaf(pj, __half2float(__ushort_as_half((unsigned short)vraw[jj][0])), acc[0]);
       }
     }
   }
@@ -593,6 +639,8 @@ template <int HD>
 __global__ void __launch_bounds__(256)
 attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
                     KVGeom g, int slot, int32_t* __restrict__ status) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int BQ = 64, BK = 64, DPT = HD / 16;
   extern __shared__ float4 smem_pf[];
   float* Qs = reinterpret_cast<float*>(smem_pf);  // [HD][BQ]  (pre-scaled)
@@ -735,6 +783,8 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* 
 __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ h,
                                    const float* __restrict__ h_in, int d, EEParams ee,
                                    uint8_t* __restrict__ exit_mask_out, unsigned long long* __restrict__ lane_iters) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ double red[32];
   const int r = blockIdx.x;
   if (r >= rows.n[0]) return;
@@ -780,11 +830,14 @@ enum HeadMode : int32_t { HEAD_ONLY = 0, HEAD_DECODE = 1 };
 // or moves it to its next position: cap = depth (monotonic clamp), L_run =
 // min(L_req, cap), embed the token, mark it for its pre blocks.  One CTA per row.
 __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ part_val,
-                                     const int32_t* __restrict__ part_idx, int n_parts, int32_t mode,
+                                     const int32_t* __restrict__ part_idx, const int32_t* __restrict__ n_parts_dev,
+                                     int32_t mode,
                                      int32_t* __restrict__ argmax_out, int32_t* __restrict__ tokens_out,
                                      int32_t* __restrict__ depths_out, int n_new, MatView E, float* __restrict__ h,
                                      int d, int max_seq, int32_t* __restrict__ status,
                                      unsigned long long* __restrict__ tok_count) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float sv[32];
   __shared__ int si[32];
   __shared__ int tok_s;
@@ -792,6 +845,7 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
   const int r = blockIdx.x;
   if (r >= rows.n[0]) return;
   const int ln = rows.lane[r];
+  const int n_parts = n_parts_dev[0];
   float bv = -INFINITY;
   int bi = 0x7fffffff;
   for (int p = threadIdx.x; p < n_parts; p += blockDim.x) {
@@ -846,6 +900,8 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
 __global__ void embed_next_kernel(LaneState* __restrict__ lanes, int n_lanes, const uint8_t* __restrict__ mask,
                                   const int32_t* __restrict__ tokens, MatView E, float* __restrict__ h, int d,
                                   int max_seq, int32_t* __restrict__ status) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int tok_s, go_s;
   const int ln = blockIdx.x;
   if (ln >= n_lanes) return;
@@ -879,6 +935,8 @@ __global__ void embed_next_kernel(LaneState* __restrict__ lanes, int n_lanes, co
 // the lane's cap sets ST_EKV and leaves the lane out.
 __global__ void decode_init_kernel(LaneState* __restrict__ lanes, int n_lanes, const int32_t* __restrict__ req_L,
                                    int n_new, int32_t* __restrict__ status) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n_lanes) return;
   LaneState& st = lanes[i];
@@ -897,6 +955,8 @@ __global__ void decode_init_kernel(LaneState* __restrict__ lanes, int n_lanes, c
 // hrows, position last_pos), cap = depth = L, waiting for the head.
 __global__ void prefill_finish_kernel(LaneState* __restrict__ lanes, int ln, int Tn, int last_pos, int L,
                                       const float* __restrict__ hrows, float* __restrict__ h, int d) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int k = threadIdx.x; k < d; k += blockDim.x) h[(int64_t)ln * d + k] = hrows[(int64_t)(Tn - 1) * d + k];
   if (threadIdx.x == 0) {
     LaneState& st = lanes[ln];
@@ -917,6 +977,8 @@ __global__ void prefill_finish_kernel(LaneState* __restrict__ lanes, int ln, int
 
 // Rows of a prefill: row t is position pos0 + t of lane ln at iteration 0.
 __global__ void prefill_rows_kernel(Rows rows, int ln, int pos0, int T) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
     rows.lane[t] = ln;
     rows.pos[t] = pos0 + t;

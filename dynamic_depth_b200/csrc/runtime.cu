@@ -89,6 +89,7 @@ static size_t blob_bytes(const tl_config* c) {
 // ------------------------------------------------- tensor-core tiling ----
 
 constexpr int kGemvMaxRows = 8;  // row counts the CUDA-core GEMV takes; more go to the tensor cores
+enum ProjPath { PATH_AUTO = 0, PATH_GEMV = 1, PATH_TC = 2 };
 // head GEMV: output features per warp (its registers hold that many raw chunks
 // and 8 row accumulators each)
 constexpr int head_rpw(int fmt) { return fmt == TL_FMT_INT4 ? 4 : 2; }
@@ -165,7 +166,7 @@ struct Layout {
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[4], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
       mask_stage,
-      out_tok, out_dep, status, counters, alive, total;
+      out_tok, out_dep, status, counters, body_kernels, alive, total;
 };
 
 static Layout make_layout(const tl_config* c) {
@@ -179,6 +180,7 @@ static Layout make_layout(const tl_config* c) {
   L.max_rows = c->max_lanes > L.max_prefill ? c->max_lanes : L.max_prefill;
   L.n_parts = (c->vocab + GEMV_WARPS * 2 - 1) / (GEMV_WARPS * 2);  // the smallest head_rpw
   if (L.n_parts < 1024) L.n_parts = 1024;                            // streamed GEMV: one per SM
+  if (L.n_parts < (c->vocab + 127) / 128) L.n_parts = (c->vocab + 127) / 128;  // tensor-core head: one per tile
   size_t o = 0;
   for (const auto& m : mat_specs(c)) {
     L.mat_off.push_back(o);
@@ -214,6 +216,7 @@ static Layout make_layout(const tl_config* c) {
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
   L.counters = take(4 * 8);
+  L.body_kernels = take(8 * 4);
   L.alive = take(4);
   L.total = o;
   return L;
@@ -255,17 +258,22 @@ struct tl_ctx {
   int32_t* part_idx;
   int32_t *tok_stage, *L_stage, *out_tok, *out_dep, *status, *alive;
   uint8_t* mask_stage;
-  unsigned long long* counters;  // 0 lane iterations, 1 tokens
+  unsigned long long* counters;  // 0 lane iterations, 1 tokens, 2 kernels run inside conditional graph bodies
+  int32_t* body_kernels;          // [stage][variant] kernels of each conditional body (graph ticks)
   EEParams ee{0.0, 2, 0, 1, 0};
   int n_sms = 148;
   int head_parts = 0;  // partial results per row written by the head projection
+  CUtensorMap mhead;   // TMA map of the head's raw weight tiles
+  int32_t* head_nparts;  // device: partial count written by whichever head kernel ran
   // CUDA graph of one decode tick (captured on cap_stream, replayed on stream)
-  cudaStream_t cap_stream = nullptr;
+  cudaStream_t cap_stream = nullptr, cap_body = nullptr;
   cudaGraphExec_t tick_exec = nullptr;
   int tick_lanes = 0, tick_new = 0;
   int32_t *tick_tok = nullptr, *tick_dep = nullptr;
   EEParams tick_ee{};
   int64_t tick_launches = 0;
+  bool graphs_enabled = true;
+  bool pdl = true;  // programmatic dependent launch between consecutive kernels
   // host state
   std::vector<int32_t> h_page_table;  // [lanes][slots][pages]
   std::vector<int32_t> refcount;      // per page
@@ -292,6 +300,26 @@ namespace {
 int launch_err(tl_ctx* c) {
   c->launches++;
   return check_cuda(cudaGetLastError());
+}
+
+// Every kernel of the library goes through here: cudaLaunchKernelEx with
+// programmatic stream serialization (each kernel waits for its predecessor
+// with griddepcontrol.wait before touching its outputs, and lets its successor
+// start its prologue early), unless the context turned that off.
+template <typename... KArgs, typename... Args>
+int launch_k(tl_ctx* c, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, Args... args) {
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = c->stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = c->pdl ? 1 : 0;
+  TL_CUDA(cudaLaunchKernelEx(&lc, kern, args...));
+  return launch_err(c);
 }
 
 // Per-kind device time: event pairs around every launch group of a profiled
@@ -337,8 +365,8 @@ int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView&
   }
   if (smem > 200 * 1024) return TL_EINVAL;
   const unsigned grid = (unsigned)((W.N + GEMV_WARPS * RPW - 1) / (GEMV_WARPS * RPW));
-  kern<<<grid, GEMV_WARPS * 32, smem, c->stream>>>(X, n_rows, W, W2, o, skip_above);
-  return launch_err(c);
+  TL_TRY(launch_k(c, kern, dim3(grid), dim3(GEMV_WARPS * 32), smem, X, n_rows, W, W2, o, skip_above));
+  return TL_OK;
 }
 
 template <int FMT, int EPI>
@@ -350,8 +378,8 @@ int gemv_stream_launch(tl_ctx* c, const GsChoice& g, const float* X, const int32
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem));
     attr_smem = g.smem;
   }
-  kern<<<g.grid, GS_THREADS, g.smem, c->stream>>>(X, n_rows, W, W2, o, skip_above, g.pl, c->status);
-  return launch_err(c);
+  TL_TRY(launch_k(c, kern, dim3(g.grid), dim3(GS_THREADS), g.smem, X, n_rows, W, W2, o, skip_above, g.pl, c->status));
+  return TL_OK;
 }
 
 // Few-row projection: the streamed GEMV where its ring fits, else the
@@ -383,13 +411,15 @@ int tc_launch_t(tl_ctx* c, const CUtensorMap& mw, const CUtensorMap& mw2, const 
   lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = Cf::SMEM;
   lc.stream = c->stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;  // the split-K CTAs of a tile share a cluster
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = grid.z;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = at;
-  lc.numAttrs = 1;
+  lc.numAttrs = c->pdl ? 2 : 1;
   TL_CUDA(cudaLaunchKernelEx(&lc, kern, mw, mw2, mx, p));
   return launch_err(c);
 }
@@ -408,7 +438,7 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
             const MatView* W2, const CUtensorMap* mw2, const ProjOut& o, __half* out16, int skip) {
   const int nmat = W2 ? 2 : 1;
   const int nt = tc_nt(max_rows);
-  const int S = tc_splits(W.N, W.K, max_rows, nmat, W.fmt, W.group);
+  const int S = o.epi == EPI_ARGMAX ? 1 : tc_splits(W.N, W.K, max_rows, nmat, W.fmt, W.group);
   dim3 grid((W.N + 127) / 128, (max_rows + nt - 1) / nt, S);
   TcParams p{};
   p.n_rows = n;
@@ -425,10 +455,12 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   const CUtensorMap& mx = c->xmap[xsel][nt == 64 ? 0 : (nt == 128 ? 1 : 2)];
   const CUtensorMap& m2 = mw2 ? *mw2 : mw;
   if (W.fmt == TL_FMT_INT4) {
+    if (o.epi == EPI_ARGMAX) return tc_launch_nt<1, TL_FMT_INT4, EPI_ARGMAX>(c, nt, mw, m2, mx, p, grid);
     if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, TL_FMT_INT4, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);
     if (o.epi == EPI_RESID) return tc_launch_nt<1, TL_FMT_INT4, EPI_RESID>(c, nt, mw, m2, mx, p, grid);
     return tc_launch_nt<1, TL_FMT_INT4, EPI_STORE>(c, nt, mw, m2, mx, p, grid);
   }
+  if (o.epi == EPI_ARGMAX) return tc_launch_nt<1, TL_FMT_BF16, EPI_ARGMAX>(c, nt, mw, m2, mx, p, grid);
   if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, TL_FMT_BF16, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);
   if (o.epi == EPI_RESID) return tc_launch_nt<1, TL_FMT_BF16, EPI_RESID>(c, nt, mw, m2, mx, p, grid);
   return tc_launch_nt<1, TL_FMT_BF16, EPI_STORE>(c, nt, mw, m2, mx, p, grid);
@@ -436,18 +468,19 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
 
 // Projection over the device-side row count: the CUDA-core GEMV takes up to 8
 // rows (exact fp32 weights and activations); larger counts go to the tensor
-// cores.  When the host only knows an upper bound both are launched and the
-// one that does not apply returns at once; when it knows the exact count
-// (`exact`, prompts) only the right one is launched.  The head (EPI_ARGMAX)
-// always uses the GEMV, which loops over its rows 8 at a time.
-int proj(tl_ctx* c, int max_rows, bool exact, const float* X, int xsel, const int32_t* n, const MatView& W,
+// cores.  PATH_AUTO (only an upper bound known on the host): both are launched
+// and the one that does not apply returns at once.  PATH_GEMV / PATH_TC: the
+// caller knows which applies (prompts, or a graph branch chosen on the
+// device), and only that one is launched.  The head (EPI_ARGMAX) always uses
+// the GEMV, which loops over its rows 8 at a time.
+int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int32_t* n, const MatView& W,
          const CUtensorMap* mw, const MatView* W2, const CUtensorMap* mw2, ProjOut o, __half* out16,
          int prof_kind = TL_PROF_PROJ) {
   const MatView& w2 = W2 ? *W2 : W;
   TL_TRY(prof_start(c, prof_kind));
   const bool argmax = o.epi == EPI_ARGMAX;
-  const bool use_tc = !argmax && max_rows > kGemvMaxRows;
-  const bool use_gemv = argmax || !use_tc || !exact;
+  const bool use_tc = max_rows > kGemvMaxRows && path != PATH_GEMV;
+  const bool use_gemv = argmax || !use_tc || path == PATH_AUTO;
   if (use_gemv) {
     const int skip = use_tc ? kGemvMaxRows : 0;
     int st;
@@ -468,7 +501,10 @@ int proj(tl_ctx* c, int max_rows, bool exact, const float* X, int xsel, const in
     }
     TL_TRY(st);
   }
-  if (use_tc) TL_TRY(tc_proj(c, max_rows, xsel, n, W, *mw, W2, mw2, o, out16, exact ? 0 : kGemvMaxRows));
+  if (use_tc) {
+    if (argmax) o.n_parts = (W.N + 127) / 128;  // one partial per 128-row tile
+    TL_TRY(tc_proj(c, max_rows, xsel, n, W, *mw, W2, mw2, o, out16, path == PATH_AUTO ? kGemvMaxRows : 0));
+  }
   return prof_stop(c, prof_kind);
 }
 
@@ -480,11 +516,10 @@ int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int sl
   if (max_rows > 1) ks = kAttnSplits < 4 ? kAttnSplits : (ks < 4 ? 4 : ks);
   dim3 grid(max_rows, c->cfg.n_heads, ks);
   switch (c->hd) {
-    case 32: attn_decode_kernel<32><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
-    case 64: attn_decode_kernel<64><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
-    default: attn_decode_kernel<128><<<grid, 128, 0, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
+    case 32: TL_TRY(launch_k(c, attn_decode_kernel<32>, dim3(grid), dim3(128), 0, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
+    case 64: TL_TRY(launch_k(c, attn_decode_kernel<64>, dim3(grid), dim3(128), 0, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
+    default: TL_TRY(launch_k(c, attn_decode_kernel<128>, dim3(grid), dim3(128), 0, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
   }
-  TL_TRY(launch_err(c));
   return prof_stop(c, TL_PROF_ATTN);
 }
 
@@ -498,9 +533,9 @@ int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot) 
     attr_done = true;
   }
   dim3 grid((max_rows + 63) / 64, c->cfg.n_heads);
-  attn_prefill_kernel<HD><<<grid, 256, smem, c->stream>>>(c->act_q, c->act_o, c->act_o16, rows, c->kv, slot,
-                                                            c->status);
-  return launch_err(c);
+  TL_TRY(launch_k(c, attn_prefill_kernel<HD>, dim3(grid), dim3(256), smem, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot,
+                                                            c->status));
+  return TL_OK;
 }
 
 int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
@@ -519,20 +554,19 @@ int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
 // (indexed through map, or by row when map is null).
 // prompt = rows are consecutive positions of one lane (tiled causal attention).
 int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int32_t* map, const BlockW& w,
-              int slot_base, int slot_stride, float* h_in, bool prompt = false) {
+              int slot_base, int slot_stride, float* h_in, bool prompt = false, int path = PATH_AUTO) {
+  if (prompt) path = max_rows > kGemvMaxRows ? PATH_TC : PATH_GEMV;
   const int d = c->cfg.d, F = c->cfg.ffn;
   const float eps = c->cfg.rms_eps;
-  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in, c->act_a16,
-                                                       nullptr, 0);
-  TL_TRY(launch_err(c));
+  TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in, c->act_a16,
+                                                       nullptr, 0));
   ProjOut o{};
   o.epi = EPI_STORE;
   o.out = c->act_qkv;
   o.ldo = 3 * d;
-  TL_TRY(proj(c, max_rows, prompt, c->act_a, 0, rows.n, w.wqkv, &w.mqkv, nullptr, nullptr, o, nullptr));
-  rope_kv_kernel<<<max_rows, d / 2, 0, c->stream>>>(c->act_qkv, c->act_q, rows, c->kv, c->rope, slot_base,
-                                                     slot_stride, nullptr, c->status);
-  TL_TRY(launch_err(c));
+  TL_TRY(proj(c, max_rows, path, c->act_a, 0, rows.n, w.wqkv, &w.mqkv, nullptr, nullptr, o, nullptr));
+  TL_TRY(launch_k(c, rope_kv_kernel, dim3(max_rows), dim3(d / 2), 0, c->act_qkv, c->act_q, rows, c->kv, c->rope, slot_base,
+                                                     slot_stride, nullptr, c->status));
   if (prompt)
     TL_TRY(attn_prefill_launch(c, max_rows, rows, slot_base));
   else
@@ -541,55 +575,62 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   r.epi = EPI_RESID;
   r.h = hbuf;
   r.map = map;
-  TL_TRY(proj(c, max_rows, prompt, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
-  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr,
-                                                       c->act_a16, nullptr, 0);
-  TL_TRY(launch_err(c));
+  TL_TRY(proj(c, max_rows, path, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
+  TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr,
+                                                       c->act_a16, nullptr, 0));
   ProjOut sw{};
   sw.epi = EPI_SWIGLU;
   sw.out = c->act_u;
   sw.ldo = F;
-  TL_TRY(proj(c, max_rows, prompt, c->act_a, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16));
-  return proj(c, max_rows, prompt, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr);
+  TL_TRY(proj(c, max_rows, path, c->act_a, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16));
+  return proj(c, max_rows, path, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr);
 }
 
-// Row table `which` from lanes 0..n_consider-1 (all lanes when n_consider <= 0).
+// Row table `which` from lanes 0..n_consider-1 (all lanes when n_consider <= 0);
+// optionally sets a conditional graph node's value from the row count.
 int build_rows(tl_ctx* c, int which, int sel, const uint8_t* mask, const int32_t* per_lane_L, uint8_t* exit_mask,
-               int32_t* alive, int n_consider = 0) {
+               int32_t* alive, int n_consider = 0, cudaGraphConditionalHandle cond = 0, int cond_mode = COND_NONE,
+               const int32_t* body_kernels = nullptr) {
   const int n = n_consider > 0 ? n_consider : c->cfg.max_lanes;
-  build_rows_kernel<<<1, 1024, 0, c->stream>>>(c->lanes, n, sel, mask, per_lane_L, c->rows[which], exit_mask,
-                                               alive, c->status);
-  return launch_err(c);
-}
-
-// One loop iteration for the lanes selected into rows[0].
-int loop_iteration(tl_ctx* c, int max_rows, uint8_t* exit_mask) {
-  const Rows& R = c->rows[0];
-  const int Lb = c->cfg.n_loop_layers;
-  for (int m = 0; m < Lb; ++m)
-    TL_TRY(run_block(c, R, max_rows, c->h, R.lane, c->loop[m], c->cfg.n_pre + m, Lb, m == 0 ? c->h_in : nullptr));
-  exit_update_kernel<<<max_rows, 256, 0, c->stream>>>(R, c->lanes, c->h, c->h_in, c->cfg.d, c->ee, exit_mask,
-                                                      &c->counters[0]);
-  c->steps++;
-  return launch_err(c);
-}
-
-int pre_blocks_for_entered(tl_ctx* c, int max_rows) {
-  if (c->cfg.n_pre == 0) return build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, max_rows);
-  TL_TRY(build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, max_rows));
-  const Rows& E = c->rows[2];
-  for (int b = 0; b < c->cfg.n_pre; ++b) TL_TRY(run_block(c, E, max_rows, c->h, E.lane, c->pre[b], b, 0, nullptr));
+  TL_TRY(launch_k(c, build_rows_kernel, dim3(1), dim3(1024), 0, c->lanes, n, sel, mask, per_lane_L, c->rows[which], exit_mask,
+                                               alive, c->status, cond, cond_mode, kGemvMaxRows, body_kernels,
+                                               &c->counters[2]));
   return TL_OK;
 }
 
-// Boundary stage for the lanes in rows[1]: final norm, head, argmax, then
-// (decode mode) token bookkeeping, embedding and pre blocks.
-int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax, int32_t* tok_out,
-               int32_t* dep_out, int n_new) {
+// One loop iteration for the lanes selected into rows[0].
+int loop_iteration(tl_ctx* c, int max_rows, uint8_t* exit_mask, int path = PATH_AUTO) {
+  const Rows& R = c->rows[0];
+  const int Lb = c->cfg.n_loop_layers;
+  for (int m = 0; m < Lb; ++m)
+    TL_TRY(run_block(c, R, max_rows, c->h, R.lane, c->loop[m], c->cfg.n_pre + m, Lb, m == 0 ? c->h_in : nullptr,
+                     false, path));
+  TL_TRY(launch_k(c, exit_update_kernel, dim3(max_rows), dim3(256), 0, R, c->lanes, c->h, c->h_in, c->cfg.d, c->ee, exit_mask,
+                                                      &c->counters[0]));
+  c->steps++;
+  return TL_OK;
+}
+
+// Pre blocks for the lanes in rows[2] (lanes that just took a token).
+int pre_blocks(tl_ctx* c, int max_rows, int path = PATH_AUTO) {
+  const Rows& E = c->rows[2];
+  for (int b = 0; b < c->cfg.n_pre; ++b)
+    TL_TRY(run_block(c, E, max_rows, c->h, E.lane, c->pre[b], b, 0, nullptr, false, path));
+  return TL_OK;
+}
+
+int pre_blocks_for_entered(tl_ctx* c, int max_rows) {
+  TL_TRY(build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, max_rows));
+  return pre_blocks(c, max_rows);
+}
+
+// Boundary stage, head part, for the lanes in rows[1]: final norm, head,
+// argmax, and in decode mode the token bookkeeping and embedding.
+int head_core(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax, int32_t* tok_out, int32_t* dep_out,
+              int n_new, int path = PATH_AUTO) {
   const Rows& B = c->rows[1];
-  rmsnorm_rows_kernel<<<max_rows, 256, 0, c->stream>>>(c->h, B.lane, B.n, c->cfg.d, c->g_final, c->cfg.rms_eps,
-                                                       c->act_a, nullptr, nullptr, nullptr, 0);
-  TL_TRY(launch_err(c));
+  TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, c->h, B.lane, B.n, c->cfg.d, c->g_final, c->cfg.rms_eps,
+                                                       c->act_a, nullptr, c->act_a16, nullptr, 0));
   ProjOut o{};
   o.epi = EPI_ARGMAX;
   o.logits = logits;
@@ -597,12 +638,18 @@ int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax
   o.ldo = c->cfg.vocab;
   o.part_val = c->part_val;
   o.part_idx = c->part_idx;
-  TL_TRY(proj(c, max_rows, false, c->act_a, 0, B.n, c->head, nullptr, nullptr, nullptr, o, nullptr, TL_PROF_HEAD));
-  const int n_parts = c->head_parts;
-  head_finalize_kernel<<<max_rows, 256, 0, c->stream>>>(B, c->lanes, c->part_val, c->part_idx, n_parts, mode, argmax,
-                                                        tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
-                                                        c->cfg.max_seq, c->status, &c->counters[1]);
-  TL_TRY(launch_err(c));
+  o.n_parts_dev = c->head_nparts;
+  TL_TRY(proj(c, max_rows, path, c->act_a, 0, B.n, c->head, &c->mhead, nullptr, nullptr, o, nullptr, TL_PROF_HEAD));
+  TL_TRY(launch_k(c, head_finalize_kernel, dim3(max_rows), dim3(256), 0, B, c->lanes, c->part_val, c->part_idx, c->head_nparts, mode,
+                                                        argmax, tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
+                                                        c->cfg.max_seq, c->status, &c->counters[1]));
+  return TL_OK;
+}
+
+// Whole boundary stage: head, then (decode mode) pre blocks for the lanes that took a token.
+int head_stage(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax, int32_t* tok_out,
+               int32_t* dep_out, int n_new) {
+  TL_TRY(head_core(c, max_rows, mode, logits, argmax, tok_out, dep_out, n_new));
   if (mode == HEAD_DECODE) return pre_blocks_for_entered(c, max_rows);
   return TL_OK;
 }
@@ -672,6 +719,7 @@ int encode_all_maps(tl_ctx* c) {
       TL_TRY(encode_weight_map(&b.mu, b.wu));
       TL_TRY(encode_weight_map(&b.md, b.wd));
     }
+  TL_TRY(encode_weight_map(&c->mhead, c->head));
   const __half* xs[3] = {c->act_a16, c->act_o16, c->act_u16};
   const int ks[3] = {c->cfg.d, c->cfg.d, c->cfg.ffn};
   const int nts[3] = {64, 128, 256};
@@ -715,6 +763,8 @@ extern "C" const char* tl_strerror(int s) {
 extern "C" const char* tl_last_cuda_error(void) { return g_cuda_err.c_str(); }
 
 __global__ void rope_table_kernel(float2* t, int max_seq, int half, double base) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)max_seq * half) return;
   const int p = (int)(i / half), k = (int)(i % half);
@@ -725,6 +775,8 @@ __global__ void rope_table_kernel(float2* t, int max_seq, int half, double base)
 }
 
 __global__ void lanes_init_kernel(LaneState* l, int n) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
     LaneState z{};
@@ -818,6 +870,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->out_dep = (int32_t*)(w + lay.out_dep);
   c->status = (int32_t*)(w + lay.status);
   c->counters = (unsigned long long*)(w + lay.counters);
+  c->body_kernels = (int32_t*)(w + lay.body_kernels);
+  c->head_nparts = c->body_kernels + 7;
   c->alive = (int32_t*)(w + lay.alive);
   {
     int dev = 0, sms = 0;
@@ -838,11 +892,12 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   do {
     const int half = c->hd / 2;
     const int64_t n = (int64_t)cfg->max_seq * half;
-    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, c->stream>>>(c->rope, cfg->max_seq, half,
-                                                                         (double)cfg->rope_base);
-    if ((st = launch_err(c)) != TL_OK) break;
-    lanes_init_kernel<<<(cfg->max_lanes + 255) / 256, 256, 0, c->stream>>>(c->lanes, cfg->max_lanes);
-    if ((st = launch_err(c)) != TL_OK) break;
+    if ((st = launch_k(c, rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, c->rope, cfg->max_seq,
+                       half, (double)cfg->rope_base)) != TL_OK)
+      break;
+    if ((st = launch_k(c, lanes_init_kernel, dim3((cfg->max_lanes + 255) / 256), dim3(256), 0, c->lanes,
+                       cfg->max_lanes)) != TL_OK)
+      break;
     if ((st = check_cuda(cudaMemsetAsync(w + lay.page_table, 0xFF, per_lane * cfg->max_lanes * 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->status, 0, 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->counters, 0, 32, c->stream))) != TL_OK) break;
@@ -856,6 +911,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
       if ((st = check_cuda(cudaEventCreateWithFlags(&c->alive_ev[i], cudaEventDisableTiming))) != TL_OK) break;
     if (st != TL_OK) break;
     if ((st = check_cuda(cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking))) != TL_OK) break;
+    if ((st = check_cuda(cudaStreamCreateWithFlags(&c->cap_body, cudaStreamNonBlocking))) != TL_OK) break;
   } while (0);
   if (st != TL_OK) {
     if (c->pinned_alive) cudaFreeHost(c->pinned_alive);
@@ -871,6 +927,7 @@ extern "C" int tl_destroy(tl_ctx* c) {
   cudaStreamSynchronize(c->stream);
   if (c->tick_exec) cudaGraphExecDestroy(c->tick_exec);
   if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
+  if (c->cap_body) cudaStreamDestroy(c->cap_body);
   for (int i = 0; i < kAliveRing; ++i) cudaEventDestroy(c->alive_ev[i]);
   for (auto& e : c->prof_ev) {
     cudaEventDestroy(e[0]);
@@ -911,8 +968,7 @@ extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
   for (const MatView* m : mats) {
     if (m->fmt != TL_FMT_INT4) continue;
     const int64_t words = (int64_t)m->N * m->K / 8;
-    int4_repack_kernel<<<(unsigned)((words + 255) / 256), 256, 0, c->stream>>>((uint32_t*)m->q, words);
-    TL_TRY(launch_err(c));
+    TL_TRY(launch_k(c, int4_repack_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, (uint32_t*)m->q, words));
   }
   TL_CUDA(cudaStreamSynchronize(c->stream));
   c->loaded = true;
@@ -974,16 +1030,13 @@ extern "C" int tl_prefill(tl_ctx* c, int32_t lane, const int32_t* host_tokens, i
   const int Tn = T - pos0;
   const Rows& R = c->rows[3];
   TL_CUDA(cudaMemcpyAsync(c->tok_stage, host_tokens + pos0, (size_t)Tn * 4, cudaMemcpyHostToDevice, c->stream));
-  prefill_rows_kernel<<<(Tn + 255) / 256, 256, 0, c->stream>>>(R, lane, pos0, Tn);
-  TL_TRY(launch_err(c));
-  embed_rows_kernel<<<Tn, 256, 0, c->stream>>>(c->embed, c->tok_stage, Tn, cfg.d, c->hrows, c->status);
-  TL_TRY(launch_err(c));
+  TL_TRY(launch_k(c, prefill_rows_kernel, dim3((Tn + 255) / 256), dim3(256), 0, R, lane, pos0, Tn));
+  TL_TRY(launch_k(c, embed_rows_kernel, dim3(Tn), dim3(256), 0, c->embed, c->tok_stage, Tn, cfg.d, c->hrows, c->status));
   for (int b = 0; b < P; ++b) TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->pre[b], b, 0, nullptr, true));
   for (int l = 0; l < L; ++l)
     for (int m = 0; m < Lb; ++m)
       TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr, true));
-  prefill_finish_kernel<<<1, 256, 0, c->stream>>>(c->lanes, lane, Tn, T - 1, L, c->hrows, c->h, cfg.d);
-  TL_TRY(launch_err(c));
+  TL_TRY(launch_k(c, prefill_finish_kernel, dim3(1), dim3(256), 0, c->lanes, lane, Tn, T - 1, L, c->hrows, c->h, cfg.d));
   if (dev_hidden_out)
     TL_CUDA(cudaMemcpyAsync(dev_hidden_out, c->hrows, (size_t)Tn * cfg.d * 4, cudaMemcpyDeviceToDevice, c->stream));
   c->prefill_tokens += Tn;
@@ -1007,9 +1060,8 @@ extern "C" int tl_head_logits(tl_ctx* c, const uint8_t* dev_mask, float* dev_log
 extern "C" int tl_embed_next(tl_ctx* c, const uint8_t* dev_mask, const int32_t* dev_tokens) {
   if (!c || !dev_tokens) return TL_EINVAL;
   if (!c->loaded) return TL_ESTATE;
-  embed_next_kernel<<<c->cfg.max_lanes, 256, 0, c->stream>>>(c->lanes, c->cfg.max_lanes, dev_mask, dev_tokens,
-                                                             c->embed, c->h, c->cfg.d, c->cfg.max_seq, c->status);
-  TL_TRY(launch_err(c));
+  TL_TRY(launch_k(c, embed_next_kernel, dim3(c->cfg.max_lanes), dim3(256), 0, c->lanes, c->cfg.max_lanes, dev_mask, dev_tokens,
+                                                             c->embed, c->h, c->cfg.d, c->cfg.max_seq, c->status));
   return pre_blocks_for_entered(c, c->cfg.max_lanes);
 }
 
@@ -1027,9 +1079,94 @@ static bool same_ee(const EEParams& a, const EEParams& b) {
          a.enabled == b.enabled;
 }
 
-// The tick as a CUDA graph: every kernel reads its row count from device
-// memory, so one capture serves every tick of a decode with the same lanes,
-// token budget, outputs and early-exit parameters.
+// Conditional node after the current position of the capture on `s`.
+static int add_conditional(cudaStream_t s, cudaGraphConditionalHandle h, cudaGraphConditionalNodeType type, int size,
+                           cudaGraph_t* bodies) {
+  cudaStreamCaptureStatus st;
+  cudaGraph_t g = nullptr;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t nd = 0;
+  TL_CUDA(cudaStreamGetCaptureInfo(s, &st, nullptr, &g, &deps, &nd));
+  cudaGraphNodeParams p{};
+  p.type = cudaGraphNodeTypeConditional;
+  p.conditional.handle = h;
+  p.conditional.type = type;
+  p.conditional.size = size;
+  cudaGraphNode_t node;
+  TL_CUDA(cudaGraphAddNode(&node, g, deps, nd, &p));
+  for (int i = 0; i < size; ++i) bodies[i] = p.conditional.phGraph_out[i];
+  TL_CUDA(cudaStreamUpdateCaptureDependencies(s, &node, 1, cudaStreamSetCaptureDependencies));
+  return TL_OK;
+}
+
+static int new_handle(cudaStream_t s, cudaGraphConditionalHandle* h) {
+  cudaStreamCaptureStatus st;
+  cudaGraph_t g = nullptr;
+  TL_CUDA(cudaStreamGetCaptureInfo(s, &st, nullptr, &g, nullptr, nullptr));
+  TL_CUDA(cudaGraphConditionalHandleCreate(h, g, 0, cudaGraphCondAssignDefault));
+  return TL_OK;
+}
+
+// Captures fn() into an (empty) body graph; *n_kernels = kernels it launched.
+template <class F>
+static int capture_body(tl_ctx* c, cudaGraph_t body, int64_t* n_kernels, F fn) {
+  TL_CUDA(cudaStreamBeginCaptureToGraph(c->cap_body, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal));
+  cudaStream_t saved = c->stream;
+  c->stream = c->cap_body;
+  const int64_t l0 = c->launches;
+  const int st = fn();
+  *n_kernels = c->launches - l0;
+  c->stream = saved;
+  cudaGraph_t out = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(c->cap_body, &out);
+  TL_TRY(st);
+  return check_cuda(e);
+}
+
+// The tick as a CUDA graph with device-chosen branches: the row-table kernel
+// of each stage sets a conditional node, so a stage with no rows runs nothing
+// and a stage runs either its CUDA-core GEMV variant (<= 8 rows) or its
+// tensor-core variant, never both.  Every kernel reads its row count from
+// device memory, so one capture serves every tick of a decode with the same
+// lanes, token budget, outputs and early-exit parameters.
+//   rows(boundary) -> SWITCH { norm, head, argmax + token + embedding: GEMV | tensor cores }
+//   rows(entered)  -> SWITCH { pre blocks: GEMV | tensor cores }
+//   rows(loop)     -> SWITCH { loop body + exit rule: GEMV | tensor cores }
+static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out, int32_t* kcount) {
+  cudaGraphConditionalHandle hb, he, hl;
+  cudaGraph_t body[2];
+  int64_t nk[2] = {0, 0};
+  // boundary rows -> head (CUDA-core GEMV for <= 8 rows, tensor cores above)
+  TL_TRY(new_handle(c->stream, &hb));
+  TL_TRY(build_rows(c, 1, SEL_BOUNDARY, nullptr, nullptr, nullptr, c->alive, n_lanes, hb, COND_SWITCH, c->body_kernels + 0));
+  TL_TRY(add_conditional(c->stream, hb, cudaGraphCondTypeSwitch, 2, body));
+  TL_TRY(capture_body(c, body[0], &nk[0], [&] { return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_GEMV); }));
+  TL_TRY(capture_body(c, body[1], &nk[1], [&] { return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_TC); }));
+  kcount[0] = (int32_t)nk[0];
+  kcount[1] = (int32_t)nk[1];
+  // entered rows -> pre blocks
+  TL_TRY(new_handle(c->stream, &he));
+  TL_TRY(build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, n_lanes, he, COND_SWITCH, c->body_kernels + 2));
+  if (c->cfg.n_pre > 0) {
+    TL_TRY(add_conditional(c->stream, he, cudaGraphCondTypeSwitch, 2, body));
+    TL_TRY(capture_body(c, body[0], &nk[0], [&] { return pre_blocks(c, n_lanes, PATH_GEMV); }));
+    TL_TRY(capture_body(c, body[1], &nk[1], [&] { return pre_blocks(c, n_lanes, PATH_TC); }));
+    kcount[2] = (int32_t)nk[0];
+    kcount[3] = (int32_t)nk[1];
+  } else {
+    kcount[2] = kcount[3] = 0;
+  }
+  // loop rows -> loop body
+  TL_TRY(new_handle(c->stream, &hl));
+  TL_TRY(build_rows(c, 0, SEL_LOOP, nullptr, nullptr, nullptr, nullptr, n_lanes, hl, COND_SWITCH, c->body_kernels + 4));
+  TL_TRY(add_conditional(c->stream, hl, cudaGraphCondTypeSwitch, 2, body));
+  TL_TRY(capture_body(c, body[0], &nk[0], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_GEMV); }));
+  TL_TRY(capture_body(c, body[1], &nk[1], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_TC); }));
+  kcount[4] = (int32_t)nk[0];
+  kcount[5] = (int32_t)nk[1];
+  return TL_OK;
+}
+
 static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
   if (c->tick_exec && c->tick_lanes == n_lanes && c->tick_new == n_new && c->tick_tok == tok_out &&
       c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee))
@@ -1039,14 +1176,14 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
     c->tick_exec = nullptr;
   }
   const int64_t l0 = c->launches, s0 = c->steps;
+  int32_t kcount[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   cudaStream_t saved = c->stream;
   TL_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
   c->stream = c->cap_stream;
-  const int st = enqueue_tick(c, n_lanes, n_new, tok_out, dep_out);
+  const int st = capture_tick(c, n_lanes, n_new, tok_out, dep_out, kcount);
   c->stream = saved;
   cudaGraph_t g = nullptr;
   const cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
-  const int64_t per_tick = c->launches - l0;
   c->launches = l0;
   c->steps = s0;
   if (st != TL_OK) {
@@ -1057,20 +1194,22 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   const cudaError_t ei = cudaGraphInstantiate(&c->tick_exec, g, 0);
   cudaGraphDestroy(g);
   TL_CUDA(ei);
+  // the row-table kernels add the chosen bodies' kernel counts on the device
+  TL_CUDA(cudaMemcpyAsync(c->body_kernels, kcount, sizeof(kcount), cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaStreamSynchronize(c->stream));
   c->tick_lanes = n_lanes;
   c->tick_new = n_new;
   c->tick_tok = tok_out;
   c->tick_dep = dep_out;
   c->tick_ee = c->ee;
-  c->tick_launches = per_tick;
+  c->tick_launches = 3;  // the three row-table kernels outside the conditional bodies
   return TL_OK;
 }
 
 static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
-  decode_init_kernel<<<(n_lanes + 255) / 256, 256, 0, c->stream>>>(c->lanes, n_lanes, c->L_stage, n_new, c->status);
-  TL_TRY(launch_err(c));
+  TL_TRY(launch_k(c, decode_init_kernel, dim3((n_lanes + 255) / 256), dim3(256), 0, c->lanes, n_lanes, c->L_stage, n_new, c->status));
   // per-kind event profiling needs individual launches; otherwise replay a captured tick
-  const bool graphs = c->prof_mask == 0;
+  const bool graphs = c->prof_mask == 0 && c->graphs_enabled;
   if (graphs) TL_TRY(tick_graph(c, n_lanes, n_new, tok_out, dep_out));
   // upper bound on ticks: every token runs at most L_max iterations, plus the first
   const int64_t max_ticks = (int64_t)n_new * (c->cfg.L_max + 1) + 4;
@@ -1138,7 +1277,7 @@ extern "C" int tl_stats_get(tl_ctx* c, tl_stats* out) {
   out->lane_iterations = (int64_t)ctr[0];
   out->tokens_emitted = (int64_t)ctr[1];
   out->prefill_tokens = c->prefill_tokens;
-  out->kernel_launches = c->launches;
+  out->kernel_launches = c->launches + (int64_t)ctr[2];
   out->device_status = st;
   out->kv_pages_used = c->lay.n_pages - (int32_t)c->free_pages.size();
   return TL_OK;
@@ -1193,5 +1332,11 @@ extern "C" int tl_profile_end(tl_ctx* c, int64_t* groups, double* total_ms) {
     if (total_ms) total_ms[k] = c->prof_ms[k];
   }
   c->prof_mask = 0;
+  return TL_OK;
+}
+
+extern "C" int tl_set_graphs(tl_ctx* c, int32_t enabled) {
+  if (!c) return TL_EINVAL;
+  c->graphs_enabled = enabled != 0;
   return TL_OK;
 }

@@ -135,7 +135,7 @@ __device__ __forceinline__ void tc_emit(const TcParams& p, int row, int m, float
     const float u = silu_f(v) * v2;
     o.out[(int64_t)row * o.ldo + m] = u;
     if (p.out16) p.out16[(int64_t)row * o.ldo + m] = __float2half_rn(u);
-  } else {
+  } else if constexpr (EPI == EPI_RESID) {
     const int hr = o.map ? o.map[row] : row;
     o.h[(int64_t)hr * p.N + m] += v;
   }
@@ -162,13 +162,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rows = p.n_rows[0];
   const int m0 = blockIdx.x * 128, n0 = blockIdx.y * NT;
-  if (rows <= p.skip_at_or_below || n0 >= rows) return;
   const int nkb = p.kb_per_split, kb0 = blockIdx.z * nkb;
   const int S = gridDim.z;                      // split-K CTAs of this tile = cluster size
-  const int ncols = min(NT, rows - n0);
   float* red = reinterpret_cast<float*>(sA);    // [NMAT][NT][128] partial tile after the main loop
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -191,19 +189,51 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  // Weight tiles depend on no earlier kernel: when this launch certainly runs
+  // (no row-count skip), the first stages are requested before waiting for
+  // the previous kernel.  Their barriers expect the weight bytes now and get
+  // their arrival (with the activation bytes) after the wait.
+  const int pre = (p.skip_at_or_below == 0) ? min(nkb, STAGES) : 0;
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < pre; ++i) {
+      const uint32_t fb = smem_u32(&full[i]);
+      mbar_add_tx(fb, NMAT * C::RAW_BYTES);
+      const int kb = kb0 + i;
+      const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
+      tma_load_2d(smem_u32(sRaw + (i * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
+      if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (i * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+    }
+  }
+  pdl_wait();
+  const int rows = p.n_rows[0];
+  const bool active = !(rows <= p.skip_at_or_below || n0 >= rows);
+  const int ncols = active ? min(NT, rows - n0) : 0;
+
+  if (!active) {
+    if (warp == 0 && lane == 0) {  // nothing to compute: let the early weight copies land, then leave
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive(smem_u32(&full[i]));
+        volatile int32_t never = 0;
+        mbar_wait(smem_u32(&full[i]), 0, &never);
+      }
+    }
+  } else if (warp == 0) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % STAGES, r = i / STAGES;
-        if (r > 0 && !mbar_wait(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) break;
-        const uint32_t fb = smem_u32(&full[s]);
-        mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
         const int kb = kb0 + i;
-        const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
-        tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
-        if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+        const uint32_t fb = smem_u32(&full[s]);
+        if (i < pre) {
+          mbar_expect_tx(fb, C::B_BYTES);
+        } else {
+          if (r > 0 && !mbar_wait(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) break;
+          mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
+          const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
+          tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
+          if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+        }
         tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
         issued = i + 1;
       }
@@ -287,6 +317,39 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int m = m0 + t;
       const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+      if constexpr (EPI == EPI_ARGMAX) {
+        // per activation row: the best (value, index) of this tile's 128 outputs
+        float* bv_s = reinterpret_cast<float*>(sA);          // [4 warps][NT]
+        int* bi_s = reinterpret_cast<int*>(sA) + 4 * NT;      // [4 warps][NT]
+        for (int j = 0; j < ncols; j += 8) {
+          float v[8];
+          tmem_ld8(tl + j, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (j + e >= ncols) break;
+            float bv = (m < p.N) ? v[e] : -INFINITY;
+            int bi = (m < p.N) ? m : 0x7fffffff;
+            if (p.o.logits && m < p.N) p.o.logits[(int64_t)p.o.lmap[n0 + j + e] * p.o.ldo + m] = v[e];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+              const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+              if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) { bv_s[q * NT + j + e] = bv; bi_s[q * NT + j + e] = bi; }
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (t < ncols) {
+          float bv = bv_s[t];
+          int bi = bi_s[t];
+          for (int w = 1; w < 4; ++w)
+            if (better(bv_s[w * NT + t], bi_s[w * NT + t], bv, bi)) { bv = bv_s[w * NT + t]; bi = bi_s[w * NT + t]; }
+          p.o.part_val[(int64_t)(n0 + t) * p.o.n_parts + blockIdx.x] = bv;
+          p.o.part_idx[(int64_t)(n0 + t) * p.o.n_parts + blockIdx.x] = bi;
+        }
+        if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0 && p.o.n_parts_dev) p.o.n_parts_dev[0] = p.o.n_parts;
+      } else
       for (int j = 0; j < ncols; j += 8) {
         float v[8], v2[8];
         tmem_ld8(tl + j, v);
@@ -307,7 +370,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
       }
     }
   }
-  if (S > 1) {
+  if (active && S > 1) {
     // split-K: reduce this CTA's slice of rows over the cluster's partial tiles
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -340,6 +403,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
 // 8-element word in nibble e) into the device layout used above and by the
 // CUDA-core kernels (element 2i in nibble i, 2i+1 in nibble i + 4).  In place.
 __global__ void int4_repack_kernel(uint32_t* __restrict__ w, int64_t n_words) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n_words) return;
   const uint32_t x = w[i];

@@ -241,6 +241,15 @@ int tl_generate(tl_ctx* ctx, const int32_t* host_prompts, int32_t n_lanes, int32
                 const int32_t* host_per_lane_L, int32_t n_new, int32_t* host_tokens_out,
                 int32_t* host_depths_out);
 
+/* Replay of decode ticks as CUDA graphs (default on): each tick of tl_decode /
+ * tl_generate is one captured graph whose conditional nodes, set on the
+ * device from the live row counts, skip empty stages and pick the CUDA-core or
+ * tensor-core variant of a stage.  enabled = 0 launches every kernel of a tick
+ * individually instead (same kernels and results; what profilers that cannot
+ * look inside graphs with conditional nodes need).  Timing with
+ * tl_profile_begin also launches individually. */
+int tl_set_graphs(tl_ctx* ctx, int32_t enabled);
+
 /* ------------------------------------------------- lane-state checkpoint -- */
 
 /* Bytes of a lane-state snapshot: the scheduling state and the fp32 hidden row
