@@ -8,7 +8,8 @@
 // stages with cp.async.bulk (untiled TMA, no multicast), several stages ahead,
 // while 8 consumer warps turn each stage into outputs.  The activation rows
 // are staged once per CTA (fp32, 16-byte slots XOR-swizzled as in the
-// CUDA-core GEMV).  A consumer warp owns whole output features: every lane
+// CUDA-core GEMV), optionally normalised on the way in (GsNorm).  A consumer
+// warp owns whole output features: every lane
 // takes 32-element chunks of the row from shared memory, and one warp
 // reduction per (feature, row) finishes it.  Memory parallelism comes from the
 // bulk copies in flight (tens of KB per SM), not from registers.
@@ -140,10 +141,21 @@ __device__ __forceinline__ void gs_issue(const MatView& W, const MatView& W2, co
   }
 }
 
+// RMSNorm folded into the activation staging (g != null): X holds the
+// residual rows h, row r of this projection is h row map[r] (row r when map is
+// null), and each CTA stages x * rsqrt(mean(x^2) + eps) * g itself; CTA 0 also
+// copies the raw rows to h_in (indexed like h) when h_in is given.
+struct GsNorm {
+  const float* g;
+  const int32_t* map;
+  float eps;
+  float* h_in;
+};
+
 template <int FMT, int EPI>
 __global__ void __launch_bounds__(GS_THREADS, 1)
 gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_rows, MatView W, MatView W2, ProjOut o,
-                   int skip_above, GsPlan pl, int32_t* __restrict__ status) {
+                   int skip_above, GsPlan pl, GsNorm nrm, int32_t* __restrict__ status) {
   constexpr int NMAT = (EPI == EPI_SWIGLU) ? 2 : 1;
   extern __shared__ __align__(128) uint8_t gs_smem[];
   uint8_t* ring = gs_smem;
@@ -153,6 +165,7 @@ gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_ro
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(empty + pl.stages);
   __shared__ float best_v[GS_CONSUMERS][8];
   __shared__ int best_i[GS_CONSUMERS][8];
+  __shared__ float inv_s[8];
 
   const int K = W.K, N = W.N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -187,12 +200,39 @@ gemv_stream_kernel(const float* __restrict__ X, const int32_t* __restrict__ n_ro
   int it = 0;  // pipeline position, continued across row chunks
   for (int r0 = 0; r0 < rows; r0 += 8) {
     const int nr = min(8, rows - r0);
+    float4* xs4 = reinterpret_cast<float4*>(xs);
+    const bool copy_in = nrm.h_in && blockIdx.x == 0;
     for (int f = threadIdx.x; f < nr * K / 4; f += blockDim.x) {
       const int r = f / (K / 4), fi = f % (K / 4);
-      reinterpret_cast<float4*>(xs)[r * (K / 4) + swz_slot(fi)] =
-          reinterpret_cast<const float4*>(X + (int64_t)(r0 + r) * K)[fi];
+      const int src = nrm.map ? nrm.map[r0 + r] : r0 + r;
+      const float4 v = reinterpret_cast<const float4*>(X + (int64_t)src * K)[fi];
+      xs4[r * (K / 4) + swz_slot(fi)] = v;
+      if (copy_in) reinterpret_cast<float4*>(nrm.h_in + (int64_t)src * K)[fi] = v;
     }
     __syncthreads();
+    if (nrm.g) {
+      if (warp < nr) {  // warp r: sum of squares of row r
+        float ss = 0.f;
+        for (int q = lane; q < K / 4; q += 32) {
+          const float4 v = xs4[warp * (K / 4) + q];
+          ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) inv_s[warp] = rsqrtf(ss / (float)K + nrm.eps);
+      }
+      __syncthreads();
+      for (int f = threadIdx.x; f < nr * K / 4; f += blockDim.x) {
+        const int r = f / (K / 4), fi = f % (K / 4);
+        const float inv = inv_s[r];
+        const float4 gg = reinterpret_cast<const float4*>(nrm.g)[fi];
+        float4& v = xs4[r * (K / 4) + swz_slot(fi)];
+        v.x = v.x * inv * gg.x;
+        v.y = v.y * inv * gg.y;
+        v.z = v.z * inv * gg.z;
+        v.w = v.w * inv * gg.w;
+      }
+      __syncthreads();
+    }
     if (warp == GS_CONSUMERS) {
       // ------------------------------------------------------------ producer
       if (lane == 0) {

@@ -147,22 +147,115 @@ __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, in
   }
 }
 
+// The three row tables of a decode tick from the lane states at its start,
+// in lane order, decided one stage ahead: boundary rows (loop finished: head,
+// token), entered rows (boundary lanes that will take a token and continue:
+// their pre blocks run at position pos + 1) and loop rows (lanes in their loop
+// plus the entering lanes at iteration 0).  Whether a boundary lane continues
+// is fixed before its head runs, by the same test head_finalize_kernel applies
+// (n_emitted + 1 < n_target and pos + 1 < max_seq).  alive = lanes in their
+// loop or at a boundary.  With conditional graph nodes, sets the SWITCH value
+// of each table whose bit is set in cond.use, as build_rows_kernel does.  One
+// CTA of 1024 threads; thread i looks at lane i.
+struct TickConds {
+  cudaGraphConditionalHandle h[3];  // boundary, entered, loop
+  int32_t use;                      // bit t: h[t] is a live handle
+};
+
+__global__ void plan_tick_kernel(const LaneState* __restrict__ lanes, int n_lanes, Rows boundary, Rows entered,
+                                 Rows loop, int32_t* __restrict__ alive, int max_seq, TickConds cond,
+                                 int32_t gemv_max_rows, const int32_t* __restrict__ body_kernels,
+                                 unsigned long long* __restrict__ kernel_count) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ int32_t cnt[3][32];
+  const int i = threadIdx.x, lane = i & 31, w = i >> 5;
+  int take[3] = {0, 0, 0}, live = 0, pos = 0, iter = 0;
+  if (i < n_lanes) {
+    const LaneState st = lanes[i];
+    pos = st.pos;
+    iter = st.iter;
+    const bool b = st.phase == PH_BOUNDARY;
+    const bool e = b && st.n_emitted + 1 < st.n_target && st.pos + 1 < max_seq;
+    take[0] = b;
+    take[1] = e;
+    take[2] = st.phase == PH_LOOP || e;
+    live = st.phase == PH_LOOP || b;
+  }
+  unsigned bal[3];
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    bal[t] = __ballot_sync(0xffffffffu, take[t]);
+    if (lane == 0) cnt[t][w] = __popc(bal[t]);
+  }
+  const unsigned live_bal = __ballot_sync(0xffffffffu, live);
+  __shared__ int32_t live_cnt[32];
+  if (lane == 0) live_cnt[w] = __popc(live_bal);
+  __syncthreads();
+  if (w < 3) {  // warp t scans table t's per-warp counts
+    int v = cnt[w][lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    cnt[w][lane] = v;  // inclusive
+  } else if (w == 3) {
+    const int v = warp_sum(live_cnt[lane]);
+    if (lane == 0) live_cnt[0] = v;
+  }
+  __syncthreads();
+  const unsigned below = (1u << lane) - 1u;
+  const Rows* tab[3] = {&boundary, &entered, &loop};
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    if (take[t]) {
+      const int r = (w == 0 ? 0 : cnt[t][w - 1]) + __popc(bal[t] & below);
+      const bool fresh = t == 1 || (t == 2 && take[1]);  // entering: next position, iteration 0
+      tab[t]->lane[r] = i;
+      tab[t]->pos[r] = fresh ? pos + 1 : pos;
+      tab[t]->iter[r] = fresh ? 0 : iter;
+    }
+  }
+  if (i == 0) {
+    int n[3];
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      n[t] = cnt[t][31];
+      tab[t]->n[0] = n[t];
+    }
+    if (alive) alive[0] = live_cnt[0];
+    unsigned long long k = 0;
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      if (!((cond.use >> t) & 1)) continue;
+      const unsigned v = n[t] == 0 ? 2u : (n[t] <= gemv_max_rows ? 0u : 1u);
+      cudaGraphSetConditional(cond.h[t], v);
+      if (v < 2) k += (unsigned long long)body_kernels[2 * t + v];
+    }
+    if (k) atomicAdd(kernel_count, k);
+  }
+}
+
 // --------------------------------------------------------------- norms ----
 
 // out[r] = RMSNorm(h[map ? map[r] : r]) * g, fp32 (and an fp16 copy for the
 // tensor-core projections when out16 is given).  One CTA per row.  When h_in is
 // given, also copies the source row there (indexed like h); when zero_rows is
 // given, clears row r of that [rows][zero_cols] accumulator, which the next
-// (split-K) projection adds into.
+// (split-K) projection adds into.  Does nothing when the row count is at most
+// min_rows (those counts are served by a GEMV that normalises by itself).
 __global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* __restrict__ map,
                                     const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
                                     float eps, float* __restrict__ out, float* __restrict__ h_in,
-                                    __half* __restrict__ out16, float* __restrict__ zero_rows, int zero_cols) {
+                                    __half* __restrict__ out16, float* __restrict__ zero_rows, int zero_cols,
+                                    int min_rows) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float red[32];
   const int r = blockIdx.x;
-  if (r >= n_rows[0]) return;
+  const int n = n_rows[0];
+  if (r >= n || n <= min_rows) return;
   const int src = map ? map[r] : r;
   const float* x = h + (int64_t)src * d;
   float ss = 0.f;
@@ -465,7 +558,13 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
 // ------------------------------------------------------------- attention ----
 //
 // o[r][h] = softmax(q k^T / sqrt(hd)) v over positions 0..pos of the row's
-// (lane, slot) cache.  One CTA of 4 warps per (row, head, split): the key
+// (lane, slot) cache, with RoPE and the KV append of the row's own position
+// folded in: every CTA rotates its head's query from the projection output
+// (qkv, [rows][3d]), and the CTA of the last split, whose key range holds
+// position pos, first rotates and stores that position's key and value, then
+// reads them back with the rest of its range (ordered by __syncthreads within
+// the CTA; no other CTA reads that position).  One CTA of 4 warps per
+// (row, head, split): the key
 // blocks of 32 positions are divided into S contiguous ranges, S chosen on the
 // device from the live row count so that few rows still spread over the SMs
 // (S <= gridDim.z).  Inside a CTA warp w takes blocks w, w+4, ...: one key per
@@ -475,9 +574,9 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
 // (row, head) to finish, in split order.  Requires kv_page_tokens >= 32.
 template <int HD>
 __global__ void __launch_bounds__(128)
-attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows, KVGeom g,
-                   int slot_base, int slot_stride, float* __restrict__ part, int32_t* __restrict__ counters,
-                   int32_t* __restrict__ status) {
+attn_decode_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
+                   KVGeom g, const float2* __restrict__ rope_cs, int slot_base, int slot_stride,
+                   float* __restrict__ part, int32_t* __restrict__ counters, int32_t* __restrict__ status) {
   pdl_launch_dependents();
   pdl_wait();
   constexpr int DPL = HD / 32;  // output dims per lane
@@ -500,7 +599,28 @@ attn_decode_kernel(const float* __restrict__ q, float* __restrict__ o, __half* _
   if (z >= S) return;
   const int b0 = (z * nblk) / S, b1 = ((z + 1) * nblk) / S;
   const float scale = rsqrtf((float)HD);
-  for (int i = threadIdx.x; i < HD; i += blockDim.x) qs[i] = q[(int64_t)r * d + h * HD + i] * scale;
+  {
+    constexpr int HALF = HD / 2;
+    const float* src = qkv + (int64_t)r * 3 * d + h * HD;
+    const int i = threadIdx.x;
+    if (i < HALF) {
+      const float2 cs = rope_cs[(int64_t)pos * HALF + i];
+      const float q0 = src[i], q1 = src[i + HALF];
+      qs[i] = (q0 * cs.x - q1 * cs.y) * scale;
+      qs[i + HALF] = (q1 * cs.x + q0 * cs.y) * scale;
+      if (z == S - 1) {  // this split's range ends at pos: append the row's key and value
+        __half* kp = kv_k_ptr(g, ln, slot, pos, h, status);
+        if (kp) {
+          __half* vp = kp + (int64_t)g.H * g.page_tokens * HD;
+          const float k0 = src[d + i], k1 = src[d + i + HALF];
+          kp[i] = __float2half_rn(k0 * cs.x - k1 * cs.y);
+          kp[i + HALF] = __float2half_rn(k1 * cs.x + k0 * cs.y);
+          vp[i] = __float2half_rn(src[2 * d + i]);
+          vp[i + HALF] = __float2half_rn(src[2 * d + i + HALF]);
+        }
+      }
+    }
+  }
   __syncthreads();
   float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
@@ -828,13 +948,15 @@ enum HeadMode : int32_t { HEAD_ONLY = 0, HEAD_DECODE = 1 };
 // Argmax over the head's partial results for each boundary row; HEAD_DECODE
 // also records the token and the depth behind it, and either retires the lane
 // or moves it to its next position: cap = depth (monotonic clamp), L_run =
-// min(L_req, cap), embed the token, mark it for its pre blocks.  One CTA per row.
+// min(L_req, cap), embed the token, and (mark_entered) flag it for a later
+// SEL_ENTERED table; a decode tick plans its entered rows beforehand and
+// passes 0.  One CTA per row.
 __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ part_val,
                                      const int32_t* __restrict__ part_idx, const int32_t* __restrict__ n_parts_dev,
                                      int32_t mode,
                                      int32_t* __restrict__ argmax_out, int32_t* __restrict__ tokens_out,
                                      int32_t* __restrict__ depths_out, int n_new, MatView E, float* __restrict__ h,
-                                     int d, int max_seq, int32_t* __restrict__ status,
+                                     int d, int max_seq, int32_t mark_entered, int32_t* __restrict__ status,
                                      unsigned long long* __restrict__ tok_count) {
   pdl_launch_dependents();
   pdl_wait();
@@ -887,7 +1009,7 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
         st.streak = 0;
         st.token = bi;
         st.phase = PH_LOOP;
-        st.entered = 1;
+        st.entered = mark_entered;
         go_s = 1;
       }
     }

@@ -371,27 +371,30 @@ int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView&
 
 template <int FMT, int EPI>
 int gemv_stream_launch(tl_ctx* c, const GsChoice& g, const float* X, const int32_t* n_rows, const MatView& W,
-                       const MatView& W2, const ProjOut& o, int skip_above) {
+                       const MatView& W2, const ProjOut& o, int skip_above, const GsNorm& nrm) {
   auto kern = gemv_stream_kernel<FMT, EPI>;
   static int attr_smem = 0;  // per instantiation: largest opt-in requested so far
   if (g.smem > attr_smem) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem));
     attr_smem = g.smem;
   }
-  TL_TRY(launch_k(c, kern, dim3(g.grid), dim3(GS_THREADS), g.smem, X, n_rows, W, W2, o, skip_above, g.pl, c->status));
+  TL_TRY(launch_k(c, kern, dim3(g.grid), dim3(GS_THREADS), g.smem, X, n_rows, W, W2, o, skip_above, g.pl, nrm,
+                  c->status));
   return TL_OK;
 }
 
 // Few-row projection: the streamed GEMV where its ring fits, else the
-// register-blocked CUDA-core GEMV.
+// register-blocked CUDA-core GEMV.  nrm (streamed GEMV only): X is the
+// residual and the kernel applies the RMSNorm itself.
 template <int FMT, int EPI, int RPW>
 int small_rows_proj(tl_ctx* c, const float* X, const int32_t* n, const MatView& W, const MatView& W2, ProjOut o,
-                    int skip) {
+                    int skip, const GsNorm* nrm) {
   const GsChoice g = gs_plan(FMT, W.N, W.K, W.group, EPI == EPI_SWIGLU ? 2 : 1, c->n_sms);
   if (g.ok) {
     if (EPI == EPI_ARGMAX) o.n_parts = g.grid;
-    return gemv_stream_launch<FMT, EPI>(c, g, X, n, W, W2, o, skip);
+    return gemv_stream_launch<FMT, EPI>(c, g, X, n, W, W2, o, skip, nrm ? *nrm : GsNorm{});
   }
+  if (nrm) return TL_EINVAL;  // callers check gemv_norms_itself first
   if (EPI == EPI_ARGMAX) o.n_parts = (W.N + GEMV_WARPS * RPW - 1) / (GEMV_WARPS * RPW);
   return gemv_launch<FMT, EPI, RPW>(c, X, n, W, W2, o, skip);
 }
@@ -471,32 +474,32 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
 // cores.  PATH_AUTO (only an upper bound known on the host): both are launched
 // and the one that does not apply returns at once.  PATH_GEMV / PATH_TC: the
 // caller knows which applies (prompts, or a graph branch chosen on the
-// device), and only that one is launched.  The head (EPI_ARGMAX) always uses
-// the GEMV, which loops over its rows 8 at a time.
+// device), and only that one is launched.  nrm: see small_rows_proj (the
+// tensor-core variant reads the fp16 copy of a separate norm kernel).
 int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int32_t* n, const MatView& W,
          const CUtensorMap* mw, const MatView* W2, const CUtensorMap* mw2, ProjOut o, __half* out16,
-         int prof_kind = TL_PROF_PROJ) {
+         int prof_kind = TL_PROF_PROJ, const GsNorm* nrm = nullptr) {
   const MatView& w2 = W2 ? *W2 : W;
   TL_TRY(prof_start(c, prof_kind));
   const bool argmax = o.epi == EPI_ARGMAX;
   const bool use_tc = max_rows > kGemvMaxRows && path != PATH_GEMV;
-  const bool use_gemv = argmax || !use_tc || path == PATH_AUTO;
+  const bool use_gemv = !use_tc || path == PATH_AUTO;
   if (use_gemv) {
     const int skip = use_tc ? kGemvMaxRows : 0;
     int st;
     if (W.fmt == TL_FMT_INT4) {
       switch (o.epi) {
-        case EPI_STORE: st = small_rows_proj<TL_FMT_INT4, EPI_STORE, 1>(c, X, n, W, w2, o, skip); break;
-        case EPI_RESID: st = small_rows_proj<TL_FMT_INT4, EPI_RESID, 1>(c, X, n, W, w2, o, skip); break;
-        case EPI_SWIGLU: st = small_rows_proj<TL_FMT_INT4, EPI_SWIGLU, 1>(c, X, n, W, w2, o, skip); break;
-        default: st = small_rows_proj<TL_FMT_INT4, EPI_ARGMAX, head_rpw(TL_FMT_INT4)>(c, X, n, W, w2, o, skip); break;
+        case EPI_STORE: st = small_rows_proj<TL_FMT_INT4, EPI_STORE, 1>(c, X, n, W, w2, o, skip, nrm); break;
+        case EPI_RESID: st = small_rows_proj<TL_FMT_INT4, EPI_RESID, 1>(c, X, n, W, w2, o, skip, nrm); break;
+        case EPI_SWIGLU: st = small_rows_proj<TL_FMT_INT4, EPI_SWIGLU, 1>(c, X, n, W, w2, o, skip, nrm); break;
+        default: st = small_rows_proj<TL_FMT_INT4, EPI_ARGMAX, head_rpw(TL_FMT_INT4)>(c, X, n, W, w2, o, skip, nrm); break;
       }
     } else {
       switch (o.epi) {
-        case EPI_STORE: st = small_rows_proj<TL_FMT_BF16, EPI_STORE, 1>(c, X, n, W, w2, o, skip); break;
-        case EPI_RESID: st = small_rows_proj<TL_FMT_BF16, EPI_RESID, 1>(c, X, n, W, w2, o, skip); break;
-        case EPI_SWIGLU: st = small_rows_proj<TL_FMT_BF16, EPI_SWIGLU, 1>(c, X, n, W, w2, o, skip); break;
-        default: st = small_rows_proj<TL_FMT_BF16, EPI_ARGMAX, head_rpw(TL_FMT_BF16)>(c, X, n, W, w2, o, skip); break;
+        case EPI_STORE: st = small_rows_proj<TL_FMT_BF16, EPI_STORE, 1>(c, X, n, W, w2, o, skip, nrm); break;
+        case EPI_RESID: st = small_rows_proj<TL_FMT_BF16, EPI_RESID, 1>(c, X, n, W, w2, o, skip, nrm); break;
+        case EPI_SWIGLU: st = small_rows_proj<TL_FMT_BF16, EPI_SWIGLU, 1>(c, X, n, W, w2, o, skip, nrm); break;
+        default: st = small_rows_proj<TL_FMT_BF16, EPI_ARGMAX, head_rpw(TL_FMT_BF16)>(c, X, n, W, w2, o, skip, nrm); break;
       }
     }
     TL_TRY(st);
@@ -516,9 +519,9 @@ int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int sl
   if (max_rows > 1) ks = kAttnSplits < 4 ? kAttnSplits : (ks < 4 ? 4 : ks);
   dim3 grid(max_rows, c->cfg.n_heads, ks);
   switch (c->hd) {
-    case 32: TL_TRY(launch_k(c, attn_decode_kernel<32>, dim3(grid), dim3(128), 0, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
-    case 64: TL_TRY(launch_k(c, attn_decode_kernel<64>, dim3(grid), dim3(128), 0, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
-    default: TL_TRY(launch_k(c, attn_decode_kernel<128>, dim3(grid), dim3(128), 0, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
+    case 32: TL_TRY(launch_k(c, attn_decode_kernel<32>, dim3(grid), dim3(128), 0, c->act_qkv, c->act_o, c->act_o16, rows, c->kv, c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
+    case 64: TL_TRY(launch_k(c, attn_decode_kernel<64>, dim3(grid), dim3(128), 0, c->act_qkv, c->act_o, c->act_o16, rows, c->kv, c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
+    default: TL_TRY(launch_k(c, attn_decode_kernel<128>, dim3(grid), dim3(128), 0, c->act_qkv, c->act_o, c->act_o16, rows, c->kv, c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
   }
   return prof_stop(c, TL_PROF_ATTN);
 }
@@ -550,6 +553,33 @@ int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
   return prof_stop(c, TL_PROF_ATTN);
 }
 
+// Whether the few-row GEMV for W (nmat matrices) applies the RMSNorm in its
+// own activation staging (the streamed GEMV does; its fallback does not).
+bool gemv_norms_itself(tl_ctx* c, const MatView& W, int nmat) {
+  return gs_plan(W.fmt, W.N, W.K, W.group, nmat, c->n_sms).ok;
+}
+
+// RMSNorm(hbuf rows) * g feeding a projection of W on `path`.  Returns the
+// GEMV's activation source and norm arguments; launches the separate norm
+// kernel (fp32 act_a + fp16 act_a16, and the h_in copy) only where a
+// projection that needs it can run: the tensor-core variant (more than 8 rows)
+// or a GEMV that does not normalise itself.
+int norm_for_proj(tl_ctx* c, int max_rows, int path, const int32_t* n, float* hbuf, const int32_t* map,
+                  const float* g, float* h_in, const MatView& W, int nmat, const float** X, GsNorm* nrm,
+                  bool* use_nrm) {
+  const bool fused = path != PATH_TC && gemv_norms_itself(c, W, nmat);
+  const bool tc_possible = path != PATH_GEMV && max_rows > kGemvMaxRows;
+  *use_nrm = fused;
+  *nrm = GsNorm{g, map, c->cfg.rms_eps, h_in};
+  *X = fused ? hbuf : c->act_a;
+  if (!fused || tc_possible) {
+    const int min_rows = (fused && path == PATH_AUTO) ? kGemvMaxRows : 0;  // <= 8 rows: the GEMV normalises
+    TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, hbuf, map, n, c->cfg.d, g, c->cfg.rms_eps,
+                    c->act_a, h_in, c->act_a16, nullptr, 0, min_rows));
+  }
+  return TL_OK;
+}
+
 // One transformer block on the rows of `rows`; hidden rows live in hbuf
 // (indexed through map, or by row when map is null).
 // prompt = rows are consecutive positions of one lane (tiled causal attention).
@@ -557,32 +587,35 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
               int slot_base, int slot_stride, float* h_in, bool prompt = false, int path = PATH_AUTO) {
   if (prompt) path = max_rows > kGemvMaxRows ? PATH_TC : PATH_GEMV;
   const int d = c->cfg.d, F = c->cfg.ffn;
-  const float eps = c->cfg.rms_eps;
-  TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, hbuf, map, rows.n, d, w.g1, eps, c->act_a, h_in, c->act_a16,
-                                                       nullptr, 0));
+  const float* X = nullptr;
+  GsNorm nrm{};
+  bool use_nrm = false;
+  TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g1, h_in, w.wqkv, 1, &X, &nrm, &use_nrm));
   ProjOut o{};
   o.epi = EPI_STORE;
   o.out = c->act_qkv;
   o.ldo = 3 * d;
-  TL_TRY(proj(c, max_rows, path, c->act_a, 0, rows.n, w.wqkv, &w.mqkv, nullptr, nullptr, o, nullptr));
-  TL_TRY(launch_k(c, rope_kv_kernel, dim3(max_rows), dim3(d / 2), 0, c->act_qkv, c->act_q, rows, c->kv, c->rope, slot_base,
-                                                     slot_stride, nullptr, c->status));
-  if (prompt)
+  TL_TRY(proj(c, max_rows, path, X, 0, rows.n, w.wqkv, &w.mqkv, nullptr, nullptr, o, nullptr, TL_PROF_PROJ,
+              use_nrm ? &nrm : nullptr));
+  if (prompt) {
+    TL_TRY(launch_k(c, rope_kv_kernel, dim3(max_rows), dim3(d / 2), 0, c->act_qkv, c->act_q, rows, c->kv, c->rope,
+                    slot_base, slot_stride, nullptr, c->status));
     TL_TRY(attn_prefill_launch(c, max_rows, rows, slot_base));
-  else
-    TL_TRY(attn_launch(c, max_rows, rows, slot_base, slot_stride));
+  } else {
+    TL_TRY(attn_launch(c, max_rows, rows, slot_base, slot_stride));  // RoPE and the KV append run inside
+  }
   ProjOut r{};
   r.epi = EPI_RESID;
   r.h = hbuf;
   r.map = map;
   TL_TRY(proj(c, max_rows, path, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
-  TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, hbuf, map, rows.n, d, w.g2, eps, c->act_a, nullptr,
-                                                       c->act_a16, nullptr, 0));
+  TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g2, nullptr, w.wg, 2, &X, &nrm, &use_nrm));
   ProjOut sw{};
   sw.epi = EPI_SWIGLU;
   sw.out = c->act_u;
   sw.ldo = F;
-  TL_TRY(proj(c, max_rows, path, c->act_a, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16));
+  TL_TRY(proj(c, max_rows, path, X, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16, TL_PROF_PROJ,
+              use_nrm ? &nrm : nullptr));
   return proj(c, max_rows, path, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr);
 }
 
@@ -627,10 +660,12 @@ int pre_blocks_for_entered(tl_ctx* c, int max_rows) {
 // Boundary stage, head part, for the lanes in rows[1]: final norm, head,
 // argmax, and in decode mode the token bookkeeping and embedding.
 int head_core(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax, int32_t* tok_out, int32_t* dep_out,
-              int n_new, int path = PATH_AUTO) {
+              int n_new, int path = PATH_AUTO, int mark_entered = 1) {
   const Rows& B = c->rows[1];
-  TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, c->h, B.lane, B.n, c->cfg.d, c->g_final, c->cfg.rms_eps,
-                                                       c->act_a, nullptr, c->act_a16, nullptr, 0));
+  const float* X = nullptr;
+  GsNorm nrm{};
+  bool use_nrm = false;
+  TL_TRY(norm_for_proj(c, max_rows, path, B.n, c->h, B.lane, c->g_final, nullptr, c->head, 1, &X, &nrm, &use_nrm));
   ProjOut o{};
   o.epi = EPI_ARGMAX;
   o.logits = logits;
@@ -639,10 +674,11 @@ int head_core(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax,
   o.part_val = c->part_val;
   o.part_idx = c->part_idx;
   o.n_parts_dev = c->head_nparts;
-  TL_TRY(proj(c, max_rows, path, c->act_a, 0, B.n, c->head, &c->mhead, nullptr, nullptr, o, nullptr, TL_PROF_HEAD));
+  TL_TRY(proj(c, max_rows, path, X, 0, B.n, c->head, &c->mhead, nullptr, nullptr, o, nullptr, TL_PROF_HEAD,
+              use_nrm ? &nrm : nullptr));
   TL_TRY(launch_k(c, head_finalize_kernel, dim3(max_rows), dim3(256), 0, B, c->lanes, c->part_val, c->part_idx, c->head_nparts, mode,
                                                         argmax, tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
-                                                        c->cfg.max_seq, c->status, &c->counters[1]));
+                                                        c->cfg.max_seq, mark_entered, c->status, &c->counters[1]));
   return TL_OK;
 }
 
@@ -1065,12 +1101,21 @@ extern "C" int tl_embed_next(tl_ctx* c, const uint8_t* dev_mask, const int32_t* 
   return pre_blocks_for_entered(c, c->cfg.max_lanes);
 }
 
+// The tick's three row tables (boundary -> rows[1], entered -> rows[2],
+// loop -> rows[0]) and alive count from one kernel; with conditional nodes it
+// also chooses their bodies.
+static int plan_tick(tl_ctx* c, int n_lanes, const TickConds& tc) {
+  return launch_k(c, plan_tick_kernel, dim3(1), dim3(1024), 0, c->lanes, n_lanes, c->rows[1], c->rows[2], c->rows[0],
+                  c->alive, c->cfg.max_seq, tc, kGemvMaxRows, c->body_kernels, &c->counters[2]);
+}
+
 // One decode tick: boundary stage (head, tokens, embedding, pre blocks) for
-// lanes whose loop finished, then one loop iteration for lanes in their loop.
+// lanes whose loop finished, then one loop iteration for lanes in their loop
+// (including the lanes that just entered).
 static int enqueue_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
-  TL_TRY(build_rows(c, 1, SEL_BOUNDARY, nullptr, nullptr, nullptr, c->alive, n_lanes));
-  TL_TRY(head_stage(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new));
-  TL_TRY(build_rows(c, 0, SEL_LOOP, nullptr, nullptr, nullptr, nullptr, n_lanes));
+  TL_TRY(plan_tick(c, n_lanes, TickConds{}));
+  TL_TRY(head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_AUTO, 0));
+  TL_TRY(pre_blocks(c, n_lanes));
   return loop_iteration(c, n_lanes, nullptr);
 }
 
@@ -1123,43 +1168,46 @@ static int capture_body(tl_ctx* c, cudaGraph_t body, int64_t* n_kernels, F fn) {
   return check_cuda(e);
 }
 
-// The tick as a CUDA graph with device-chosen branches: the row-table kernel
-// of each stage sets a conditional node, so a stage with no rows runs nothing
-// and a stage runs either its CUDA-core GEMV variant (<= 8 rows) or its
-// tensor-core variant, never both.  Every kernel reads its row count from
-// device memory, so one capture serves every tick of a decode with the same
-// lanes, token budget, outputs and early-exit parameters.
-//   rows(boundary) -> SWITCH { norm, head, argmax + token + embedding: GEMV | tensor cores }
-//   rows(entered)  -> SWITCH { pre blocks: GEMV | tensor cores }
-//   rows(loop)     -> SWITCH { loop body + exit rule: GEMV | tensor cores }
+// The tick as a CUDA graph with device-chosen branches: one planning kernel
+// builds the three row tables and sets one conditional node per stage, so a
+// stage with no rows runs nothing and a stage runs either its CUDA-core GEMV
+// variant (<= 8 rows) or its tensor-core variant, never both.  Every kernel
+// reads its row count from device memory, so one capture serves every tick of
+// a decode with the same lanes, token budget, outputs and early-exit
+// parameters.
+//   plan -> SWITCH { norm, head, argmax + token + embedding: GEMV | tensor cores }
+//        -> SWITCH { pre blocks of the entering lanes: GEMV | tensor cores }
+//        -> SWITCH { loop body + exit rule: GEMV | tensor cores }
 static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out, int32_t* kcount) {
-  cudaGraphConditionalHandle hb, he, hl;
+  TickConds tc{};
+  const bool pre = c->cfg.n_pre > 0;
+  for (int t = 0; t < 3; ++t)
+    if (t != 1 || pre) TL_TRY(new_handle(c->stream, &tc.h[t]));
+  tc.use = pre ? 7 : 5;
+  TL_TRY(plan_tick(c, n_lanes, tc));
   cudaGraph_t body[2];
   int64_t nk[2] = {0, 0};
   // boundary rows -> head (CUDA-core GEMV for <= 8 rows, tensor cores above)
-  TL_TRY(new_handle(c->stream, &hb));
-  TL_TRY(build_rows(c, 1, SEL_BOUNDARY, nullptr, nullptr, nullptr, c->alive, n_lanes, hb, COND_SWITCH, c->body_kernels + 0));
-  TL_TRY(add_conditional(c->stream, hb, cudaGraphCondTypeSwitch, 2, body));
-  TL_TRY(capture_body(c, body[0], &nk[0], [&] { return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_GEMV); }));
-  TL_TRY(capture_body(c, body[1], &nk[1], [&] { return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_TC); }));
+  TL_TRY(add_conditional(c->stream, tc.h[0], cudaGraphCondTypeSwitch, 2, body));
+  TL_TRY(capture_body(c, body[0], &nk[0], [&] {
+    return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_GEMV, 0);
+  }));
+  TL_TRY(capture_body(c, body[1], &nk[1], [&] {
+    return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_TC, 0);
+  }));
   kcount[0] = (int32_t)nk[0];
   kcount[1] = (int32_t)nk[1];
   // entered rows -> pre blocks
-  TL_TRY(new_handle(c->stream, &he));
-  TL_TRY(build_rows(c, 2, SEL_ENTERED, nullptr, nullptr, nullptr, nullptr, n_lanes, he, COND_SWITCH, c->body_kernels + 2));
-  if (c->cfg.n_pre > 0) {
-    TL_TRY(add_conditional(c->stream, he, cudaGraphCondTypeSwitch, 2, body));
+  kcount[2] = kcount[3] = 0;
+  if (pre) {
+    TL_TRY(add_conditional(c->stream, tc.h[1], cudaGraphCondTypeSwitch, 2, body));
     TL_TRY(capture_body(c, body[0], &nk[0], [&] { return pre_blocks(c, n_lanes, PATH_GEMV); }));
     TL_TRY(capture_body(c, body[1], &nk[1], [&] { return pre_blocks(c, n_lanes, PATH_TC); }));
     kcount[2] = (int32_t)nk[0];
     kcount[3] = (int32_t)nk[1];
-  } else {
-    kcount[2] = kcount[3] = 0;
   }
   // loop rows -> loop body
-  TL_TRY(new_handle(c->stream, &hl));
-  TL_TRY(build_rows(c, 0, SEL_LOOP, nullptr, nullptr, nullptr, nullptr, n_lanes, hl, COND_SWITCH, c->body_kernels + 4));
-  TL_TRY(add_conditional(c->stream, hl, cudaGraphCondTypeSwitch, 2, body));
+  TL_TRY(add_conditional(c->stream, tc.h[2], cudaGraphCondTypeSwitch, 2, body));
   TL_TRY(capture_body(c, body[0], &nk[0], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_GEMV); }));
   TL_TRY(capture_body(c, body[1], &nk[1], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_TC); }));
   kcount[4] = (int32_t)nk[0];
@@ -1202,7 +1250,7 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   c->tick_tok = tok_out;
   c->tick_dep = dep_out;
   c->tick_ee = c->ee;
-  c->tick_launches = 3;  // the three row-table kernels outside the conditional bodies
+  c->tick_launches = 1;  // the planning kernel outside the conditional bodies
   return TL_OK;
 }
 

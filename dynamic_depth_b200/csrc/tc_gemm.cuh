@@ -377,13 +377,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     cluster.sync();
     const int z = blockIdx.z;
     const int f0 = (z * 128) / S, nf = ((z + 1) * 128) / S - f0;
+    const float* rz[8];
+#pragma unroll
+    for (int zz = 0; zz < 8; ++zz) rz[zz] = cluster.map_shared_rank(red, zz < S ? zz : 0);
     for (int i = threadIdx.x; i < nf * ncols; i += blockDim.x) {
       const int tt = f0 + i % nf, j = i / nf;
+      float pa[8], pb[8];
+#pragma unroll
+      for (int zz = 0; zz < 8; ++zz) {  // all remote loads first, then the sum in split order
+        pa[zz] = zz < S ? rz[zz][j * 128 + tt] : 0.f;
+        if constexpr (NMAT == 2) pb[zz] = zz < S ? rz[zz][(NT + j) * 128 + tt] : 0.f;
+      }
       float a = 0.f, b = 0.f;
-      for (int zz = 0; zz < S; ++zz) {
-        const float* rz = cluster.map_shared_rank(red, zz);
-        a += rz[j * 128 + tt];
-        if constexpr (NMAT == 2) b += rz[(NT + j) * 128 + tt];
+#pragma unroll
+      for (int zz = 0; zz < 8; ++zz) {
+        if (zz < S) {
+          a += pa[zz];
+          if constexpr (NMAT == 2) b += pb[zz];
+        }
       }
       if (m0 + tt < p.N) tc_emit<EPI>(p, n0 + j, m0 + tt, a, b);
     }
