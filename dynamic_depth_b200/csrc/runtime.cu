@@ -4,6 +4,7 @@
 // waits are the lagged "lanes still alive" polls of tl_decode and the explicit
 // synchronisations of tl_generate / tl_stats_get.
 #include <cstdio>
+#include <cstdlib>
 #include <array>
 #include <cstring>
 #include <string>
@@ -833,6 +834,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->ws = (char*)dev_ws;
   c->ws_bytes = bytes;
   c->hd = cfg->d / cfg->n_heads;
+  if (const char* e = std::getenv("TL_PDL")) c->pdl = std::strcmp(e, "0") != 0;
   char* w = c->ws;
   // weight views
   auto specs = mat_specs(cfg);

@@ -60,6 +60,12 @@ struct TcCfg {
   // split-K parks a [NMAT][NT][128] fp32 partial tile in the stage buffers
   static constexpr bool SPLIT_OK = NMAT * NT * 128 * 4 <= STAGES * stage_bytes;
   static_assert(STAGES >= 2, "tile does not fit in shared memory");
+  // TMEM is allocated before the programmatic-dependency wait, so a CTA may
+  // allocate while a CTA of the previous kernel on its SM still has to.  The
+  // smallest tile uses ~95 KB of shared memory, so any tile holding more than
+  // 64 columns must leave no room for a second tensor-core CTA on its SM; two
+  // 64-column CTAs fit TMEM's 512 columns together.
+  static_assert(TMEM_COLS <= 64 || SMEM > 133 * 1024, "TMEM could be oversubscribed by co-resident CTAs");
 };
 
 // K-major, SWIZZLE_128B canonical layout: 8-row groups 1024 B apart.

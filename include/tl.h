@@ -129,6 +129,9 @@ int tl_weights_bytes(const tl_config* cfg, size_t* out_bytes);
 /* Carve the caller's workspace (>= tl_workspace_bytes, 256-byte aligned) and
  * bind the stream.  The workspace must stay allocated until tl_destroy().
  * Launches initialisation kernels (RoPE table, page table, lane state).
+ * Kernels launch with programmatic dependent launch (each may start while
+ * its predecessor finishes); the environment variable TL_PDL=0, read here,
+ * launches them fully serialised instead.
  * TL_EINVAL bad cfg/pointer; TL_ENOMEM workspace too small; TL_ECUDA. */
 int tl_create(const tl_config* cfg, void* dev_workspace, size_t workspace_bytes,
               void* cuda_stream, tl_ctx** out_ctx);

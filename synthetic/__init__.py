@@ -69,7 +69,12 @@ M407_BF16LOOP = replace(M407, fmt_loop=BF16)
 # no pre blocks, 24-layer loop body, BF16 everywhere.
 M1B4 = ModelShape(49152, 2048, 16, 5632, 0, 24, BF16, BF16, BF16, 0)
 
-SHAPES = {"tiny": TINY, "m407": M407, "m407_bf16loop": M407_BF16LOOP, "m1b4": M1B4}
+# The same layout at test size (every structural feature of M1B4: BF16
+# everywhere, 128-wide heads, no pre blocks, a multi-layer loop body, a vocab
+# and FFN that are not multiples of the 128-row tile).
+M1B4_MINI = ModelShape(4000, 256, 2, 704, 0, 3, BF16, BF16, BF16, 0)
+
+SHAPES = {"tiny": TINY, "m407": M407, "m407_bf16loop": M407_BF16LOOP, "m1b4": M1B4, "m1b4_mini": M1B4_MINI}
 
 
 def matrix_shapes(shape: ModelShape) -> list[Tuple[str, Tuple[int, int]]]:
@@ -166,4 +171,16 @@ def workload(name: str) -> Workload:
     if name == "m1b4_prefix256":
         return Workload("m1b4_prefix256", M1B4, 256, 64, 64, tuple(int(x) for x in uniform_L(256)),
                         shared_prefix=1024)
+    if name == "m1b4_mini_prefix":
+        return Workload("m1b4_mini_prefix", M1B4_MINI, 4, 8, 4, tuple(int(x) for x in uniform_L(4)),
+                        shared_prefix=96)
     raise KeyError(name)
+
+
+def prefix_prompts(wl: Workload) -> Tuple[np.ndarray, np.ndarray]:
+    """Shared-prefix workloads: the common prefix (int32 [shared_prefix], from
+    PCG64(1)) and each lane's suffix (int32 [n_lanes, prompt_len], from
+    PCG64(3)); lane i's prompt is prefix + suffix[i]."""
+    pre = prompts(1, wl.shared_prefix, wl.shape.vocab, seed=1)[0]
+    suf = prompts(wl.n_lanes, wl.prompt_len, wl.shape.vocab, seed=3)
+    return pre, suf

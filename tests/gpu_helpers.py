@@ -53,9 +53,10 @@ def status_clean(m):
     return st
 
 
-def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None):
+def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None, prefill=None):
     """Drive the CUDA path with the oracle's tokens (prefill, head, then
     embed_next + loop steps until every lane's loop finished, head again).
+    prefill(i, lane) replaces the plain m.prefill of prompt i when given.
     Returns (oracle results, GPU logits [n_lanes, n_new, V], GPU argmax, GPU
     depths [n_lanes, n_new])."""
     import torch as _t
@@ -76,7 +77,10 @@ def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None):
     tok = torch.zeros(max_lanes, dtype=torch.int32, device=dev)
     m.set_early_exit(ee.tau, ee.min_L, ee.patience, ee.peek_every)
     for i, ln in enumerate(lanes):
-        m.prefill(ln, prompts[i], Ls[i])
+        if prefill is None:
+            m.prefill(ln, prompts[i], Ls[i])
+        else:
+            prefill(i, ln)
     out_logits = np.zeros((n, n_new, V))
     out_arg = np.zeros((n, n_new), dtype=np.int64)
     depths = np.zeros((n, n_new), dtype=np.int64)
