@@ -92,6 +92,18 @@ class LoopedLM:
         check(lib().tl_prefill(self.h, lane, tok.ctypes.data, len(tok), L, share_from, shared_tokens,
                                _ptr(hidden_out)), "tl_prefill")
 
+    def prefill_batch(self, lanes, prompts, per_lane_L, share_from: int = -1, shared_tokens: int = 0):
+        """Prompts of several lanes in one pass (tl_prefill_batch); prompts: a list of int sequences."""
+        ln = np.ascontiguousarray(lanes, dtype=np.int32)
+        toks = [np.ascontiguousarray(p, dtype=np.int32) for p in prompts]
+        T = np.array([len(t) for t in toks], dtype=np.int32)
+        L = np.ascontiguousarray(per_lane_L, dtype=np.int32)
+        if not (len(ln) == len(toks) == len(L)):
+            raise ValueError("lanes, prompts and per_lane_L differ in length")
+        flat = np.concatenate(toks) if toks else np.zeros(0, np.int32)
+        check(lib().tl_prefill_batch(self.h, len(ln), ln.ctypes.data, flat.ctypes.data, T.ctypes.data, L.ctypes.data,
+                                     share_from, shared_tokens), "tl_prefill_batch")
+
     def set_early_exit(self, tau: float, min_L: int = 2, patience: int = 0, peek_every: int = 1):
         check(lib().tl_set_early_exit(self.h, float(tau), min_L, patience, peek_every), "tl_set_early_exit")
 

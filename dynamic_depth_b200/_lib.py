@@ -47,6 +47,8 @@ SIGNATURES = {
     "tl_round_bf16": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p]),
     "tl_prefill": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                              C.c_void_p]),
+    "tl_prefill_batch": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                   C.c_int32, C.c_int32]),
     "tl_set_early_exit": (C.c_int, [C.c_void_p, C.c_double, C.c_int32, C.c_int32, C.c_int32]),
     "tl_loop_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "tl_head_logits": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),

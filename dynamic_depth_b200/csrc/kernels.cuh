@@ -748,9 +748,11 @@ attn_decode_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half*
 
 // --------------------------------------------------- prefill attention ----
 //
-// Causal attention for a block of consecutive prompt rows of one lane: CTA
-// (qb, h) takes query rows r in [64 qb, 64 qb + 64) (positions rows.pos[r],
-// consecutive) and walks key blocks of 64 positions from 0 up to its last
+// Causal attention for blocks of consecutive prompt rows of one lane each: CTA
+// (qb, h) takes query tile qb = tiles[qb] = (first row, row count <= 64) of
+// the row table (every row of a tile belongs to one lane and the positions
+// rows.pos[r] are consecutive; tiles == null: rows 64 qb .. 64 qb + 63 of a
+// one-lane table) and walks key blocks of 64 positions from 0 up to its last
 // query position, staging K and V once per block in shared memory (fp32) and
 // keeping a running max / sum per query row.  256 threads: for the scores
 // thread (ty, tx) owns rows 4ty..4ty+3 and keys 4tx..4tx+3; for the output it
@@ -758,7 +760,7 @@ attn_decode_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half*
 template <int HD>
 __global__ void __launch_bounds__(256)
 attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
-                    KVGeom g, int slot, int32_t* __restrict__ status) {
+                    const int2* __restrict__ tiles, KVGeom g, int slot, int32_t* __restrict__ status) {
   pdl_launch_dependents();
   pdl_wait();
   constexpr int BQ = 64, BK = 64, DPT = HD / 16;
@@ -768,12 +770,13 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* 
   float* Vs = Ks + HD * BK;                        // [BK][HD]
   float* Ps = Vs + BK * HD;                        // [BQ][BK + 1]
   const int n = rows.n[0];
-  const int r0 = blockIdx.x * BQ, h = blockIdx.y;
-  if (r0 >= n) return;
+  const int2 tile = tiles ? tiles[blockIdx.x] : make_int2(blockIdx.x * BQ, min(BQ, n - (int)blockIdx.x * BQ));
+  const int r0 = tile.x, h = blockIdx.y;
+  if (r0 >= n || tile.y <= 0) return;
   const int ln = rows.lane[r0];
   const int d = g.H * HD;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int nq = min(BQ, n - r0);
+  const int nq = min(min(BQ, tile.y), n - r0);
   const int pos_first = rows.pos[r0];
   const int pos_last = pos_first + nq - 1;
   const float scale = rsqrtf((float)HD);
@@ -1073,13 +1076,16 @@ __global__ void decode_init_kernel(LaneState* __restrict__ lanes, int n_lanes, c
   st.n_target = n_new;
 }
 
-// Lane state after its prompt: hidden of the last prompt row (row Tn - 1 of
-// hrows, position last_pos), cap = depth = L, waiting for the head.
-__global__ void prefill_finish_kernel(LaneState* __restrict__ lanes, int ln, int Tn, int last_pos, int L,
-                                      const float* __restrict__ hrows, float* __restrict__ h, int d) {
+// Lane states after a batch of prompts: lane lanes[i] takes hidden row
+// last_row[i] of hrows (its position last_pos[i]), cap = depth = L[i].
+__global__ void prefill_finish_batch_kernel(LaneState* __restrict__ lanes, const int32_t* __restrict__ info, int n,
+                                            const float* __restrict__ hrows, float* __restrict__ h, int d) {
   pdl_launch_dependents();
   pdl_wait();
-  for (int k = threadIdx.x; k < d; k += blockDim.x) h[(int64_t)ln * d + k] = hrows[(int64_t)(Tn - 1) * d + k];
+  const int i = blockIdx.x;
+  if (i >= n) return;
+  const int ln = info[4 * i], last_row = info[4 * i + 1], last_pos = info[4 * i + 2], L = info[4 * i + 3];
+  for (int k = threadIdx.x; k < d; k += blockDim.x) h[(int64_t)ln * d + k] = hrows[(int64_t)last_row * d + k];
   if (threadIdx.x == 0) {
     LaneState& st = lanes[ln];
     st.L_req = L;
@@ -1095,18 +1101,6 @@ __global__ void prefill_finish_kernel(LaneState* __restrict__ lanes, int ln, int
     st.token = -1;
     st.entered = 0;
   }
-}
-
-// Rows of a prefill: row t is position pos0 + t of lane ln at iteration 0.
-__global__ void prefill_rows_kernel(Rows rows, int ln, int pos0, int T) {
-  pdl_launch_dependents();
-  pdl_wait();
-  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
-    rows.lane[t] = ln;
-    rows.pos[t] = pos0 + t;
-    rows.iter[t] = 0;
-  }
-  if (blockIdx.x == 0 && threadIdx.x == 0) rows.n[0] = T;
 }
 
 }  // namespace tl

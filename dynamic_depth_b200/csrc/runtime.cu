@@ -5,6 +5,7 @@
 // synchronisations of tl_generate / tl_stats_get.
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <array>
 #include <cstring>
 #include <string>
@@ -48,7 +49,7 @@ static bool cfg_valid(const tl_config* c) {
   if (!(c->rms_eps >= 0.f) || !(c->rope_base > 0.f)) return false;
   if (c->max_lanes < 1 || c->max_lanes > 1024 || c->max_seq < 1 || c->L_max < 1) return false;
   if (c->kv_page_tokens < 32 || (c->kv_page_tokens & (c->kv_page_tokens - 1))) return false;
-  if (c->kv_pool_pages < 0 || c->max_prefill_tokens < 0 || c->max_prefill_tokens > c->max_seq) return false;
+  if (c->kv_pool_pages < 0 || c->max_prefill_tokens < 0) return false;
   return true;
 }
 
@@ -166,7 +167,7 @@ struct Layout {
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[4], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
-      mask_stage,
+      mask_stage, pf_n, pf_tiles, pf_info,
       out_tok, out_dep, status, counters, body_kernels, alive, total;
 };
 
@@ -213,6 +214,9 @@ static Layout make_layout(const tl_config* c) {
   L.tok_stage = take(R * 4);
   L.L_stage = take(lanes * 4);
   L.mask_stage = take(lanes);
+  L.pf_n = take((size_t)(c->L_max + 2) * 4);
+  L.pf_tiles = take((R / 64 + lanes + 2) * 8);
+  L.pf_info = take(lanes * 16);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
@@ -258,6 +262,9 @@ struct tl_ctx {
   float* part_val;
   int32_t* part_idx;
   int32_t *tok_stage, *L_stage, *out_tok, *out_dep, *status, *alive;
+  int32_t* pf_n;     // prompt batches: row count of each stage (stage l = loop iteration l)
+  int2* pf_tiles;    // prompt batches: attention tiles (first row, rows)
+  int32_t* pf_info;  // prompt batches: per lane (lane, last row, last position, L)
   uint8_t* mask_stage;
   unsigned long long* counters;  // 0 lane iterations, 1 tokens, 2 kernels run inside conditional graph bodies
   int32_t* body_kernels;          // [stage][variant] kernels of each conditional body (graph ticks)
@@ -529,26 +536,26 @@ int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int sl
 
 // Causal attention over a prompt block (rows of one lane, consecutive positions).
 template <int HD>
-int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
+int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot, const int2* tiles, int n_tiles) {
   const size_t smem = (size_t)(3 * HD * 64 + 64 * 65) * 4;
   static bool attr_done = false;
   if (!attr_done) {
     TL_CUDA(cudaFuncSetAttribute(attn_prefill_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr_done = true;
   }
-  dim3 grid((max_rows + 63) / 64, c->cfg.n_heads);
-  TL_TRY(launch_k(c, attn_prefill_kernel<HD>, dim3(grid), dim3(256), smem, c->act_q, c->act_o, c->act_o16, rows, c->kv, slot,
-                                                            c->status));
+  dim3 grid(tiles ? n_tiles : (max_rows + 63) / 64, c->cfg.n_heads);
+  TL_TRY(launch_k(c, attn_prefill_kernel<HD>, dim3(grid), dim3(256), smem, c->act_q, c->act_o, c->act_o16, rows,
+                  tiles, c->kv, slot, c->status));
   return TL_OK;
 }
 
-int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot) {
+int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot, const int2* tiles, int n_tiles) {
   TL_TRY(prof_start(c, TL_PROF_ATTN));
   int st;
   switch (c->hd) {
-    case 32: st = attn_prefill_launch_hd<32>(c, max_rows, rows, slot); break;
-    case 64: st = attn_prefill_launch_hd<64>(c, max_rows, rows, slot); break;
-    default: st = attn_prefill_launch_hd<128>(c, max_rows, rows, slot); break;
+    case 32: st = attn_prefill_launch_hd<32>(c, max_rows, rows, slot, tiles, n_tiles); break;
+    case 64: st = attn_prefill_launch_hd<64>(c, max_rows, rows, slot, tiles, n_tiles); break;
+    default: st = attn_prefill_launch_hd<128>(c, max_rows, rows, slot, tiles, n_tiles); break;
   }
   TL_TRY(st);
   return prof_stop(c, TL_PROF_ATTN);
@@ -583,9 +590,11 @@ int norm_for_proj(tl_ctx* c, int max_rows, int path, const int32_t* n, float* hb
 
 // One transformer block on the rows of `rows`; hidden rows live in hbuf
 // (indexed through map, or by row when map is null).
-// prompt = rows are consecutive positions of one lane (tiled causal attention).
+// prompt = rows are runs of consecutive positions of one lane each, attended
+// causally in the n_tiles tiles of `tiles`.
 int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int32_t* map, const BlockW& w,
-              int slot_base, int slot_stride, float* h_in, bool prompt = false, int path = PATH_AUTO) {
+              int slot_base, int slot_stride, float* h_in, bool prompt = false, int path = PATH_AUTO,
+              const int2* tiles = nullptr, int n_tiles = 0) {
   if (prompt) path = max_rows > kGemvMaxRows ? PATH_TC : PATH_GEMV;
   const int d = c->cfg.d, F = c->cfg.ffn;
   const float* X = nullptr;
@@ -601,7 +610,7 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   if (prompt) {
     TL_TRY(launch_k(c, rope_kv_kernel, dim3(max_rows), dim3(d / 2), 0, c->act_qkv, c->act_q, rows, c->kv, c->rope,
                     slot_base, slot_stride, nullptr, c->status));
-    TL_TRY(attn_prefill_launch(c, max_rows, rows, slot_base));
+    TL_TRY(attn_prefill_launch(c, max_rows, rows, slot_base, tiles, n_tiles));
   } else {
     TL_TRY(attn_launch(c, max_rows, rows, slot_base, slot_stride));  // RoPE and the KV append run inside
   }
@@ -903,6 +912,9 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->part_idx = (int32_t*)(w + lay.part_idx);
   c->tok_stage = (int32_t*)(w + lay.tok_stage);
   c->L_stage = (int32_t*)(w + lay.L_stage);
+  c->pf_n = (int32_t*)(w + lay.pf_n);
+  c->pf_tiles = (int2*)(w + lay.pf_tiles);
+  c->pf_info = (int32_t*)(w + lay.pf_info);
   c->mask_stage = (uint8_t*)(w + lay.mask_stage);
   c->out_tok = (int32_t*)(w + lay.out_tok);
   c->out_dep = (int32_t*)(w + lay.out_dep);
@@ -1023,62 +1035,156 @@ extern "C" int tl_set_early_exit(tl_ctx* c, double tau, int32_t min_L, int32_t p
   return TL_OK;
 }
 
+// Prompts of several lanes in one pass over the weights.  Every block runs
+// once on the rows of all lanes (the loop's iteration l on the lanes whose L
+// exceeds l: lanes are ordered by L, deepest first, so those rows are a prefix
+// of the row table); attention runs per lane, in tiles of up to 64 rows that
+// never straddle two lanes.
+struct PromptLane {
+  int lane;
+  const int32_t* tokens;
+  int T, L;
+};
+
+static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t share_from, int32_t shared_tokens,
+                        float* dev_hidden_out) {
+  const tl_config& cfg = c->cfg;
+  const int n = (int)in.size();
+  if (n < 1 || n > cfg.max_lanes) return TL_EINVAL;
+  const int P = cfg.n_pre, Lb = cfg.n_loop_layers, pps = c->lay.pages_per_seq, pt = cfg.kv_page_tokens;
+  std::vector<char> seen(cfg.max_lanes, 0);
+  std::vector<int> share_pages(n, 0);
+  int64_t total = 0;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    const PromptLane& p = in[i];
+    if (p.lane < 0 || p.lane >= cfg.max_lanes || seen[p.lane] || !p.tokens || p.T < 1 || p.T > cfg.max_seq ||
+        p.L < 1 || p.L > cfg.L_max)
+      return TL_EINVAL;
+    seen[p.lane] = 1;
+    for (int t = 0; t < p.T; ++t)
+      if (p.tokens[t] < 0 || p.tokens[t] >= cfg.vocab) return TL_EINVAL;
+    if (share_from >= 0) {
+      // the donor keeps its pages: it is not re-run in this batch and holds every slot this lane needs
+      if (share_from >= cfg.max_lanes || share_from == p.lane || c->lane_L[share_from] < p.L || shared_tokens < 0 ||
+          shared_tokens > p.T)
+        return TL_EINVAL;
+      // whole pages only, and never the last prompt position (this lane computes it)
+      share_pages[i] = (shared_tokens < p.T ? shared_tokens : p.T - 1) / pt;
+    }
+    total += p.T - share_pages[i] * pt;
+    need += (int64_t)(P + p.L * Lb) * (pps - share_pages[i]);
+  }
+  if (share_from >= 0 && seen[share_from]) return TL_EINVAL;
+  if (total > c->lay.max_prefill) return TL_EINVAL;
+  // pages: slots of the pre blocks and of iterations 1..L, for every position up to max_seq
+  for (int i = 0; i < n; ++i) release_lane_pages(c, in[i].lane);
+  if ((int64_t)c->free_pages.size() < need) return TL_ENOMEM;
+  const size_t per_lane = (size_t)c->lay.n_slots * pps;
+  for (int i = 0; i < n; ++i) {
+    const int used_slots = P + in[i].L * Lb;
+    int32_t* t = &c->h_page_table[(size_t)in[i].lane * per_lane];
+    const int32_t* donor = share_from >= 0 ? &c->h_page_table[(size_t)share_from * per_lane] : nullptr;
+    for (int sl = 0; sl < used_slots; ++sl)
+      for (int pg = 0; pg < pps; ++pg) {
+        int32_t id;
+        if (pg < share_pages[i]) {
+          id = donor[(size_t)sl * pps + pg];
+        } else {
+          id = c->free_pages.back();
+          c->free_pages.pop_back();
+        }
+        c->refcount[id]++;
+        t[(size_t)sl * pps + pg] = id;
+      }
+    c->lane_L[in[i].lane] = in[i].L;
+    TL_CUDA(cudaMemcpyAsync(c->page_table + (size_t)in[i].lane * per_lane, t, per_lane * 4, cudaMemcpyHostToDevice,
+                            c->stream));
+  }
+  // row table (deepest lanes first), tokens, attention tiles, per-lane finish info
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return in[a].L > in[b].L; });
+  std::vector<int32_t> r_lane, r_pos, r_iter, tok, info;
+  std::vector<int2> tiles;
+  std::vector<int64_t> rows_upto(n + 1, 0), tiles_upto(n + 1, 0);
+  r_lane.reserve(total);
+  r_pos.reserve(total);
+  tok.reserve(total);
+  for (int k = 0; k < n; ++k) {
+    const PromptLane& p = in[order[k]];
+    const int pos0 = share_pages[order[k]] * pt, Tn = p.T - pos0;
+    const int row0 = (int)r_lane.size();
+    for (int t = 0; t < Tn; ++t) {
+      r_lane.push_back(p.lane);
+      r_pos.push_back(pos0 + t);
+      tok.push_back(p.tokens[pos0 + t]);
+    }
+    for (int t0 = 0; t0 < Tn; t0 += 64) tiles.push_back(make_int2(row0 + t0, Tn - t0 < 64 ? Tn - t0 : 64));
+    info.insert(info.end(), {p.lane, row0 + Tn - 1, p.T - 1, p.L});
+    rows_upto[k + 1] = (int64_t)r_lane.size();
+    tiles_upto[k + 1] = (int64_t)tiles.size();
+  }
+  r_iter.assign(total, 0);
+  const int Lmax = in[order[0]].L;
+  std::vector<int32_t> stage_rows(Lmax), stage_tiles(Lmax);
+  for (int l = 0; l < Lmax; ++l) {
+    int k = 0;
+    while (k < n && in[order[k]].L > l) ++k;  // lanes 0..k-1 of the order run iteration l
+    stage_rows[l] = (int32_t)rows_upto[k];
+    stage_tiles[l] = (int32_t)tiles_upto[k];
+  }
+  const Rows& R = c->rows[3];
+  TL_CUDA(cudaMemcpyAsync(R.lane, r_lane.data(), total * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(R.pos, r_pos.data(), total * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(R.iter, r_iter.data(), total * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->tok_stage, tok.data(), total * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->pf_tiles, tiles.data(), tiles.size() * sizeof(int2), cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->pf_info, info.data(), info.size() * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->pf_n, stage_rows.data(), Lmax * 4, cudaMemcpyHostToDevice, c->stream));
+  Rows Rs = R;
+  Rs.n = c->pf_n;  // stage 0: every row (every lane has L >= 1)
+  const int all = (int)total;
+  TL_TRY(launch_k(c, embed_rows_kernel, dim3(all), dim3(256), 0, c->embed, c->tok_stage, all, cfg.d, c->hrows,
+                  c->status));
+  for (int b = 0; b < P; ++b)
+    TL_TRY(run_block(c, Rs, all, c->hrows, nullptr, c->pre[b], b, 0, nullptr, true, PATH_AUTO, c->pf_tiles,
+                     stage_tiles[0]));
+  for (int l = 0; l < Lmax; ++l) {
+    Rs.n = c->pf_n + l;
+    for (int m = 0; m < Lb; ++m)
+      TL_TRY(run_block(c, Rs, stage_rows[l], c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr, true,
+                       PATH_AUTO, c->pf_tiles, stage_tiles[l]));
+  }
+  TL_TRY(launch_k(c, prefill_finish_batch_kernel, dim3(n), dim3(256), 0, c->lanes, c->pf_info, n, c->hrows, c->h,
+                  cfg.d));
+  if (dev_hidden_out)
+    TL_CUDA(cudaMemcpyAsync(dev_hidden_out, c->hrows, (size_t)total * cfg.d * 4, cudaMemcpyDeviceToDevice,
+                            c->stream));
+  c->prefill_tokens += total;
+  // the host tables above are pageable: the copies have consumed them by the time cudaMemcpyAsync returns
+  return TL_OK;
+}
+
 extern "C" int tl_prefill(tl_ctx* c, int32_t lane, const int32_t* host_tokens, int32_t T, int32_t L,
                           int32_t share_from, int32_t shared_tokens, float* dev_hidden_out) {
   if (!c || !host_tokens) return TL_EINVAL;
   if (!c->loaded) return TL_ESTATE;
-  const tl_config& cfg = c->cfg;
-  if (lane < 0 || lane >= cfg.max_lanes || T < 1 || T > c->lay.max_prefill || L < 1 || L > cfg.L_max)
-    return TL_EINVAL;
-  for (int i = 0; i < T; ++i)
-    if (host_tokens[i] < 0 || host_tokens[i] >= cfg.vocab) return TL_EINVAL;
-  int share_pages = 0;
-  if (share_from >= 0) {
-    if (share_from >= cfg.max_lanes || share_from == lane || c->lane_L[share_from] < L || shared_tokens < 0 ||
-        shared_tokens > T)
-      return TL_EINVAL;
-    // whole pages only, and never the last prompt position (this lane computes it)
-    share_pages = (shared_tokens < T ? shared_tokens : T - 1) / cfg.kv_page_tokens;
+  return prefill_impl(c, {PromptLane{lane, host_tokens, T, L}}, share_from, shared_tokens, dev_hidden_out);
+}
+
+extern "C" int tl_prefill_batch(tl_ctx* c, int32_t n, const int32_t* lanes, const int32_t* host_tokens,
+                                const int32_t* T, const int32_t* L, int32_t share_from, int32_t shared_tokens) {
+  if (!c || !lanes || !host_tokens || !T || !L || n < 1) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  std::vector<PromptLane> in(n);
+  size_t off = 0;
+  for (int i = 0; i < n; ++i) {
+    if (T[i] < 1) return TL_EINVAL;
+    in[i] = PromptLane{lanes[i], host_tokens + off, T[i], L[i]};
+    off += (size_t)T[i];
   }
-  // pages: slots of the pre blocks and of iterations 1..L, for every position up to max_seq
-  const int P = cfg.n_pre, Lb = cfg.n_loop_layers, pps = c->lay.pages_per_seq;
-  const int used_slots = P + L * Lb;
-  const int need = used_slots * (pps - share_pages);
-  release_lane_pages(c, lane);
-  if ((int)c->free_pages.size() < need) return TL_ENOMEM;
-  const size_t per_lane = (size_t)c->lay.n_slots * pps;
-  int32_t* t = &c->h_page_table[(size_t)lane * per_lane];
-  const int32_t* donor = share_from >= 0 ? &c->h_page_table[(size_t)share_from * per_lane] : nullptr;
-  for (int s = 0; s < used_slots; ++s)
-    for (int p = 0; p < pps; ++p) {
-      int32_t pg;
-      if (p < share_pages) {
-        pg = donor[(size_t)s * pps + p];
-      } else {
-        pg = c->free_pages.back();
-        c->free_pages.pop_back();
-      }
-      c->refcount[pg]++;
-      t[(size_t)s * pps + p] = pg;
-    }
-  c->lane_L[lane] = L;
-  TL_CUDA(cudaMemcpyAsync(c->page_table + (size_t)lane * per_lane, t, per_lane * 4, cudaMemcpyHostToDevice, c->stream));
-  // rows: the positions not covered by the shared pages
-  const int pos0 = share_pages * cfg.kv_page_tokens;
-  const int Tn = T - pos0;
-  const Rows& R = c->rows[3];
-  TL_CUDA(cudaMemcpyAsync(c->tok_stage, host_tokens + pos0, (size_t)Tn * 4, cudaMemcpyHostToDevice, c->stream));
-  TL_TRY(launch_k(c, prefill_rows_kernel, dim3((Tn + 255) / 256), dim3(256), 0, R, lane, pos0, Tn));
-  TL_TRY(launch_k(c, embed_rows_kernel, dim3(Tn), dim3(256), 0, c->embed, c->tok_stage, Tn, cfg.d, c->hrows, c->status));
-  for (int b = 0; b < P; ++b) TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->pre[b], b, 0, nullptr, true));
-  for (int l = 0; l < L; ++l)
-    for (int m = 0; m < Lb; ++m)
-      TL_TRY(run_block(c, R, Tn, c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr, true));
-  TL_TRY(launch_k(c, prefill_finish_kernel, dim3(1), dim3(256), 0, c->lanes, lane, Tn, T - 1, L, c->hrows, c->h, cfg.d));
-  if (dev_hidden_out)
-    TL_CUDA(cudaMemcpyAsync(dev_hidden_out, c->hrows, (size_t)Tn * cfg.d * 4, cudaMemcpyDeviceToDevice, c->stream));
-  c->prefill_tokens += Tn;
-  return TL_OK;
+  return prefill_impl(c, in, share_from, shared_tokens, nullptr);
 }
 
 extern "C" int tl_loop_step(tl_ctx* c, const int32_t* dev_L, const uint8_t* dev_mask, uint8_t* dev_exit) {
@@ -1304,8 +1410,15 @@ extern "C" int tl_generate(tl_ctx* c, const int32_t* host_prompts, int32_t n_lan
   if (!c->loaded) return TL_ESTATE;
   if (n_lanes < 1 || n_lanes > c->cfg.max_lanes || n_new < 1 || T < 1 || T + n_new - 1 > c->cfg.max_seq)
     return TL_EINVAL;
-  for (int i = 0; i < n_lanes; ++i)
-    TL_TRY(tl_prefill(c, i, host_prompts + (size_t)i * T, T, host_L[i], -1, 0, nullptr));
+  if (T > c->lay.max_prefill) return TL_EINVAL;
+  // prompts in batches of as many lanes as the prompt rows allow
+  const int per_batch = (int)(c->lay.max_prefill / T);
+  for (int i0 = 0; i0 < n_lanes; i0 += per_batch) {
+    std::vector<PromptLane> in;
+    for (int i = i0; i < n_lanes && i < i0 + per_batch; ++i)
+      in.push_back(PromptLane{i, host_prompts + (size_t)i * T, T, host_L[i]});
+    TL_TRY(prefill_impl(c, in, -1, 0, nullptr));
+  }
   TL_CUDA(cudaMemcpyAsync(c->L_stage, host_L, (size_t)n_lanes * 4, cudaMemcpyHostToDevice, c->stream));
   TL_TRY(decode_impl(c, n_lanes, n_new, c->out_tok, c->out_dep));
   TL_CUDA(cudaMemcpyAsync(host_tok, c->out_tok, (size_t)n_lanes * n_new * 4, cudaMemcpyDeviceToHost, c->stream));

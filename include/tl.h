@@ -84,7 +84,8 @@ typedef struct tl_config {
     int32_t L_max;            /* largest per-lane loop count                      */
     int32_t kv_page_tokens;   /* tokens per KV page (power of two, >= 16)         */
     int32_t kv_pool_pages;    /* pages in the pool; 0 = one per lane/slot/page    */
-    int32_t max_prefill_tokens; /* rows of one prefill call; 0 = max_seq          */
+    int32_t max_prefill_tokens; /* prompt rows one prefill call computes, summed
+                                   over its lanes; 0 = max_seq                   */
 } tl_config;
 
 typedef struct tl_ctx tl_ctx;
@@ -174,7 +175,8 @@ int tl_round_bf16(const double* dev_w, int64_t n, uint16_t* dev_out, void* cuda_
  * token (tl_head_logits / tl_decode) with cap L.  Early exit does not apply to
  * the prompt.
  *   lane: 0..max_lanes-1 (any earlier content of the lane is dropped);
- *   host_tokens: int32 [T], ids in [0, vocab); 1 <= T <= max_prefill_tokens;
+ *   host_tokens: int32 [T], ids in [0, vocab); 1 <= T <= max_seq, and the
+ *     positions it computes (T minus the shared ones) <= max_prefill_tokens;
  *   L: 1..L_max;
  *   share_prefix_from_lane: -1, or a lane whose prompt starts with the same
  *     tokens and was prefilled at L' >= L; its full KV pages covering the first
@@ -182,10 +184,31 @@ int tl_round_bf16(const double* dev_w, int64_t n, uint16_t* dev_out, void* cuda_
  *     recomputed ("Benchmark Comparison" (measured benchmarks), section 2,
  *     SHARED prefix reuse); shared_tokens is rounded down to whole pages;
  *   dev_hidden_out: NULL or fp32 [T, d], the final hidden rows (before the
- *     head norm).
+ *     head norm) of the positions computed (all T without a shared prefix).
+ *   The donor must not be re-prefilled while lanes map its pages.
  * TL_EINVAL bad lane/T/L/token; TL_ENOMEM page pool exhausted. */
 int tl_prefill(tl_ctx* ctx, int32_t lane, const int32_t* host_tokens, int32_t T, int32_t L,
                int32_t share_prefix_from_lane, int32_t shared_tokens, float* dev_hidden_out);
+
+/* tl_prefill for n lanes in one pass: every block runs once over the rows of
+ * all n prompts (a wide causal batch on the tensor cores), iteration l over
+ * the lanes whose L exceeds l; attention stays per lane.  Same result per
+ * lane as n tl_prefill calls.  This is the prompt side of L-aware batching
+ * ("Dynamic-L Inference", "L-Aware Batching": one batch call with a loop
+ * count per lane).
+ *   lanes: host int32 [n], distinct, 0..max_lanes-1;
+ *   host_tokens: the n prompts back to back, lane i's T[i] ids after lane
+ *     i-1's;
+ *   T, L: host int32 [n], as for tl_prefill;
+ *   share_prefix_from_lane, shared_tokens: as for tl_prefill, applied to
+ *     every lane of the batch (the donor must not be one of them).
+ *   The positions computed, summed over the lanes, must be <=
+ *   max_prefill_tokens.
+ * TL_EINVAL bad arguments (nothing is changed); TL_ENOMEM page pool
+ * exhausted (the batch's lanes are left empty). */
+int tl_prefill_batch(tl_ctx* ctx, int32_t n, const int32_t* lanes, const int32_t* host_tokens,
+                     const int32_t* T, const int32_t* L, int32_t share_prefix_from_lane,
+                     int32_t shared_tokens);
 
 /* Early-exit parameters for all lanes ("CLI Reference", generate options):
  * probe at iteration l when l > min_L and (l - min_L - 1) % peek_every == 0;

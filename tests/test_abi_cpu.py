@@ -84,7 +84,7 @@ def test_workspace_grows_with_capacity_and_kv_formula():
 
 @pytest.mark.parametrize("field,value", [("d", 100), ("n_heads", 3), ("group", 48), ("kv_page_tokens", 48),
                                          ("kv_page_tokens", 16), ("max_lanes", 0), ("max_lanes", 2048),
-                                         ("L_max", 0), ("fmt_loop", 7), ("max_prefill_tokens", 1000)])
+                                         ("L_max", 0), ("fmt_loop", 7), ("max_prefill_tokens", -1)])
 def test_invalid_configs_rejected(field, value):
     cfg = T.config_from_shape(S.TINY, max_lanes=2, max_seq=64, L_max=4)
     setattr(cfg, field, value)
@@ -113,3 +113,10 @@ def test_blob_header_layout():
     assert len(h) == 56 and h[:8] == b"TLWBLOB1"
     assert Wt.gain_order(cfg) == S.gain_names(S.TINY)
     assert len(Wt.matrix_formats(cfg)) == len(S.matrix_shapes(S.TINY))
+
+
+def test_prompt_rows_may_exceed_one_sequence():
+    # a batched prefill computes the prompts of several lanes at once
+    cfg = T.config_from_shape(S.TINY, max_lanes=8, max_seq=64, L_max=4, max_prefill_tokens=512)
+    small = T.config_from_shape(S.TINY, max_lanes=8, max_seq=64, L_max=4)
+    assert T.workspace_bytes(cfg) > T.workspace_bytes(small)
