@@ -18,6 +18,7 @@
 #include "gemv_stream.cuh"
 #include "kernels.cuh"
 #include "tc_gemm.cuh"
+#include "tc_gemm_wide.cuh"
 
 namespace tl {
 
@@ -443,6 +444,25 @@ int tc_launch_nt(tl_ctx* c, int nt, const CUtensorMap& mw, const CUtensorMap& mw
   return tc_launch_t<256, NMAT, FMT, EPI>(c, mw, mw2, mx, p, grid);
 }
 
+// Persistent tensor-core projection for many rows (prompt batches).
+template <int NMAT, int FMT, int EPI>
+int tc_wide_launch(tl_ctx* c, int max_rows, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+                   const TcParams& p) {
+  using Cf = TcWideCfg<NMAT, FMT>;
+  auto kern = tc_gemm_wide_kernel<NMAT, FMT, EPI>;
+  static bool attr_done = false;  // once per instantiation
+  if (!attr_done) {
+    TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
+    attr_done = true;
+  }
+  const int64_t tiles = (int64_t)((p.N + 127) / 128) * ((max_rows + Cf::NT - 1) / Cf::NT);
+  const int grid = (int)(tiles < c->n_sms ? tiles : c->n_sms);
+  return launch_k(c, kern, dim3(grid), dim3(Cf::THREADS), Cf::SMEM, mw, mw2, mx, p);
+}
+
+// Rows from which prompt projections take the persistent kernel.
+constexpr int kWideRows = 512;
+
 // Tensor-core projection reading the fp16 copy `xsel` of the activations
 // (0: norm output, 1: attention output, 2: SwiGLU output).
 int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& W, const CUtensorMap& mw,
@@ -463,8 +483,20 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   p.o = o;
   p.out16 = out16;
   p.status = c->status;
-  const CUtensorMap& mx = c->xmap[xsel][nt == 64 ? 0 : (nt == 128 ? 1 : 2)];
   const CUtensorMap& m2 = mw2 ? *mw2 : mw;
+  if (max_rows >= kWideRows && o.epi != EPI_ARGMAX) {
+    p.kb_per_split = W.K / 64;
+    const CUtensorMap& mxw = c->xmap[xsel][nmat == 1 ? 2 : 1];  // 256-row tiles, 128 for the gate/up pair
+    if (W.fmt == TL_FMT_INT4) {
+      if (o.epi == EPI_SWIGLU) return tc_wide_launch<2, TL_FMT_INT4, EPI_SWIGLU>(c, max_rows, mw, m2, mxw, p);
+      if (o.epi == EPI_RESID) return tc_wide_launch<1, TL_FMT_INT4, EPI_RESID>(c, max_rows, mw, m2, mxw, p);
+      return tc_wide_launch<1, TL_FMT_INT4, EPI_STORE>(c, max_rows, mw, m2, mxw, p);
+    }
+    if (o.epi == EPI_SWIGLU) return tc_wide_launch<2, TL_FMT_BF16, EPI_SWIGLU>(c, max_rows, mw, m2, mxw, p);
+    if (o.epi == EPI_RESID) return tc_wide_launch<1, TL_FMT_BF16, EPI_RESID>(c, max_rows, mw, m2, mxw, p);
+    return tc_wide_launch<1, TL_FMT_BF16, EPI_STORE>(c, max_rows, mw, m2, mxw, p);
+  }
+  const CUtensorMap& mx = c->xmap[xsel][nt == 64 ? 0 : (nt == 128 ? 1 : 2)];
   if (W.fmt == TL_FMT_INT4) {
     if (o.epi == EPI_ARGMAX) return tc_launch_nt<1, TL_FMT_INT4, EPI_ARGMAX>(c, nt, mw, m2, mx, p, grid);
     if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, TL_FMT_INT4, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);

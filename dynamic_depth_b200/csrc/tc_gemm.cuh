@@ -1,4 +1,5 @@
 // W4A16 / BF16 projection on the 5th-generation tensor cores (tcgen05 + TMEM).
+// (The TMA and MMA warps run their loops with all lanes; one elected lane issues.)
 //
 // Y[rows, N] = X[rows, K] * W[N, K]^T computed as its transpose: the weight
 // tile is the 128-row M operand and the activation rows are the N operand
@@ -147,6 +148,32 @@ __device__ __forceinline__ void tc_emit(const TcParams& p, int row, int m, float
   }
 }
 
+// Final values of n consecutive activation rows (row0 .. row0+n-1) at output
+// m.  The residual form loads all n residual elements before storing any, so
+// the n read-modify-writes overlap instead of running one after another.
+template <int EPI, int NV>
+__device__ __forceinline__ void tc_emit_rows(const TcParams& p, int row0, int n, int m, const float (&v)[NV],
+                                             const float (&v2)[NV]) {
+  if constexpr (EPI == EPI_RESID) {
+    const ProjOut& o = p.o;
+    float* dst[NV];
+    float hv[NV];
+#pragma unroll
+    for (int e = 0; e < NV; ++e) {
+      const int hr = e < n ? (o.map ? o.map[row0 + e] : row0 + e) : 0;
+      dst[e] = o.h + (int64_t)hr * p.N + m;
+      hv[e] = e < n ? *dst[e] : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < NV; ++e)
+      if (e < n) *dst[e] = hv[e] + v[e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < NV; ++e)
+      if (e < n) tc_emit<EPI>(p, row0 + e, m, v[e], v2[e]);
+  }
+}
+
 template <int NT, int NMAT, int FMT, int EPI>
 __global__ void __launch_bounds__(256, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapW2,
@@ -225,41 +252,43 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     }
   } else if (warp == 0) {
     // ---------------------------------------------------------------- TMA
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES, r = i / STAGES;
-        const int kb = kb0 + i;
-        const uint32_t fb = smem_u32(&full[s]);
+    // the whole warp runs the loop (waits included); one elected lane issues
+    int issued = 0;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % STAGES, r = i / STAGES;
+      const int kb = kb0 + i;
+      const uint32_t fb = smem_u32(&full[s]);
+      if (i >= pre && r > 0 && !mbar_wait_warp(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) break;
+      if (elect_one()) {
         if (i < pre) {
           mbar_expect_tx(fb, C::B_BYTES);
         } else {
-          if (r > 0 && !mbar_wait(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) break;
           mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
           const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
           tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
           if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
         }
         tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
-        issued = i + 1;
       }
-      if (*abort_flag) {  // let copies already in flight land before the CTA leaves
-        for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
-          volatile int32_t never = 0;
-          mbar_wait(smem_u32(&full[i % STAGES]), (i / STAGES) & 1, &never);
-        }
+      __syncwarp();
+      issued = i + 1;
+    }
+    if (*abort_flag && lane == 0) {  // let copies already in flight land before the CTA leaves
+      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
+        volatile int32_t never = 0;
+        mbar_wait(smem_u32(&full[i % STAGES]), (i / STAGES) & 1, &never);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_f16<NT>();
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES, r = i / STAGES;
-        if (!mbar_wait(smem_u32(&afull[s]), r & 1, abort_flag)) break;
-        if (!mbar_wait(smem_u32(&full[s]), r & 1, abort_flag)) break;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
+    constexpr uint32_t idesc = umma_idesc_f16<NT>();
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % STAGES, r = i / STAGES;
+      if (!mbar_wait_warp(smem_u32(&afull[s]), r & 1, abort_flag)) break;
+      if (!mbar_wait_warp(smem_u32(&full[s]), r & 1, abort_flag)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bdesc = umma_desc(b_addr + kk * 32);
@@ -271,8 +300,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
         }
         umma_commit(smem_u32(&empty[s]));
       }
-      umma_commit(smem_u32(accfull));
+      __syncwarp();
     }
+    if (elect_one()) umma_commit(smem_u32(accfull));
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------- convert + epilogue
     const int t = threadIdx.x - 128;  // weight row within the tile == TMEM lane
@@ -291,7 +322,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     bool ok = true;
     for (int i = 0; i < nkb && ok; ++i) {
       const int s = i % STAGES, r = i / STAGES;
-      if (!mbar_wait(smem_u32(&full[s]), r & 1, abort_flag)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), r & 1, abort_flag))) { ok = false; break; }
 #pragma unroll
       for (int mat = 0; mat < NMAT; ++mat) {
         uint8_t* arow = sA + (s * NMAT + mat) * C::A_BYTES + t * 128;
@@ -301,11 +332,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
           const uint4 w1 = *reinterpret_cast<const uint4*>(raw + t * 32 + 16);
           const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
           const int kbase = (kb0 + i) * 64;
+          const __half* srow = sSc + (mat * 128 + t) * TC_SC_MAX;
+          if (p.group % 64 == 0) {  // the k-block lies inside one scale group
+            const __half sc = srow[kbase / p.group - gfirst];
+            const __half2 s2 = __halves2half2(sc, sc);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const __half sc = sSc[(mat * 128 + t) * TC_SC_MAX + (kbase + 8 * c) / p.group - gfirst];
-            const uint4 h = int4_word_to_half8(w[c], __halves2half2(sc, sc));
-            *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = h;
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = int4_word_to_half8(w[c], s2);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const __half sc = srow[(kbase + 8 * c) / p.group - gfirst];
+              *reinterpret_cast<uint4*>(arow + ((c ^ (t & 7)) << 4)) = int4_word_to_half8(w[c], __halves2half2(sc, sc));
+            }
           }
         } else {
 #pragma unroll
@@ -319,7 +358,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
     }
-    if (ok && mbar_wait(smem_u32(accfull), 0, abort_flag)) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(accfull), 0, abort_flag))) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int m = m0 + t;
       const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
@@ -361,11 +400,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
         tmem_ld8(tl + j, v);
         if constexpr (NMAT == 2) tmem_ld8(tl + NT + j, v2);
         if (S == 1) {
-          if (m < p.N) {
+          if constexpr (NMAT == 1) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (j + e < ncols) tc_emit<EPI>(p, n0 + j + e, m, v[e], NMAT == 2 ? v2[e] : 0.f);
+            for (int e = 0; e < 8; ++e) v2[e] = 0.f;
           }
+          if (m < p.N) tc_emit_rows<EPI, 8>(p, n0 + j, min(8, ncols - j), m, v, v2);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {

@@ -89,3 +89,25 @@ def test_prompt_batch_rejects_bad_arguments():
         m.prefill_batch([0, 1], P[:2], [2, 5])
     m.prefill_batch([0, 1], P[:2], [2, 3])
     status_clean(m)
+
+
+# ------------------------------------------- >= 512 prompt rows: persistent GEMM
+
+@pytest.mark.parametrize("name,gains,n,T,Ls,max_seq", [
+    ("tiny", 7, 8, 70, [3, 8, 1, 5, 8, 2, 6, 4], 80),
+    ("m407", None, 4, 160, [2, 4, 3, 1], 168),
+    ("m1b4_mini", 5, 6, 100, [1, 2, 3, 4, 4, 2], 108),
+])
+def test_wide_prompt_batch_persistent_gemm(name, gains, n, T, Ls, max_seq):
+    # 512+ prompt rows in one pass: every projection of the prompt runs on the
+    # persistent tensor-core kernel (INT4 and BF16, single matrix and gate/up pair)
+    sh = S.SHAPES[name]
+    W = oracle_weights(name, gains)
+    P = list(S.prompts(n, T, sh.vocab, seed=94))
+    m = gpu_model(name, gains, max_lanes=n, max_seq=max_seq, L_max=8, max_prefill_tokens=n * T)
+    ref, lg, am, dep = teacher_forced(m, W, P, Ls, 2, prefill=_batch_once(m, list(range(n)), P, Ls))
+    status_clean(m)
+    for i in range(n):
+        assert dep[i].tolist() == ref[i].depths.tolist()
+        for t in range(2):
+            assert_logits_close(lg[i, t], ref[i].logits[t], f"{name} lane {i} token {t}")
