@@ -243,18 +243,26 @@ __global__ void plan_tick_kernel(const LaneState* __restrict__ lanes, int n_lane
 // tensor-core projections when out16 is given).  One CTA per row.  When h_in is
 // given, also copies the source row there (indexed like h); when zero_rows is
 // given, clears row r of that [rows][zero_cols] accumulator, which the next
-// (split-K) projection adds into.  Does nothing when the row count is at most
-// min_rows (those counts are served by a GEMV that normalises by itself).
-__global__ void rmsnorm_rows_kernel(const float* __restrict__ h, const int32_t* __restrict__ map,
+// (split-K) projection adds into.  Does nothing more when the row count is
+// at most min_rows (those counts are served by a GEMV that normalises by
+// itself).  add (prompt batches): first h[row r] += add[r] for every r <
+// *n_add, the residual of a projection that stored its output instead of
+// adding it (the grid covers those rows too).
+__global__ void rmsnorm_rows_kernel(float* __restrict__ h, const int32_t* __restrict__ map,
                                     const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
                                     float eps, float* __restrict__ out, float* __restrict__ h_in,
                                     __half* __restrict__ out16, float* __restrict__ zero_rows, int zero_cols,
-                                    int min_rows) {
+                                    int min_rows, const float* __restrict__ add, const int32_t* __restrict__ n_add) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float red[32];
   const int r = blockIdx.x;
   const int n = n_rows[0];
+  if (add && r < n_add[0]) {  // deferred residual of the previous projection: h[row r] += add[r]
+    float* hx = h + (int64_t)(map ? map[r] : r) * d;
+    for (int k = threadIdx.x; k < d; k += blockDim.x) hx[k] += add[(int64_t)r * d + k];
+    __syncthreads();
+  }
   if (r >= n || n <= min_rows) return;
   const int src = map ? map[r] : r;
   const float* x = h + (int64_t)src * d;

@@ -604,18 +604,27 @@ bool gemv_norms_itself(tl_ctx* c, const MatView& W, int nmat) {
 // kernel (fp32 act_a + fp16 act_a16, and the h_in copy) only where a
 // projection that needs it can run: the tensor-core variant (more than 8 rows)
 // or a GEMV that does not normalise itself.
+// A prompt projection's residual left for the next norm kernel to add: h[row
+// r] += add[r] for r < *n (at most `rows` rows).
+struct PendingAdd {
+  const float* add = nullptr;
+  const int32_t* n = nullptr;
+  int rows = 0;
+};
+
 int norm_for_proj(tl_ctx* c, int max_rows, int path, const int32_t* n, float* hbuf, const int32_t* map,
                   const float* g, float* h_in, const MatView& W, int nmat, const float** X, GsNorm* nrm,
-                  bool* use_nrm) {
-  const bool fused = path != PATH_TC && gemv_norms_itself(c, W, nmat);
+                  bool* use_nrm, const PendingAdd& pend = PendingAdd{}) {
+  const bool fused = path != PATH_TC && gemv_norms_itself(c, W, nmat) && !pend.add;
   const bool tc_possible = path != PATH_GEMV && max_rows > kGemvMaxRows;
   *use_nrm = fused;
   *nrm = GsNorm{g, map, c->cfg.rms_eps, h_in};
   *X = fused ? hbuf : c->act_a;
   if (!fused || tc_possible) {
     const int min_rows = (fused && path == PATH_AUTO) ? kGemvMaxRows : 0;  // <= 8 rows: the GEMV normalises
-    TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(max_rows), dim3(256), 0, hbuf, map, n, c->cfg.d, g, c->cfg.rms_eps,
-                    c->act_a, h_in, c->act_a16, nullptr, 0, min_rows));
+    const int grid = pend.rows > max_rows ? pend.rows : max_rows;
+    TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(grid), dim3(256), 0, hbuf, map, n, c->cfg.d, g, c->cfg.rms_eps,
+                    c->act_a, h_in, c->act_a16, nullptr, 0, min_rows, pend.add, pend.n));
   }
   return TL_OK;
 }
@@ -624,15 +633,23 @@ int norm_for_proj(tl_ctx* c, int max_rows, int path, const int32_t* n, float* hb
 // (indexed through map, or by row when map is null).
 // prompt = rows are runs of consecutive positions of one lane each, attended
 // causally in the n_tiles tiles of `tiles`.
+// Prompt batches (pend != null): the residual projections of blocks wide
+// enough for the persistent kernel store their output (in act_q, free after
+// attention) instead of adding it into hbuf, and the next norm kernel adds it
+// (the norm after the attention, then the next block's first norm, or the
+// caller after the last block, from *pend).
 int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int32_t* map, const BlockW& w,
               int slot_base, int slot_stride, float* h_in, bool prompt = false, int path = PATH_AUTO,
-              const int2* tiles = nullptr, int n_tiles = 0) {
+              const int2* tiles = nullptr, int n_tiles = 0, PendingAdd* pend = nullptr) {
   if (prompt) path = max_rows > kGemvMaxRows ? PATH_TC : PATH_GEMV;
   const int d = c->cfg.d, F = c->cfg.ffn;
+  const bool defer = pend && prompt && max_rows >= kWideRows;
   const float* X = nullptr;
   GsNorm nrm{};
   bool use_nrm = false;
-  TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g1, h_in, w.wqkv, 1, &X, &nrm, &use_nrm));
+  TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g1, h_in, w.wqkv, 1, &X, &nrm, &use_nrm,
+                       pend ? *pend : PendingAdd{}));
+  if (pend) *pend = PendingAdd{};
   ProjOut o{};
   o.epi = EPI_STORE;
   o.out = c->act_qkv;
@@ -650,15 +667,23 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   r.epi = EPI_RESID;
   r.h = hbuf;
   r.map = map;
+  if (defer) {  // stored, added by the next norm
+    r.epi = EPI_STORE;
+    r.out = c->act_q;
+    r.ldo = d;
+  }
   TL_TRY(proj(c, max_rows, path, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
-  TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g2, nullptr, w.wg, 2, &X, &nrm, &use_nrm));
+  TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g2, nullptr, w.wg, 2, &X, &nrm, &use_nrm,
+                       defer ? PendingAdd{c->act_q, rows.n, max_rows} : PendingAdd{}));
   ProjOut sw{};
   sw.epi = EPI_SWIGLU;
   sw.out = c->act_u;
   sw.ldo = F;
   TL_TRY(proj(c, max_rows, path, X, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16, TL_PROF_PROJ,
               use_nrm ? &nrm : nullptr));
-  return proj(c, max_rows, path, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr);
+  TL_TRY(proj(c, max_rows, path, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr));
+  if (defer) *pend = PendingAdd{c->act_q, rows.n, max_rows};
+  return TL_OK;
 }
 
 // Row table `which` from lanes 0..n_consider-1 (all lanes when n_consider <= 0);
@@ -1159,7 +1184,7 @@ static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t sh
   }
   r_iter.assign(total, 0);
   const int Lmax = in[order[0]].L;
-  std::vector<int32_t> stage_rows(Lmax), stage_tiles(Lmax);
+  std::vector<int32_t> stage_rows(Lmax + 1, 0), stage_tiles(Lmax);  // stage_rows[Lmax] = 0
   for (int l = 0; l < Lmax; ++l) {
     int k = 0;
     while (k < n && in[order[k]].L > l) ++k;  // lanes 0..k-1 of the order run iteration l
@@ -1173,21 +1198,26 @@ static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t sh
   TL_CUDA(cudaMemcpyAsync(c->tok_stage, tok.data(), total * 4, cudaMemcpyHostToDevice, c->stream));
   TL_CUDA(cudaMemcpyAsync(c->pf_tiles, tiles.data(), tiles.size() * sizeof(int2), cudaMemcpyHostToDevice, c->stream));
   TL_CUDA(cudaMemcpyAsync(c->pf_info, info.data(), info.size() * 4, cudaMemcpyHostToDevice, c->stream));
-  TL_CUDA(cudaMemcpyAsync(c->pf_n, stage_rows.data(), Lmax * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->pf_n, stage_rows.data(), (Lmax + 1) * 4, cudaMemcpyHostToDevice, c->stream));
   Rows Rs = R;
   Rs.n = c->pf_n;  // stage 0: every row (every lane has L >= 1)
   const int all = (int)total;
   TL_TRY(launch_k(c, embed_rows_kernel, dim3(all), dim3(256), 0, c->embed, c->tok_stage, all, cfg.d, c->hrows,
                   c->status));
+  PendingAdd pend;
   for (int b = 0; b < P; ++b)
     TL_TRY(run_block(c, Rs, all, c->hrows, nullptr, c->pre[b], b, 0, nullptr, true, PATH_AUTO, c->pf_tiles,
-                     stage_tiles[0]));
+                     stage_tiles[0], &pend));
   for (int l = 0; l < Lmax; ++l) {
     Rs.n = c->pf_n + l;
     for (int m = 0; m < Lb; ++m)
       TL_TRY(run_block(c, Rs, stage_rows[l], c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr, true,
-                       PATH_AUTO, c->pf_tiles, stage_tiles[l]));
+                       PATH_AUTO, c->pf_tiles, stage_tiles[l], &pend));
   }
+  if (pend.add)  // the last block's residual (the norm kernel with no rows to normalise only adds)
+    TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(pend.rows), dim3(256), 0, c->hrows, (const int32_t*)nullptr,
+                    (const int32_t*)(c->pf_n + Lmax), cfg.d, (const float*)nullptr, cfg.rms_eps, (float*)nullptr,
+                    (float*)nullptr, (__half*)nullptr, (float*)nullptr, 0, 0, pend.add, pend.n));
   TL_TRY(launch_k(c, prefill_finish_batch_kernel, dim3(n), dim3(256), 0, c->lanes, c->pf_info, n, c->hrows, c->h,
                   cfg.d));
   if (dev_hidden_out)

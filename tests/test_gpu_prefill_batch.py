@@ -95,12 +95,15 @@ def test_prompt_batch_rejects_bad_arguments():
 
 @pytest.mark.parametrize("name,gains,n,T,Ls,max_seq", [
     ("tiny", 7, 8, 70, [3, 8, 1, 5, 8, 2, 6, 4], 80),
+    ("tiny", None, 8, 70, [2] * 8, 80),  # every stage wide: the last block's residual is added after it
     ("m407", None, 4, 160, [2, 4, 3, 1], 168),
     ("m1b4_mini", 5, 6, 100, [1, 2, 3, 4, 4, 2], 108),
 ])
 def test_wide_prompt_batch_persistent_gemm(name, gains, n, T, Ls, max_seq):
     # 512+ prompt rows in one pass: every projection of the prompt runs on the
-    # persistent tensor-core kernel (INT4 and BF16, single matrix and gate/up pair)
+    # persistent tensor-core kernel (INT4 and BF16, single matrix and gate/up pair),
+    # and the residual projections leave their sums to the next norm kernel,
+    # including across a stage that drops below 512 rows
     sh = S.SHAPES[name]
     W = oracle_weights(name, gains)
     P = list(S.prompts(n, T, sh.vocab, seed=94))
