@@ -342,7 +342,7 @@ def run_ours(args, rank, world, local_rank):
             "tokens_per_s": round(wl.n_lanes * wl.prompt_len / prefill_s, 1),
             "rows_through_blocks": pf_rows,
             "projection_ms": round(pf_ms[2], 3), "attention_ms": round(pf_ms[1], 3),
-            "gemm_roofline": {"kernel": "tc_gemm_kernel (tcgen05 W4A16 projections over all prompt rows)",
+            "gemm_roofline": {"kernel": "tc_gemm_wide_kernel (persistent tcgen05 W4A16 projections over all prompt rows)",
                               "bound": "tensor", "achieved": round(pf_ach, 1), "peak": pf_peak, "unit": "TFLOP/s",
                               "frac": round(pf_ach / pf_peak, 4), "flops": pf_flops,
                               "peak_source": "of measured bf16 burst (fp16 operands have the same dense rate)"}},
