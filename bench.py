@@ -13,10 +13,11 @@ before timing; every step restores the post-prompt lane state and decodes all
 ~1.7 GB (plus 79 MB of weights) against a 126 MB L2, so no flush is needed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload cdb64|prefill128|lsweep|prefix256]
+                    [--workload cdb64|tiny|prefill128|lsweep|prefix256]
 
 --workload selects one of the other measured configurations instead (each
-prints its own JSON line): prefill128 = 407M-class scoring forward, one
+prints its own JSON line): tiny = the tiny looped LM's 2-lane job, timed beside
+the oracle; prefill128 = 407M-class scoring forward, one
 128-token sequence at L=8 with the hidden states out; lsweep = one lane, a
 32-token prompt and 32 greedy tokens at L in {2, 4, 8, 16, 32}, with the INT4
 and then the BF16 loop block; prefix256 = the 1.4B-class BF16 model, 256 lanes
@@ -247,13 +248,9 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     st1 = m.stats()
     assert st1["device_status"] == 0, f"device status {st1['device_status']:#x}"
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = _max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     tokens_per_step = wl.n_lanes * wl.n_new
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = whole_job_rate(tokens_per_step * args.steps, ms, world)
     # the same steps again with per-kind event timing (kept out of the headline timing)
     m.profile_begin(args.profile_mask)
     ev0.record(stream)
@@ -318,12 +315,8 @@ def run_ours(args, rank, world, local_rank):
         t0 = time.perf_counter()
         for _ in range(reps):
             m.generate(hp.numpy(), Ls, wl.n_new, ht, hd)
-        e2e_s = (time.perf_counter() - t0) / reps
-        if world > 1:
-            t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_s = float(t.item())
-        e2e = {"value": round(world * tokens_per_step / e2e_s, 1), "unit": UNIT,
+        e2e_s = _max_over_ranks((time.perf_counter() - t0) / reps, world, dev)
+        e2e = {"value": round(whole_job_rate(tokens_per_step, e2e_s * 1e3, world), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(P.nbytes + Ls.nbytes),
                "d2h_bytes_per_step": int(2 * wl.n_lanes * wl.n_new * 4),
                "includes": "prompt upload, 64 x 512-token prefill, decode, token download (tl_generate)"}
@@ -412,12 +405,21 @@ def _timed_reps(fn, warmup, steps, flush=None):
 
 
 def _max_over_ranks(x: float, world: int, dev) -> float:
+    """The largest x over the ranks (every rank calls it, in the same order)."""
     if world <= 1:
         return x
     import torch
+    if torch.distributed.get_backend() == "gloo":
+        dev = "cpu"
     t = torch.tensor([x], device=dev, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, max_ms: float, world: int) -> float:
+    """Units per second of the whole job: every rank processed units_per_rank
+    (weak scaling, one replica per rank) within the slowest rank's max_ms."""
+    return world * units_per_rank / (max_ms / 1e3)
 
 
 def _l2_copy_gbs(dev) -> float:
@@ -445,6 +447,64 @@ def _common(metric, value, unit, world, args, ms, config, dtype, hib=True):
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": hib, "scaling": "weak",
             "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded random weights and token ids)",
             "config": config}
+
+
+def run_tiny(args, rank, world, local_rank):
+    """The tiny looped LM: 2 lanes, 16-token prompts, 8 greedy tokens at L = {2, 4}; the decode timed on
+    the GPU and the whole job (prompts + decode) timed for the oracle beside it, with a parity check."""
+    import torch
+    dev = f"cuda:{local_rank}"
+    torch.cuda.set_device(dev)
+    wl = S.workload("tiny")
+    sh = wl.shape
+    m = _build_model(sh, dev, max_lanes=wl.n_lanes, max_seq=wl.prompt_len + wl.n_new, L_max=8,
+                     max_prefill_tokens=wl.n_lanes * wl.prompt_len)
+    P = S.prompts(wl.n_lanes, wl.prompt_len, sh.vocab)
+    Ls = np.array(wl.per_lane_L, dtype=np.int32)
+    m.prefill_batch(list(range(wl.n_lanes)), list(P), Ls)
+    snap = m.lane_state_save()
+    tok = torch.zeros((wl.n_lanes, wl.n_new), dtype=torch.int32, device=dev)
+    dep = torch.zeros_like(tok)
+
+    def step():
+        m.lane_state_load(snap)
+        m.decode(Ls, wl.n_new, tok, dep)
+    with ClockSampler(gpu_id(dev)) as clk:
+        reps = _timed_reps(step, args.warmup, args.steps)
+    assert m.stats()["device_status"] == 0
+    ms = _max_over_ranks(statistics.median(reps), world, dev)
+    n_tok = wl.n_lanes * wl.n_new
+    e2e_reps = []
+    for _ in range(max(3, args.steps)):
+        t0 = time.perf_counter()
+        ht, hd = m.generate(P, Ls, wl.n_new)
+        e2e_reps.append(time.perf_counter() - t0)
+    e2e_s = _max_over_ranks(statistics.median(e2e_reps), world, dev)
+    out = _common("decode tokens/s (tiny looped LM, per-lane L)", round(whole_job_rate(n_tok, ms, world), 1),
+                  "tokens/s", world, args, ms,
+                  {"workload": "tiny looped LM: 2 lanes x (16-token prompt + 8 greedy tokens), L = {2, 4}",
+                   "model": "vocab 512, d 128, 4x32 heads, SwiGLU 512, 1 pre + 1 loop block, INT4 g32",
+                   "weights": "random N(0,0.02) seed 0", "l2": "everything L2-resident (small case)",
+                   "parallelism": f"replicas x{world}"},
+                  "fp32 activations and accumulate; INT4 weights; fp16 KV")
+    out.update({"clocks": clk.summary(), "roofline": None,
+                "roofline_note": "launch-latency bound at this size; see the 64-lane workload",
+                "e2e": {"value": round(whole_job_rate(n_tok, e2e_s * 1e3, world), 1), "unit": "tokens/s",
+                        "h2d_bytes_per_step": int(P.nbytes + Ls.nbytes), "d2h_bytes_per_step": int(2 * n_tok * 4)}})
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle as O
+        from oracle import decode as D
+        from oracle import model as Mo
+        W = O.build_weights(sh, S.master_weights(sh), S.gains(sh))
+        t0 = time.perf_counter()
+        ref = [D.generate_lane(W, P[i], int(Ls[i]), wl.n_new) for i in range(wl.n_lanes)]
+        dt = time.perf_counter() - t0
+        agree = all(int(ht[i, t]) == int(ref[i].tokens[t]) for i in range(wl.n_lanes) for t in range(wl.n_new)
+                    if all(Mo.top2_margin(ref[i].logits[u]) > 1e-3 for u in range(t + 1)))
+        out["cpu_baseline"] = {"value": round(n_tok / dt, 2), "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+                               "kind": "oracle", "sample": f"the whole job (2 prompts + 16 tokens) in {dt:.2f} s"}
+        out["tokens_match_oracle"] = bool(agree)
+    return out
 
 
 def run_prefill128(args, rank, world, local_rank):
@@ -628,14 +688,15 @@ def run_prefix256(args, rank, world, local_rank):
     pool = 2 * slots * pps + int(sum((sh.n_pre + int(L) * sh.n_loop_layers) * own_pages for L in Ls))
     donor = n  # an extra lane holds the prefix at the deepest L
     m = _build_model(sh, dev, max_lanes=n + 1, max_seq=max_seq, L_max=Lmax, kv_page_tokens=page,
-                     kv_pool_pages=pool, max_prefill_tokens=Tp + Ts)
+                     kv_pool_pages=pool, max_prefill_tokens=max(Tp + Ts, n * Ts))
+    prompts = [np.concatenate([pre, suf[i]]) for i in range(n)]
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     m.prefill(donor, pre, Lmax)
     torch.cuda.synchronize()
     t1 = time.perf_counter()
-    for i in range(n):
-        m.prefill(i, np.concatenate([pre, suf[i]]), int(Ls[i]), share_from=donor, shared_tokens=Tp)
+    # every lane's suffix in one batched pass, its prefix pages mapped from the donor
+    m.prefill_batch(list(range(n)), prompts, Ls, share_from=donor, shared_tokens=Tp)
     torch.cuda.synchronize()
     t2 = time.perf_counter()
     snap = m.lane_state_save()
@@ -701,7 +762,7 @@ def run_prefix256(args, rank, world, local_rank):
                   "fp32 activations and accumulate; BF16 weights; fp16 KV")
     out.update({
         "prefix_prefill_ms": round((t1 - t0) * 1e3, 2),
-        "suffix_prefill_ms_per_lane": round((t2 - t1) * 1e3 / n, 3),
+        "suffix_prefill_ms_all_lanes": round((t2 - t1) * 1e3, 2),
         "gpu_launches": int(st1["kernel_launches"] - st0["kernel_launches"]) // max(1, args.steps + args.warmup),
         "kernel_ms_per_step": {"attention": round(kind_ms[1], 3), "projections": round(kind_ms[2], 3),
                                "head": round(kind_ms[3], 3)},
@@ -788,7 +849,7 @@ def main():
     ap.add_argument("--lanes", type=int, default=0, help="reduced case: lanes (profiling captures only)")
     ap.add_argument("--prompt-len", type=int, default=0, help="reduced case: prompt tokens")
     ap.add_argument("--new-tokens", type=int, default=0, help="reduced case: generated tokens")
-    ap.add_argument("--workload", choices=["cdb64", "prefill128", "lsweep", "prefix256"], default="cdb64")
+    ap.add_argument("--workload", choices=["cdb64", "tiny", "prefill128", "lsweep", "prefix256"], default="cdb64")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -806,7 +867,8 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     if args.workload != "cdb64":
-        fn = {"prefill128": run_prefill128, "lsweep": run_lsweep, "prefix256": run_prefix256}[args.workload]
+        fn = {"tiny": run_tiny, "prefill128": run_prefill128, "lsweep": run_lsweep,
+              "prefix256": run_prefix256}[args.workload]
         out = fn(args, rank, world, local_rank)
         if world > 1:
             import torch

@@ -580,6 +580,11 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
 // value sum (all 32 value loads of a block issued together); running max and
 // sum are merged across warps, and across splits by the last CTA of the
 // (row, head) to finish, in split order.  Requires kv_page_tokens >= 32.
+// Working CTAs the context split aims for: four per SM on 148 SMs (a
+// larger target, 12 per SM, split the 64-row case in two and measured
+// slower: the split partials and their combine cost more than the waves save).
+constexpr int kAttnCtaTarget = 4 * 148;
+
 template <int HD>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
@@ -602,7 +607,7 @@ attn_decode_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half*
   const int slot = slot_base + rows.iter[r] * slot_stride;
   const int ctx = pos + 1;
   const int nblk = (ctx + 31) / 32;
-  int S = (4 * 148 + n * g.H - 1) / (n * g.H);
+  int S = (kAttnCtaTarget + n * g.H - 1) / (n * g.H);
   S = min(min(S, (int)gridDim.z), nblk);
   if (z >= S) return;
   const int b0 = (z * nblk) / S, b1 = ((z + 1) * nblk) / S;

@@ -554,7 +554,7 @@ int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int3
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
   TL_TRY(prof_start(c, TL_PROF_ATTN));
   // splits beyond what max_rows * heads needs to fill the GPU are never used
-  int ks = (4 * 148 + max_rows * c->cfg.n_heads - 1) / (max_rows * c->cfg.n_heads);
+  int ks = (kAttnCtaTarget + max_rows * c->cfg.n_heads - 1) / (max_rows * c->cfg.n_heads);
   ks = ks < 1 ? 1 : (ks > kAttnSplits ? kAttnSplits : ks);
   if (max_rows > 1) ks = kAttnSplits < 4 ? kAttnSplits : (ks < 4 ? 4 : ks);
   dim3 grid(max_rows, c->cfg.n_heads, ks);
