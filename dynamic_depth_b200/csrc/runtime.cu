@@ -362,15 +362,27 @@ int prof_stop(tl_ctx* c, int kind) {
   return TL_OK;
 }
 
+// Kernel attributes (shared-memory opt-in) are per device: each launch helper
+// keeps one bit per device ordinal (< 64) for "already set on this device".
+static int current_device() {
+  int dev = 0;
+  return (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) ? dev : 0;
+}
+static bool attr_needed(uint64_t* done_mask) {
+  const uint64_t bit = 1ull << current_device();
+  if (*done_mask & bit) return false;
+  *done_mask |= bit;
+  return true;
+}
+
 template <int FMT, int EPI, int RPW = 1>
 int gemv_launch(tl_ctx* c, const float* X, const int32_t* n_rows, const MatView& W, const MatView& W2,
                 const ProjOut& o, int skip_above) {
   const size_t smem = (size_t)8 * W.K * 4;
   auto kern = gemv_kernel<FMT, EPI, RPW>;
-  static bool attr_done = false;  // once per instantiation
-  if (!attr_done) {
+  static uint64_t attr_done = 0;  // per instantiation: one bit per device
+  if (attr_needed(&attr_done)) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-    attr_done = true;
   }
   if (smem > 200 * 1024) return TL_EINVAL;
   const unsigned grid = (unsigned)((W.N + GEMV_WARPS * RPW - 1) / (GEMV_WARPS * RPW));
@@ -382,10 +394,11 @@ template <int FMT, int EPI>
 int gemv_stream_launch(tl_ctx* c, const GsChoice& g, const float* X, const int32_t* n_rows, const MatView& W,
                        const MatView& W2, const ProjOut& o, int skip_above, const GsNorm& nrm) {
   auto kern = gemv_stream_kernel<FMT, EPI>;
-  static int attr_smem = 0;  // per instantiation: largest opt-in requested so far
-  if (g.smem > attr_smem) {
+  static int attr_smem[64] = {0};  // per instantiation and device: largest opt-in requested so far
+  const int dev = current_device();
+  if (g.smem > attr_smem[dev]) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem));
-    attr_smem = g.smem;
+    attr_smem[dev] = g.smem;
   }
   TL_TRY(launch_k(c, kern, dim3(g.grid), dim3(GS_THREADS), g.smem, X, n_rows, W, W2, o, skip_above, g.pl, nrm,
                   c->status));
@@ -413,10 +426,9 @@ int tc_launch_t(tl_ctx* c, const CUtensorMap& mw, const CUtensorMap& mw2, const 
                 const TcParams& p, dim3 grid) {
   using Cf = TcCfg<NT, NMAT, FMT>;
   auto kern = tc_gemm_kernel<NT, NMAT, FMT, EPI>;
-  static bool attr_done = false;  // once per instantiation
-  if (!attr_done) {
+  static uint64_t attr_done = 0;  // per instantiation: one bit per device
+  if (attr_needed(&attr_done)) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
-    attr_done = true;
   }
   cudaLaunchConfig_t lc{};
   lc.gridDim = grid;
@@ -450,10 +462,9 @@ int tc_wide_launch(tl_ctx* c, int max_rows, const CUtensorMap& mw, const CUtenso
                    const TcParams& p) {
   using Cf = TcWideCfg<NMAT, FMT>;
   auto kern = tc_gemm_wide_kernel<NMAT, FMT, EPI>;
-  static bool attr_done = false;  // once per instantiation
-  if (!attr_done) {
+  static uint64_t attr_done = 0;  // per instantiation: one bit per device
+  if (attr_needed(&attr_done)) {
     TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
-    attr_done = true;
   }
   const int64_t tiles = (int64_t)((p.N + 127) / 128) * ((max_rows + Cf::NT - 1) / Cf::NT);
   const int grid = (int)(tiles < c->n_sms ? tiles : c->n_sms);
@@ -570,10 +581,9 @@ int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int sl
 template <int HD>
 int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot, const int2* tiles, int n_tiles) {
   const size_t smem = (size_t)(3 * HD * 64 + 64 * 65) * 4;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static uint64_t attr_done = 0;  // per instantiation: one bit per device
+  if (attr_needed(&attr_done)) {
     TL_CUDA(cudaFuncSetAttribute(attn_prefill_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr_done = true;
   }
   dim3 grid(tiles ? n_tiles : (max_rows + 63) / 64, c->cfg.n_heads);
   TL_TRY(launch_k(c, attn_prefill_kernel<HD>, dim3(grid), dim3(256), smem, c->act_q, c->act_o, c->act_o16, rows,
