@@ -259,7 +259,8 @@ int tl_decode(tl_ctx* ctx, const int32_t* host_per_lane_L, int32_t n_lanes, int3
 
 /* End to end from host memory ("Dynamic-L Inference", "L-Aware Batching":
  * generate_batch(prompts, per_lane_loops)): copy prompts to the device,
- * prefill every lane at its L, decode n_new tokens per lane, copy tokens and
+ * prefill every lane at its L (as tl_prefill_batch, as many lanes per pass as
+ * max_prefill_tokens allows), decode n_new tokens per lane, copy tokens and
  * depths back.  host_prompts: int32 [n_lanes, T]; outputs int32 [n_lanes,
  * n_new] in host memory (pinned memory makes the copies asynchronous-capable).
  * Returns after the results are in host memory. */
