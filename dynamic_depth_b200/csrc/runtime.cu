@@ -39,7 +39,8 @@ static bool cfg_valid(const tl_config* c) {
   if (c->d % c->n_heads) return false;
   const int hd = c->d / c->n_heads;
   if (hd != 32 && hd != 64 && hd != 128) return false;
-  if (c->d % 32 || c->ffn % 32) return false;
+  // the tensor-core projections step through K in 64-wide blocks (K is d or ffn)
+  if (c->d % 64 || c->ffn % 64) return false;
   const int fmts[3] = {c->fmt_pre, c->fmt_loop, c->fmt_embed_head};
   bool any_int4 = false;
   for (int f : fmts) {

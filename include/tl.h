@@ -65,7 +65,9 @@ typedef enum tl_weight_fmt {
     TL_FMT_BF16 = 1    /* bfloat16 bit patterns */
 } tl_weight_fmt;
 
-/* Model and capacity.  d = n_heads * head_dim, head_dim even. */
+/* Model and capacity.  d = n_heads * head_dim with head_dim 32, 64 or 128;
+ * d and ffn multiples of 64 (the tensor-core projections take K in 64-wide
+ * blocks); for INT4, group a multiple of 32 dividing d and ffn. */
 typedef struct tl_config {
     int32_t vocab;
     int32_t d;
