@@ -48,6 +48,8 @@ static bool cfg_valid(const tl_config* c) {
     any_int4 |= f == TL_FMT_INT4;
   }
   if (any_int4 && (c->group <= 0 || c->group % 32 || c->d % c->group || c->ffn % c->group)) return false;
+  // the decode tensor-core kernel stages a row's scale groups for its K range in shared memory
+  if (any_int4 && (c->d / c->group > TC_SC_MAX - 1 || c->ffn / c->group > TC_SC_MAX - 1)) return false;
   if (!(c->rms_eps >= 0.f) || !(c->rope_base > 0.f)) return false;
   if (c->max_lanes < 1 || c->max_lanes > 1024 || c->max_seq < 1 || c->L_max < 1) return false;
   if (c->kv_page_tokens < 32 || (c->kv_page_tokens & (c->kv_page_tokens - 1))) return false;
@@ -109,7 +111,8 @@ static bool tc_split_ok(int nt) {
 
 // Split of the K loop (the cluster size, <= 8) so that the grid fills the 148
 // SMs (two CTAs per SM fit for the 64-row single-matrix tile).  Every split
-// keeps >= 2 k-blocks and its INT4 scale groups within TC_SC_MAX.
+// keeps >= 2 k-blocks; its INT4 scale groups stay within TC_SC_MAX because the
+// configuration allows at most TC_SC_MAX - 1 groups over the whole K.
 static int tc_splits(int N, int K, int max_rows, int nmat, int fmt, int group) {
   const int nt = tc_nt(max_rows);
   const bool ok = nmat == 1 ? (fmt == TL_FMT_INT4 ? tc_split_ok<1, TL_FMT_INT4>(nt) : tc_split_ok<1, TL_FMT_BF16>(nt))

@@ -67,7 +67,8 @@ typedef enum tl_weight_fmt {
 
 /* Model and capacity.  d = n_heads * head_dim with head_dim 32, 64 or 128;
  * d and ffn multiples of 64 (the tensor-core projections take K in 64-wide
- * blocks); for INT4, group a multiple of 32 dividing d and ffn. */
+ * blocks); for INT4, group a multiple of 32 dividing d and ffn, with at
+ * most 32 groups across d and across ffn. */
 typedef struct tl_config {
     int32_t vocab;
     int32_t d;

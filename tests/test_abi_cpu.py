@@ -84,6 +84,7 @@ def test_workspace_grows_with_capacity_and_kv_formula():
 
 @pytest.mark.parametrize("field,value", [("d", 100), ("n_heads", 3), ("group", 48), ("kv_page_tokens", 48),
                                          ("ffn", 544),  # a multiple of 32 but not of 64
+                                         ("ffn", 2048),  # 64 scale groups of 32 across ffn
                                          ("kv_page_tokens", 16), ("max_lanes", 0), ("max_lanes", 2048),
                                          ("L_max", 0), ("fmt_loop", 7), ("max_prefill_tokens", -1)])
 def test_invalid_configs_rejected(field, value):
