@@ -11,6 +11,10 @@ Passages followed:
     peek_every iterations past min_L; L never rises again within a generation
     once reduced (monotonic clamp keeps the cache consistent).  Early exit is a
     cached-decode feature, so the prompt always runs the full requested L.
+  * "CLI Reference", generate option --early-exit-logit-margin: when positive,
+    the probe's stability metric becomes the top-1 minus top-2 margin of the
+    head's logits at that iteration instead of the hidden-state change (a head
+    projection per probe); the lane stops when the model is confident.
   * "CLI Reference", "Current Behavior": max_seq = prompt tokens + max tokens.
   * "Depth-adaptive Inference of Looped Language Models via Continuous Depth
     Batching", CDB design: scheduling at loop-iteration granularity, boundary
@@ -24,7 +28,13 @@ Readings (pages silent or loose):
     multiple of peek_every.  The streak goes up by one when delta < tau and
     returns to zero otherwise; iterations without a probe leave it unchanged; it
     starts at zero for every token.  The lane exits at l once streak >= patience.
-  * Early exit is off when tau <= 0 or patience == 0.
+  * Early exit is off when tau <= 0 or patience == 0 (hidden-state mode), or
+    logit_margin <= 0 or patience == 0 (margin mode).
+  * Margin mode: a probe succeeds when margin >= logit_margin (the pages say
+    the loop stops when the prediction is confident; the threshold itself is
+    read as confident enough); success extends the streak, failure resets it,
+    as in hidden-state mode.  Only the per-lane definition (generate_lane)
+    implements it.
   * After a token ran D iterations the lane's cap becomes D; the next token runs
     min(L_requested, cap) iterations.
   * N emitted tokens: the first comes from the last prompt position; the N-th
@@ -45,20 +55,34 @@ class EarlyExit:
     min_L: int = 2
     patience: int = 0
     peek_every: int = 1
+    logit_margin: float = 0.0   # > 0: margin mode (tau is then unused)
+
+    @property
+    def margin_mode(self) -> bool:
+        return self.logit_margin > 0
 
     @property
     def enabled(self) -> bool:
+        if self.margin_mode:
+            return self.patience > 0
         return self.tau > 0 and self.patience > 0
 
     def is_probe(self, l: int) -> bool:
         return self.enabled and l > self.min_L and (l - self.min_L - 1) % self.peek_every == 0
 
 
+def probe_succeeds(ee: EarlyExit, metric: float) -> bool:
+    """Hidden-state mode: the relative change is below tau; margin mode: the
+    top-1 / top-2 logit margin reaches logit_margin."""
+    return metric >= ee.logit_margin if ee.margin_mode else metric < ee.tau
+
+
 def streak_update(ee: EarlyExit, l: int, delta: float, streak: int) -> tuple[int, bool]:
-    """The rule after iteration l: returns (new streak, exit now)."""
+    """The rule after iteration l (delta: the probe's metric): returns (new
+    streak, exit now)."""
     if not ee.is_probe(l):
         return streak, False
-    streak = streak + 1 if delta < ee.tau else 0
+    streak = streak + 1 if probe_succeeds(ee, delta) else 0
     return streak, streak >= ee.patience
 
 
@@ -83,8 +107,8 @@ def rel_l2(h: np.ndarray, h_prev: np.ndarray) -> float:
 class Probe:
     token: int          # index of the emitted token this iteration belongs to
     l: int              # iteration (1-based)
-    delta: float
-    below: bool         # delta < tau
+    delta: float        # the probe's metric: relative change (or top-2 logit margin in margin mode)
+    below: bool         # the probe succeeded (delta < tau, or margin >= logit_margin)
 
     def margin(self, tau: float) -> float:
         """|delta / tau - 1|: how far the decision sits from the threshold."""
@@ -100,13 +124,14 @@ class LaneResult:
     prompt_hidden: np.ndarray | None = None
 
 
-def _probe_step(ee: EarlyExit, t: int, l: int, h, h_prev, streak: int, probes: list):
-    """Record the probe after iteration l (if any) and apply the rule."""
+def _probe_step(ee: EarlyExit, t: int, l: int, h, h_prev, streak: int, probes: list, W=None):
+    """Record the probe after iteration l (if any) and apply the rule.  In
+    margin mode the metric is the head's top-2 margin at h (needs W)."""
     if not ee.is_probe(l):
         return streak, False
-    delta = rel_l2(h, h_prev)
-    probes.append(Probe(t, l, delta, delta < ee.tau))
-    return streak_update(ee, l, delta, streak)
+    metric = float(M.top2_margin(M.head_logits(W, h))) if ee.margin_mode else rel_l2(h, h_prev)
+    probes.append(Probe(t, l, metric, probe_succeeds(ee, metric)))
+    return streak_update(ee, l, metric, streak)
 
 
 def generate_lane(W: M.Weights, prompt, L_req: int, n_new: int, ee: EarlyExit = EarlyExit(),
@@ -144,7 +169,7 @@ def generate_lane(W: M.Weights, prompt, L_req: int, n_new: int, ee: EarlyExit = 
             for l in range(1, L_run + 1):
                 h_prev = h
                 h = M.loop_iteration(W, h, pos, cache, l)
-                streak, exit_now = _probe_step(ee, t, l, h[0], h_prev[0], streak, probes)
+                streak, exit_now = _probe_step(ee, t, l, h[0], h_prev[0], streak, probes, W)
                 if target is not None:
                     exit_now = l == target
                 if exit_now:
@@ -197,6 +222,8 @@ def generate_cdb(W: M.Weights, prompts, per_lane_L, n_new: int, ee: EarlyExit = 
     formed; (3) run the boundary queue: head + greedy token, then embed + pre
     blocks for lanes that still have tokens to emit.  Returns (per-lane
     LaneResult list, number of loop steps)."""
+    if ee.margin_mode:
+        raise NotImplementedError("margin-mode early exit is defined per lane (generate_lane) only")
     shape = W.shape
     d, H, hd = shape.d, shape.n_heads, shape.head_dim
     lanes = []

@@ -145,3 +145,55 @@ def test_edge_cases(tiny):
         D.generate_lane(tiny, P, 0, 2)
     with pytest.raises(ValueError):
         D.generate_lane(tiny, P, 3, 3, forced_depths=[0, 4, 1])
+
+
+# ------------------------------------------------ logit-margin early exit ----
+
+def test_margin_mode_huge_threshold_never_exits(tiny):
+    P = S.prompts(1, 8, tiny.shape.vocab, seed=61)[0]
+    ee = D.EarlyExit(min_L=1, patience=1, logit_margin=1e9)
+    r = D.generate_lane(tiny, P, 6, 4, ee)
+    assert r.depths.tolist() == [6] * 4
+    assert r.probes and not any(p.below for p in r.probes)
+    fixed = D.generate_lane(tiny, P, 6, 4)
+    assert np.array_equal(fixed.logits, r.logits)
+
+
+def test_margin_mode_tiny_threshold_exits_at_earliest_then_clamps(tiny):
+    # every probe with a non-zero margin succeeds: exit at min_L + 1 + (patience - 1) * peek_every
+    P = S.prompts(1, 8, tiny.shape.vocab, seed=62)[0]
+    ee = D.EarlyExit(min_L=2, patience=2, peek_every=2, logit_margin=1e-12)
+    r = D.generate_lane(tiny, P, 8, 4, ee)
+    assert r.depths.tolist() == [8, 5, 5, 5]
+    forced = D.generate_lane(tiny, P, 8, 4, forced_depths=[0, 5, 5, 5])
+    assert np.array_equal(forced.logits, r.logits)
+
+
+def test_margin_probe_metric_is_the_heads_top2_margin(tiny):
+    # the metric recorded at iteration l of token 1 equals the top-2 margin of the
+    # logits a run stopped at l emits for token 1 (same hidden state, same head)
+    P = S.prompts(1, 8, tiny.shape.vocab, seed=63)[0]
+    ee = D.EarlyExit(min_L=1, patience=9, logit_margin=1e9)  # probes at l = 2, 3, 4 and no exit
+    r = D.generate_lane(tiny, P, 4, 2, ee)
+    got = {p.l: p.delta for p in r.probes if p.token == 1}
+    assert sorted(got) == [2, 3, 4]
+    for l in (2, 3, 4):
+        stopped = D.generate_lane(tiny, P, 4, 2, forced_depths=[0, l])
+        s = np.sort(stopped.logits[1])
+        assert got[l] == s[-1] - s[-2]
+
+
+def test_margin_mode_rule_on_recorded_margins(tiny):
+    P = S.prompts(1, 8, tiny.shape.vocab, seed=64)[0]
+    probe_all = D.EarlyExit(min_L=0, patience=99, logit_margin=1e9)
+    margins = [p.delta for p in D.generate_lane(tiny, P, 6, 2, probe_all).probes if p.token == 1]
+    thr = float(np.median(margins))
+    ee = D.EarlyExit(min_L=0, patience=1, logit_margin=thr)
+    r = D.generate_lane(tiny, P, 6, 2, ee)
+    first = next(l for l, m in enumerate(margins, start=1) if m >= thr)
+    assert r.depths[1] == first
+
+
+def test_margin_mode_is_per_lane_only(tiny):
+    with pytest.raises(NotImplementedError):
+        D.generate_cdb(tiny, S.prompts(1, 4, tiny.shape.vocab), [2], 2, D.EarlyExit(patience=1, logit_margin=1.0))
