@@ -135,17 +135,24 @@ def _probe_step(ee: EarlyExit, t: int, l: int, h, h_prev, streak: int, probes: l
 
 
 def generate_lane(W: M.Weights, prompt, L_req: int, n_new: int, ee: EarlyExit = EarlyExit(),
-                  forced_depths=None, keep_logits: bool = True, keep_prompt_hidden: bool = False) -> LaneResult:
+                  forced_depths=None, keep_logits: bool = True, keep_prompt_hidden: bool = False,
+                  warmup_tokens: int = 0, warmup_L: int = 2) -> LaneResult:
     """The definition: one lane, token by token, iteration by iteration.
 
     forced_depths[t] (t >= 1), when given, replaces the early-exit decision of
     token t by that depth (used to follow another implementation's decision at a
-    probe that sits on the threshold); probes are still recorded."""
+    probe that sits on the threshold); probes are still recorded.
+
+    warmup_tokens > 0 ("Dynamic-L Inference", L scheduling; "CLI Reference",
+    --l-warmup-tokens / --l-warmup-L): decode tokens 1..warmup_tokens run
+    min(warmup_L, L_req) iterations and leave the cap alone; later tokens run
+    the full schedule, their deeper iterations reading the warmup positions
+    through KVCache.deep_fallback.  The prompt runs the full L_req."""
     if L_req < 1:
         raise ValueError("L must be >= 1")
     prompt = np.asarray(prompt)
     T = len(prompt)
-    cache = M.KVCache(W.shape, T + max(n_new - 1, 0))
+    cache = M.KVCache(W.shape, T + max(n_new - 1, 0), deep_fallback=warmup_tokens > 0)
     x, _ = M.forward(W, prompt, L_req, cache)
     tokens = np.zeros(n_new, dtype=np.int64)
     depths = np.zeros(n_new, dtype=np.int64)
@@ -160,7 +167,8 @@ def generate_lane(W: M.Weights, prompt, L_req: int, n_new: int, ee: EarlyExit = 
             p = T + t - 1
             pos = np.array([p])
             h = M.pre_blocks(W, M.embed(W, [tokens[t - 1]]), pos, cache)
-            L_run = min(L_req, L_cap)
+            warm = t <= warmup_tokens
+            L_run = min(warmup_L, L_req) if warm else min(L_req, L_cap)
             target = None if forced_depths is None else int(forced_depths[t])
             if target is not None and not (1 <= target <= L_run):
                 raise ValueError("forced depth out of range")
@@ -175,7 +183,8 @@ def generate_lane(W: M.Weights, prompt, L_req: int, n_new: int, ee: EarlyExit = 
                 if exit_now:
                     depth = l
                     break
-            L_cap = depth
+            if not warm:
+                L_cap = depth
         lg = M.head_logits(W, h[0])
         tokens[t] = M.argmax_lowest(lg)
         depths[t] = depth

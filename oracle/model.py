@@ -130,12 +130,18 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, q_pos: np.ndarray, k_pos
 
 class KVCache:
     """Per-lane cache: one (K, V) slab per slot; a slot is a pre block ("pre", b)
-    or a loop iteration and body layer ("loop", l, m), l counted from 1."""
+    or a loop iteration and body layer ("loop", l, m), l counted from 1.
 
-    def __init__(self, shape: ModelShape, max_seq: int):
+    deep_fallback (the reading for a lane whose L rises, e.g. after an L-warmup
+    phase; the pages do not say what a deeper iteration attends to at positions
+    computed shallower): a position with no entry in ("loop", l, m) is read from
+    the deepest iteration l' < l that holds it at the same body layer m."""
+
+    def __init__(self, shape: ModelShape, max_seq: int, deep_fallback: bool = False):
         self.shape = shape
         self.max_seq = max_seq
         self.slots: dict = {}
+        self.deep_fallback = deep_fallback
 
     def slab(self, slot):
         if slot not in self.slots:
@@ -151,10 +157,23 @@ class KVCache:
         filled[pos] = True
 
     def read_upto(self, slot, p_max: int):
-        """K, V, positions of all filled entries at positions <= p_max."""
+        """K, V, positions of all filled entries at positions <= p_max (with
+        deep_fallback, loop-slot gaps filled from shallower iterations)."""
         K, V, filled = self.slab(slot)
-        idx = np.nonzero(filled[: p_max + 1])[0]
-        return K[idx], V[idx], idx
+        if not (self.deep_fallback and slot[0] == "loop"):
+            idx = np.nonzero(filled[: p_max + 1])[0]
+            return K[idx], V[idx], idx
+        _, l, m = slot
+        Kf, Vf, have = K[: p_max + 1].copy(), V[: p_max + 1].copy(), filled[: p_max + 1].copy()
+        for lower in range(l - 1, 0, -1):  # deepest first
+            if ("loop", lower, m) not in self.slots:
+                continue
+            Kl, Vl, fl = self.slots[("loop", lower, m)]
+            take = ~have & fl[: p_max + 1]
+            Kf[take], Vf[take] = Kl[: p_max + 1][take], Vl[: p_max + 1][take]
+            have |= take
+        idx = np.nonzero(have)[0]
+        return Kf[idx], Vf[idx], idx
 
 
 # ------------------------------------------------------------------ blocks ----

@@ -197,3 +197,52 @@ def test_margin_mode_rule_on_recorded_margins(tiny):
 def test_margin_mode_is_per_lane_only(tiny):
     with pytest.raises(NotImplementedError):
         D.generate_cdb(tiny, S.prompts(1, 4, tiny.shape.vocab), [2], 2, D.EarlyExit(patience=1, logit_margin=1.0))
+
+
+# ------------------------------------------------------------- L warmup ----
+
+def test_kv_deep_fallback_reads_the_deepest_shallower_iteration():
+    from oracle import model as M
+    sh = S.TINY
+    c = M.KVCache(sh, 8, deep_fallback=True)
+    H, hd = sh.n_heads, sh.head_dim
+    for l, upto in ((1, 5), (2, 3), (3, 2)):  # iteration l holds positions 0..upto-1
+        for p in range(upto):
+            c.write(("loop", l, 0), np.array([p]), np.full((1, H, hd), 10.0 * l + p), np.full((1, H, hd), -10.0 * l - p))
+    K, V, idx = c.read_upto(("loop", 3, 0), 4)
+    assert idx.tolist() == [0, 1, 2, 3, 4]
+    assert [float(K[i, 0, 0]) for i in range(5)] == [30.0, 31.0, 22.0, 13.0, 14.0]
+    assert [float(V[i, 0, 0]) for i in range(5)] == [-30.0, -31.0, -22.0, -13.0, -14.0]
+    plain = M.KVCache(sh, 8)
+    plain.slots = c.slots
+    assert plain.read_upto(("loop", 3, 0), 4)[2].tolist() == [0, 1]  # without the reading: only its own entries
+
+
+def test_warmup_schedule_and_its_degenerate_cases(tiny):
+    P = S.prompts(1, 8, tiny.shape.vocab, seed=71)[0]
+    r = D.generate_lane(tiny, P, 6, 6, warmup_tokens=3, warmup_L=2)
+    assert r.depths.tolist() == [6, 2, 2, 2, 6, 6]     # the prompt at full L, 3 shallow tokens, then full L again
+    plain = D.generate_lane(tiny, P, 6, 6)
+    # warmup at the full depth, or no warmup tokens, is the plain run
+    assert np.array_equal(D.generate_lane(tiny, P, 6, 6, warmup_tokens=3, warmup_L=6).logits, plain.logits)
+    assert np.array_equal(D.generate_lane(tiny, P, 6, 6, warmup_tokens=0, warmup_L=2).logits, plain.logits)
+    # the shallow tokens are those of a plain run forced to depth 2 (their keys are all present)
+    forced = D.generate_lane(tiny, P, 6, 4, forced_depths=[0, 2, 2, 2])
+    assert np.array_equal(forced.logits, r.logits[:4])
+
+
+def test_warmup_deep_tokens_read_the_warmup_positions(tiny, monkeypatch):
+    # after the warmup, iterations 3..6 of token 4 read the 3 warmup positions through their
+    # iteration-2 entries: a cache without that reading (which sees only the prompt and the
+    # token itself there) gives different logits, while every token before it is unchanged
+    P = S.prompts(1, 8, tiny.shape.vocab, seed=72)[0]
+    r = D.generate_lane(tiny, P, 6, 5, warmup_tokens=3, warmup_L=2)
+    from oracle import model as M
+
+    class NoReading(M.KVCache):
+        def __init__(self, shape, max_seq, deep_fallback=False):
+            super().__init__(shape, max_seq, deep_fallback=False)
+    monkeypatch.setattr(D.M, "KVCache", NoReading)
+    other = D.generate_lane(tiny, P, 6, 5, warmup_tokens=3, warmup_L=2)
+    assert np.array_equal(other.logits[:4], r.logits[:4])
+    assert not np.allclose(other.logits[4], r.logits[4])
