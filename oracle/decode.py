@@ -193,6 +193,51 @@ def generate_lane(W: M.Weights, prompt, L_req: int, n_new: int, ee: EarlyExit = 
     return LaneResult(tokens, depths, logits_all, probes, x if keep_prompt_hidden else None)
 
 
+def speculative_lane(W: M.Weights, prompt, L_draft: int, L_verify: int, n_new: int, draft_ahead: int):
+    """Self-speculative greedy decode of one lane ("CLI Reference", speculate:
+    --draft-loops, --verify-loops, --draft-ahead, temperature 0): the same
+    weights and one cache for both passes.  Each round drafts up to draft_ahead
+    tokens at L_draft, one position at a time; then runs the drafted positions
+    at L_verify as one causal batch, keeps the drafted tokens up to the first
+    one the verify pass's greedy choice disagrees with, and takes the verify
+    pass's own token there.  The verify pass recomputes iterations 1..L_draft
+    of the drafted positions (their values equal the draft's, since the hidden
+    state at iteration j does not depend on L >= j); every position is
+    rewritten before anything later reads it.  Returns (tokens int [n_new],
+    rounds).  With greedy choices the tokens are those of a plain greedy run at
+    L_verify; the draft only decides how many positions one verify pass covers."""
+    if not (1 <= L_draft and 1 <= L_verify and draft_ahead >= 1):
+        raise ValueError("bad speculation parameters")
+    prompt = np.asarray(prompt)
+    T = len(prompt)
+    cache = M.KVCache(W.shape, T + n_new + draft_ahead)
+    x, _ = M.forward(W, prompt, L_verify, cache)
+    tokens = [int(M.argmax_lowest(M.head_logits(W, x[-1])))]
+    rounds = 0
+    while len(tokens) < n_new:
+        rounds += 1
+        p0 = T + len(tokens) - 1          # position of the last token taken (not computed yet)
+        k = min(draft_ahead, n_new - len(tokens))
+        draft, prev = [], tokens[-1]
+        for j in range(k):                # draft: one position at a time, shallow
+            pos = np.array([p0 + j])
+            h = M.pre_blocks(W, M.embed(W, [prev]), pos, cache)
+            for l in range(1, L_draft + 1):
+                h = M.loop_iteration(W, h, pos, cache, l)
+            prev = int(M.argmax_lowest(M.head_logits(W, h[0])))
+            draft.append(prev)
+        pos = np.arange(p0, p0 + k)       # verify: the same positions together, deep
+        h = M.pre_blocks(W, M.embed(W, [tokens[-1]] + draft[:-1]), pos, cache)
+        for l in range(1, L_verify + 1):
+            h = M.loop_iteration(W, h, pos, cache, l)
+        for j in range(k):
+            choice = int(M.argmax_lowest(M.head_logits(W, h[j])))
+            tokens.append(choice)
+            if choice != draft[j]:
+                break
+    return np.array(tokens[:n_new], dtype=np.int64), rounds
+
+
 # ------------------------------------------------ continuous depth batching ----
 
 LOOP, BOUNDARY, DONE = 0, 1, 2

@@ -246,3 +246,18 @@ def test_warmup_deep_tokens_read_the_warmup_positions(tiny, monkeypatch):
     other = D.generate_lane(tiny, P, 6, 5, warmup_tokens=3, warmup_L=2)
     assert np.array_equal(other.logits[:4], r.logits[:4])
     assert not np.allclose(other.logits[4], r.logits[4])
+
+
+# ------------------------------------------------ self-speculative decode ----
+
+@pytest.mark.parametrize("L_draft,draft_ahead", [(1, 1), (2, 4), (3, 3), (6, 2)])
+def test_speculative_tokens_equal_greedy_at_the_verify_depth(tiny, L_draft, draft_ahead):
+    P = S.prompts(1, 10, tiny.shape.vocab, seed=81)[0]
+    ref = D.generate_lane(tiny, P, 6, 9)
+    from oracle import model as M
+    assert min(M.top2_margin(lg) for lg in ref.logits) > 1e-9  # no near-tie for the batched verify to flip
+    tok, rounds = D.speculative_lane(tiny, P, L_draft, 6, 9, draft_ahead)
+    assert tok.tolist() == ref.tokens.tolist()
+    assert -(-8 // draft_ahead) <= rounds <= 8
+    if L_draft == 6:  # the draft is the verify model: every drafted token is accepted
+        assert rounds == -(-8 // draft_ahead)
