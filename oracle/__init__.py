@@ -13,7 +13,9 @@ It is written to be read against the pages, not to be fast:
              the transformer block, embed -> pre blocks -> loop x L -> head.
   decode.py  greedy decode with per-lane L, hidden-state relative-L2 early exit,
              monotonic L clamp, and an iteration-granularity (continuous depth
-             batching) scheduler over many lanes.
+             batching) scheduler over many lanes; per lane also logit-margin
+             early exit, an L-warmup schedule (with KVCache's deepest-iteration
+             reading) and self-speculative decoding.
 
 Parity status: every function is pinned by the `-m "not gpu"` tests in
 tests/test_oracle_*.py against closed forms, invariants, brute force on tiny
@@ -25,4 +27,4 @@ each step.
 """
 from . import quant, model, decode  # noqa: F401
 from .model import build_weights, Weights  # noqa: F401
-from .decode import EarlyExit, generate_lane, generate_cdb  # noqa: F401
+from .decode import EarlyExit, generate_lane, generate_cdb, speculative_lane  # noqa: F401
