@@ -261,3 +261,17 @@ def test_speculative_tokens_equal_greedy_at_the_verify_depth(tiny, L_draft, draf
     assert -(-8 // draft_ahead) <= rounds <= 8
     if L_draft == 6:  # the draft is the verify model: every drafted token is accepted
         assert rounds == -(-8 // draft_ahead)
+
+
+def test_golden_margin_exit_schedule():
+    with open(os.path.join(GOLDEN, "ee_margin_schedule.txt")) as f:
+        rows = [l for l in f if l.strip() and not l.startswith("#")]
+    assert rows
+    for line in rows:
+        head, metrics, probes, depth = [p.strip() for p in line.split("|")]
+        thr, min_L, pat, peek, L = head.split()
+        ee = D.EarlyExit(min_L=int(min_L), patience=int(pat), peek_every=int(peek), logit_margin=float(thr))
+        L = int(L)
+        want = [] if probes == "-" else [int(x) for x in probes.split()]
+        assert [l for l in range(1, L + 1) if ee.is_probe(l)] == want
+        assert D.exit_iteration([float(x) for x in metrics.split()], L, ee) == int(depth), line
