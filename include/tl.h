@@ -85,7 +85,7 @@ typedef struct tl_config {
     int32_t max_lanes;        /* lanes held at once                               */
     int32_t max_seq;          /* prompt + generated tokens per lane               */
     int32_t L_max;            /* largest per-lane loop count                      */
-    int32_t kv_page_tokens;   /* tokens per KV page (power of two, >= 16)         */
+    int32_t kv_page_tokens;   /* tokens per KV page (power of two, >= 32)         */
     int32_t kv_pool_pages;    /* pages in the pool; 0 = one per lane/slot/page    */
     int32_t max_prefill_tokens; /* prompt rows one prefill call computes, summed
                                    over its lanes; 0 = max_seq                   */

@@ -207,3 +207,66 @@ def test_weight_draw_order_and_effective_values():
     assert [n for n, _ in S.matrix_shapes(sh)][-1] == "head"
     W = O.build_weights(sh, S.master_weights(sh), S.gains(sh))
     assert np.max(np.abs(W.head - ws["head"])) < 0.02 * 5 / 7 / 2 * 1.01 + 1e-3
+
+
+# ------------------------------------------------------- embed and head ----
+
+def _scalar_int4_row(packed_row, scales_row, group):
+    """One row of an INT4 matrix, element by element: byte k // 2 holds element
+    k in its low nibble when k is even and in its high nibble when k is odd;
+    the value is (nibble - 8) * the fp16 scale of group k // group."""
+    out = []
+    for k in range(2 * len(packed_row)):
+        byte = int(packed_row[k // 2])
+        u = (byte & 0xF) if k % 2 == 0 else (byte >> 4)
+        out.append((u - 8) * float(scales_row[k // group]))
+    return out
+
+
+@pytest.fixture(scope="module")
+def tiny_kept():
+    sh = S.TINY
+    gains = S.gains(sh, random_seed=5)
+    W = O.build_weights(sh, S.master_weights(sh), gains, keep_int4=True)
+    return sh, gains, W
+
+
+def test_embed_is_the_dequantised_embedding_row(tiny_kept):
+    sh, _, W = tiny_kept
+    packed, scales = W.int4["embed"]
+    toks = [0, 7, sh.vocab - 1, 7]
+    got = M.embed(W, toks)
+    for r, t in enumerate(toks):
+        assert got[r].tolist() == _scalar_int4_row(packed[t], scales[t], sh.group), t
+    # the embedding table is the first matrix drawn from the seed-0 stream
+    master = np.random.Generator(np.random.PCG64(0)).standard_normal((sh.vocab, sh.d)) * 0.02
+    s = scales.astype(np.float64)
+    assert np.all(np.abs(got - master[toks]) <= np.repeat(s[toks], sh.group, axis=1) / 2 + 1e-18)
+
+
+def test_head_logits_match_scalar_loops(tiny_kept):
+    """logits[v] = sum_i RMSNorm(h; g_final)[i] * Whead[v, i] with the final
+    gain (not a block's), the norm applied, and the head's own matrix (untied:
+    the last matrix drawn, not the embedding)."""
+    sh, gains, W = tiny_kept
+    d, eps = sh.d, sh.rms_eps
+    h = S.random_vectors((2, d), seed=61, scale=3.0)   # RMS ~3: a dropped norm cannot pass
+    got = M.head_logits(W, h)
+    packed, scales = W.int4["head"]
+    g = gains["final.g"]
+    rows = [_scalar_int4_row(packed[v], scales[v], sh.group) for v in range(sh.vocab)]
+    for r in range(2):
+        ms = sum(float(x) * float(x) for x in h[r]) / d
+        y = [float(h[r][i]) / math.sqrt(ms + eps) * float(g[i]) for i in range(d)]
+        want = [sum(y[i] * row[i] for i in range(d)) for row in rows]
+        assert np.allclose(got[r], want, rtol=0, atol=1e-12)
+    # the head matrix is the last draw of the seed-0 stream
+    rng = np.random.Generator(np.random.PCG64(0))
+    last = None
+    for _, (nr, nc) in S.matrix_shapes(sh):
+        last = rng.standard_normal((nr, nc)) * 0.02
+    dq = np.array(rows)
+    assert np.all(np.abs(dq - last) <= np.repeat(scales.astype(np.float64), sh.group, axis=1) / 2 + 1e-18)
+    # and it is not the embedding table, nor does a block gain stand in for g_final
+    assert not np.array_equal(W.int4["head"][0], W.int4["embed"][0])
+    assert not np.allclose(got, M.rmsnorm(h, gains["pre0.g1"], eps) @ W.head.T, atol=1e-6)
