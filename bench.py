@@ -303,6 +303,24 @@ def run_ours(args, rank, world, local_rank):
                 "algorithmic_bytes_per_launch": round(per_launch), "launches_per_step": launches,
                 "peak_source": hbm_src}
 
+    # live read-bandwidth peaks (outside every timed region) and the projections' fraction of the L2 one:
+    # the loop block's INT4 weights are re-read every iteration, so L2 is their bound when they stay resident
+    live = live_read_peaks(dev)
+    roof_proj = None
+    if "projections" in kinds:
+        a = kinds["projections"]["algorithmic_GB_per_s"]
+        roof_proj = {"kernel": "decode W4A16 projections (gemv_stream_kernel <= 8 rows, tc_gemm_kernel above): "
+                               + alg["projections"][1],
+                     "bound": "l2", "achieved": a, "peak": live["l2_read_gbs"], "unit": "GB/s",
+                     "frac": round(a / live["l2_read_gbs"], 4), "frac_of_hbm": round(a / hbm, 4),
+                     "peak_source": "live tl_read_probe L2 read bandwidth of this run"}
+    # early exits that fired: tokens (after the first) whose loop stopped below min(L requested, cap)
+    exited = 0
+    for i in range(wl.n_lanes):
+        for t in range(1, wl.n_new):
+            if depths[i, t] < min(int(Ls[i]), int(depths[i, t - 1])):
+                exited += 1
+
     # end to end through tl_generate: pinned host prompts in, host tokens out
     e2e = None
     if not args.no_e2e:
@@ -344,12 +362,16 @@ def run_ours(args, rank, world, local_rank):
         "lane_iterations_no_exit": int(sum(int(L) * (wl.n_new - 1) for L in Ls)),
         "depth_histogram": {int(k): int(v) for k, v in zip(*np.unique(depths[:, 1:], return_counts=True))},
         "ticks_per_step": units["ticks"],
+        "early_exit_tokens": exited,
+        "early_exit_fired": exited > 0,
         "kernel_time": kinds,
         "roofline": roof,
+        "roofline_projections": roof_proj,
+        "peaks_live": live,
         "clocks": clk.summary(),
         "e2e": e2e,
     }
-    return out, m, P, Ls
+    return out, m, P, Ls, depths
 
 
 
@@ -422,24 +444,15 @@ def whole_job_rate(units_per_rank: float, max_ms: float, world: int) -> float:
     return world * units_per_rank / (max_ms / 1e3)
 
 
-def _l2_copy_gbs(dev) -> float:
-    """Live L2 figure: copy between two 24 MiB buffers (48 MiB of traffic, all
-    L2-resident), best of 20, read + write bytes."""
-    import torch
-    a = torch.randn(6 << 20, device=dev)
-    b = torch.empty_like(a)
-    for _ in range(5):
-        b.copy_(a)
-    best = 1e9
-    for _ in range(20):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(10):
-            b.copy_(a)
-        e1.record()
-        e1.synchronize()
-        best = min(best, e0.elapsed_time(e1) / 10)
-    return 2 * a.numel() * 4 / 1e9 / (best / 1e3)
+def live_read_peaks(dev) -> dict:
+    """Read bandwidth measured in this run with the library's read probe
+    (tl_read_probe): a 64 MiB buffer read 32 times per launch (L2-resident after
+    its first pass: the denominator for weights re-read across loop
+    iterations) and a 4 GiB buffer read once (HBM)."""
+    import dynamic_depth_b200 as T
+    return {"l2_read_gbs": round(T.read_bandwidth_gbs(64 << 20, 32, dev), 1),
+            "hbm_read_gbs": round(T.read_bandwidth_gbs(4 << 30, 1, dev), 1),
+            "source": "tl_read_probe, best of 5 event-timed launches (64 MiB x 32 reads; 4 GiB x 1 read)"}
 
 
 def _common(metric, value, unit, world, args, ms, config, dtype, hib=True):
@@ -615,7 +628,8 @@ def run_lsweep(args, rank, world, local_rank):
             m.close()
             del m
             torch.cuda.empty_cache()
-    l2 = _l2_copy_gbs(dev)
+    live = live_read_peaks(dev)
+    l2 = live["l2_read_gbs"]
     pk = _peaks()
     hbm = float(pk.get("hbm_gbs", 6650.0))
     sh = S.M407
@@ -640,7 +654,7 @@ def run_lsweep(args, rank, world, local_rank):
         "roofline": {"kernel": "streamed W4A16 GEMV projections (gemv_stream_kernel), INT4, L=8",
                      "bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(ach / hbm, 4), "traffic": None,
-                     "l2_copy_gbs_live": round(l2, 1), "frac_of_l2_copy": round(ach / l2, 4),
+                     "l2_read_gbs_live": l2, "frac_of_l2_read": round(ach / l2, 4),
                      "algorithmic_bytes_per_step": int(proj_bytes),
                      "peak_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in pk
                      else "of fallback 6650 GB/s"},
@@ -804,10 +818,13 @@ def oracle_sample(n_tokens: int = 8):
     t0 = time.perf_counter()
     D.generate_lane(W, P[0], L, 1, ee, keep_logits=False)
     t1 = time.perf_counter()
-    D.generate_lane(W, P[0], L, n_tokens + 1, ee, keep_logits=False)
+    r = D.generate_lane(W, P[0], L, n_tokens + 1, ee, keep_logits=False)
     t2 = time.perf_counter()
     prompt_s = t1 - t0
     decode_s = max((t2 - t1) - prompt_s, 1e-9)
+    oracle_sample.last = {"depths": r.depths.tolist(),
+                          "min_probe_delta": min((p.delta for p in r.probes), default=None),
+                          "probes": len(r.probes)}
     return n_tokens / decode_s, decode_s, prompt_s, len(os.sched_getaffinity(0)), L
 
 
@@ -877,12 +894,19 @@ def main():
         if rank == 0:
             print(json.dumps(out))
         return 0
-    out, m, P, Ls = run_ours(args, rank, world, local_rank)
+    out, m, P, Ls, depths = run_ours(args, rank, world, local_rank)
     if rank == 0 and not args.no_cpu_baseline:
         v, dec_s, pr_s, cores, L = oracle_sample(8)
         out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": f"lane 0 (L={L}): 512-token prompt ({pr_s:.1f} s, excluded) then 8 greedy "
                                          f"tokens in {dec_s:.1f} s; fp64 NumPy"}
+        # the oracle's own exit decisions on that sample, beside the GPU's lane-0 depths
+        o = oracle_sample.last
+        n = len(o["depths"])
+        out["oracle_lane0_check"] = {"oracle_depths": o["depths"], "gpu_depths": depths[0, :n].tolist(),
+                                     "equal": o["depths"] == depths[0, :n].tolist(),
+                                     "oracle_probes": o["probes"], "oracle_min_probe_delta": o["min_probe_delta"],
+                                     "tau": S.workload(WORKLOAD).ee_tau}
     if world > 1:
         import torch
         torch.distributed.barrier()

@@ -161,3 +161,29 @@ class LoopedLM:
         s = _lib.TlStats()
         check(lib().tl_stats_get(self.h, C.byref(s)), "tl_stats_get")
         return {k: getattr(s, k) for k, _ in s._fields_}
+
+
+def read_bandwidth_gbs(n_bytes: int, reps: int, device="cuda:0", trials: int = 5) -> float:
+    """Read bandwidth (GB/s) of tl_read_probe over an n_bytes device buffer read
+    reps times per launch: best of `trials` event-timed launches after one
+    untimed launch (which also brings an L2-sized buffer into L2)."""
+    import torch
+    dev = torch.device(device)
+    buf = torch.ones(n_bytes // 4, dtype=torch.int32, device=dev)
+    n_sink = 4 * torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.zeros(n_sink, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def launch():
+        check(lib().tl_read_probe(buf.data_ptr(), buf.numel() * 4, reps, sink.data_ptr(), n_sink, stream.cuda_stream),
+              "tl_read_probe")
+    launch()
+    best = float("inf")
+    for _ in range(trials):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        launch()
+        e1.record(stream)
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return buf.numel() * 4 * reps / 1e9 / (best / 1e3)

@@ -64,6 +64,7 @@ SIGNATURES = {
     "tl_profile_end": (C.c_int, [C.c_void_p, C.POINTER(C.c_int64), C.POINTER(C.c_double)]),
     "tl_head_argmax_static": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_float, C.c_void_p, C.c_void_p,
                                          C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "tl_read_probe": (C.c_int, [C.c_void_p, C.c_size_t, C.c_int32, C.c_void_p, C.c_int32, C.c_void_p]),
     "tl_stats_get": (C.c_int, [C.c_void_p, C.POINTER(TlStats)]),
     "tl_strerror": (C.c_char_p, [C.c_int]),
     "tl_last_cuda_error": (C.c_char_p, []),

@@ -156,6 +156,10 @@ extern "C" int tl_head_argmax_static(const float* dev_h, int32_t rows, const flo
   namespace hs = head_static;
   if (!dev_h || !dev_g_final || !dev_head_packed || !dev_head_scales || !dev_argmax) return TL_EINVAL;
   if (rows < 1 || d < 32 || d % 32 || group < 32 || group % 32 || d % group || V < 1) return TL_EINVAL;
+  // the head rows are read as 16-byte words; everything else by its element size
+  if (((uintptr_t)dev_head_packed & 15) || ((uintptr_t)dev_head_scales & 1) || ((uintptr_t)dev_h & 3) ||
+      ((uintptr_t)dev_g_final & 3) || ((uintptr_t)dev_logits & 3) || ((uintptr_t)dev_argmax & 3))
+    return TL_EINVAL;
   const int n_parts = (V + hs::kRowsPerCta - 1) / hs::kRowsPerCta;
   // sizes beyond the static array's capacity
   if (rows > hs::kMaxRows || d > hs::kMaxD || n_parts > hs::kMaxParts) return TL_ENOMEM;

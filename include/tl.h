@@ -342,11 +342,27 @@ int tl_profile_end(tl_ctx* ctx, int64_t* out_groups, double* out_total_ms);
  * call's contents (each call writes all it reads); calls whose kernels
  * overlap on the GPU (unordered streams) race on it.  The first call on a
  * device looks up the array's device address with that device current; make
- * that first call before any stream capture begins.  TL_EINVAL on NULL inputs
- * or d, group not multiples of 32 / group not dividing d. */
+ * that first call before any stream capture begins.  TL_EINVAL on NULL inputs,
+ * d or group not multiples of 32, group not dividing d, a head pointer not
+ * 16-byte aligned or another pointer not aligned to its element size
+ * (nothing is enqueued). */
 int tl_head_argmax_static(const float* dev_h, int32_t rows, const float* dev_g_final, float rms_eps,
                           const uint8_t* dev_head_packed, const uint16_t* dev_head_scales, int32_t V,
                           int32_t d, int32_t group, float* dev_logits, int32_t* dev_argmax, void* cuda_stream);
+
+/* ---------------------------------------------------------- measurement -- */
+
+/* Read-bandwidth probe (a measurement aid, not a step of the model; the pages
+ * relate the loop block's cost to where its weights are read from,
+ * "Benchmark Comparison" (measured benchmarks), section 6, L2 residency):
+ * 4 CTAs per SM read dev_src[0 .. bytes) with 16-byte loads, reps times over,
+ * and write one word per CTA into dev_sink.  The caller times it with events
+ * on cuda_stream: a buffer well under the L2 capacity gives the L2 read
+ * bandwidth (after a first pass), one far larger than L2 the HBM read
+ * bandwidth.  dev_src 16-byte aligned, bytes a multiple of 16, reps >= 1,
+ * n_sink >= 4 x the SM count; TL_EINVAL otherwise (nothing enqueued). */
+int tl_read_probe(const void* dev_src, size_t bytes, int32_t reps, uint32_t* dev_sink, int32_t n_sink,
+                  void* cuda_stream);
 
 /* -------------------------------------------------------------- misc -- */
 

@@ -87,6 +87,40 @@ def test_static_head_matches_workspace_head_on_consecutive_calls(name, n_lanes, 
     _check(lg2, arg2, ref_logits, ref_arg, sel)
 
 
+def test_static_head_64_rows_and_the_oracle():
+    """The array's full row count (rows 32..63 take the second half of every
+    per-lane slot), checked against the workspace head and, on the same hidden
+    rows, against the fp64 oracle's head."""
+    import oracle as O
+    from oracle import model as M
+    n = 6
+    cfg, sh, h, g_final, packed, scales, ref_logits, ref_arg = _head_inputs("tiny", n, 16, 3)
+    sel = [(7 * i + 3) % n for i in range(64)]
+    h64 = h[sel].contiguous()
+    lg, arg = _call_static(cfg, sh, h64, g_final, packed, scales)
+    _check(lg, arg, ref_logits, ref_arg, sel)
+    W = O.build_weights(sh, S.master_weights(sh), S.gains(sh, 7))
+    want = M.head_logits(W, h64.cpu().numpy().astype(np.float64))
+    for r in range(64):
+        assert_logits_close(lg[r], want[r], f"row {r} vs oracle")
+        s_ = np.sort(want[r])
+        if s_[-1] - s_[-2] > 1e-3:
+            assert int(arg[r]) == int(np.argmax(want[r])), r
+
+
+def test_static_head_rejects_misaligned_head_pointer():
+    import torch
+    from dynamic_depth_b200 import lib
+    x = torch.zeros((2, 128), dtype=torch.float32, device="cuda")
+    g = torch.ones(128, dtype=torch.float32, device="cuda")
+    q = torch.zeros(512 * 64 + 16, dtype=torch.uint8, device="cuda")
+    s = torch.zeros((512, 4), dtype=torch.int16, device="cuda")
+    a = torch.zeros(2, dtype=torch.int32, device="cuda")
+    st = lib().tl_head_argmax_static(x.data_ptr(), 2, g.data_ptr(), C.c_float(1e-5), q.data_ptr() + 8, s.data_ptr(),
+                                     512, 128, 32, None, a.data_ptr(), None)
+    assert st == -1  # TL_EINVAL, nothing enqueued
+
+
 def test_static_head_rejects_sizes_beyond_its_array():
     import torch
     from dynamic_depth_b200 import lib
@@ -98,3 +132,16 @@ def test_static_head_rejects_sizes_beyond_its_array():
     st = lib().tl_head_argmax_static(x.data_ptr(), 65, g.data_ptr(), C.c_float(1e-5), q.data_ptr(), s.data_ptr(),
                                      512, 128, 32, None, a.data_ptr(), None)
     assert st == -2  # TL_ENOMEM: more rows than the static array holds
+
+    # a width beyond 4096 and a vocabulary beyond 262144 rows
+    d = 4128
+    x = torch.zeros((2, d), dtype=torch.float32, device="cuda")
+    g = torch.ones(d, dtype=torch.float32, device="cuda")
+    q = torch.zeros((512, d // 2), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((512, d // 32), dtype=torch.int16, device="cuda")
+    st = lib().tl_head_argmax_static(x.data_ptr(), 2, g.data_ptr(), C.c_float(1e-5), q.data_ptr(), s.data_ptr(),
+                                     512, d, 32, None, a.data_ptr(), None)
+    assert st == -2
+    st = lib().tl_head_argmax_static(x.data_ptr(), 2, g.data_ptr(), C.c_float(1e-5), q.data_ptr(), s.data_ptr(),
+                                     262145, 128, 32, None, a.data_ptr(), None)
+    assert st == -2
