@@ -107,6 +107,9 @@ class LoopedLM:
     def set_early_exit(self, tau: float, min_L: int = 2, patience: int = 0, peek_every: int = 1):
         check(lib().tl_set_early_exit(self.h, float(tau), min_L, patience, peek_every), "tl_set_early_exit")
 
+    def set_l_warmup(self, warmup_tokens: int, warmup_L: int = 2):
+        check(lib().tl_set_l_warmup(self.h, warmup_tokens, warmup_L), "tl_set_l_warmup")
+
     def loop_step(self, per_lane_L=None, active_mask=None, exit_mask_out=None):
         check(lib().tl_loop_step(self.h, _ptr(per_lane_L), _ptr(active_mask), _ptr(exit_mask_out)),
               "tl_loop_step")

@@ -37,7 +37,18 @@ struct LaneState {
   int32_t n_target;   // tokens to emit
   int32_t token;      // last token fed (or emitted)
   int32_t entered;    // set when the lane just took a token and still needs its pre blocks
+  int32_t taken;      // tokens taken after the prompt: the token being computed is number `taken` (0 = prompt)
 };
+
+// L warmup ("Dynamic-L Inference", L scheduling; "CLI Reference",
+// --l-warmup-tokens / --l-warmup-L): decode tokens 1..tokens run min(L, L_req)
+// iterations and leave the cap alone; tokens == 0 disables it.
+struct WarmParams {
+  int32_t tokens;
+  int32_t L;
+};
+
+__device__ __forceinline__ bool warm_token(const WarmParams& w, int t) { return t >= 1 && t <= w.tokens; }
 
 // Early-exit parameters, copied by value into kernels.
 struct EEParams {

@@ -563,202 +563,6 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
   }
 }
 
-// ------------------------------------------------------------- attention ----
-//
-// o[r][h] = softmax(q k^T / sqrt(hd)) v over positions 0..pos of the row's
-// (lane, slot) cache, with RoPE and the KV append of the row's own position
-// folded in: every CTA rotates its head's query from the projection output
-// (qkv, [rows][3d]), and the CTA of the last split, whose key range holds
-// position pos, first rotates and stores that position's key and value, then
-// reads them back with the rest of its range (ordered by __syncthreads within
-// the CTA; no other CTA reads that position).  One CTA of 4 warps per
-// (row, head, split): the key
-// blocks of 32 positions are divided into S contiguous ranges, S chosen on the
-// device from the live row count so that few rows still spread over the SMs
-// (S <= gridDim.z).  Inside a CTA warp w takes blocks w, w+4, ...: one key per
-// lane for the scores, then every lane owns hd/32 output dimensions for the
-// value sum (all 32 value loads of a block issued together); running max and
-// sum are merged across warps, and across splits by the last CTA of the
-// (row, head) to finish, in split order.  Requires kv_page_tokens >= 32.
-// Working CTAs the context split aims for: four per SM on 148 SMs (a
-// larger target, 12 per SM, split the 64-row case in two and measured
-// slower: the split partials and their combine cost more than the waves save).
-constexpr int kAttnCtaTarget = 4 * 148;
-
-template <int HD>
-__global__ void __launch_bounds__(128)
-attn_decode_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
-                   KVGeom g, const float2* __restrict__ rope_cs, int slot_base, int slot_stride,
-                   float* __restrict__ part, int32_t* __restrict__ counters, int32_t* __restrict__ status) {
-  pdl_launch_dependents();
-  pdl_wait();
-  constexpr int DPL = HD / 32;  // output dims per lane
-  __shared__ float qs[HD];
-  __shared__ float wm[4], wl[4];
-  __shared__ float wacc[4][HD];
-  __shared__ int last_s;
-  const int r = blockIdx.x, h = blockIdx.y, z = blockIdx.z;
-  const int n = rows.n[0];
-  if (r >= n) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int d = g.H * HD;
-  const int pos = rows.pos[r];
-  const int ln = rows.lane[r];
-  const int slot = slot_base + rows.iter[r] * slot_stride;
-  const int ctx = pos + 1;
-  const int nblk = (ctx + 31) / 32;
-  int S = (kAttnCtaTarget + n * g.H - 1) / (n * g.H);
-  S = min(min(S, (int)gridDim.z), nblk);
-  if (z >= S) return;
-  const int b0 = (z * nblk) / S, b1 = ((z + 1) * nblk) / S;
-  const float scale = rsqrtf((float)HD);
-  {
-    constexpr int HALF = HD / 2;
-    const float* src = qkv + (int64_t)r * 3 * d + h * HD;
-    const int i = threadIdx.x;
-    if (i < HALF) {
-      const float2 cs = rope_cs[(int64_t)pos * HALF + i];
-      const float q0 = src[i], q1 = src[i + HALF];
-      qs[i] = (q0 * cs.x - q1 * cs.y) * scale;
-      qs[i + HALF] = (q1 * cs.x + q0 * cs.y) * scale;
-      if (z == S - 1) {  // this split's range ends at pos: append the row's key and value
-        __half* kp = kv_k_ptr(g, ln, slot, pos, h, status);
-        if (kp) {
-          __half* vp = kp + (int64_t)g.H * g.page_tokens * HD;
-          const float k0 = src[d + i], k1 = src[d + i + HALF];
-          kp[i] = __float2half_rn(k0 * cs.x - k1 * cs.y);
-          kp[i + HALF] = __float2half_rn(k1 * cs.x + k0 * cs.y);
-          vp[i] = __float2half_rn(src[2 * d + i]);
-          vp[i + HALF] = __float2half_rn(src[2 * d + i + HALF]);
-        }
-      }
-    }
-  }
-  __syncthreads();
-  float m = -INFINITY, l = 0.f, acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  for (int kb = b0 + warp; kb < b1; kb += 4) {
-    const __half* kbase = kv_k_ptr(g, ln, slot, kb * 32, h, status);
-    if (!kbase) break;
-    const __half* vbase = kbase + (int64_t)g.H * g.page_tokens * HD;
-    const int j = kb * 32 + lane;
-    const int nk = min(32, ctx - kb * 32);
-    // the block's values, loaded together with its keys (neither depends on the scores)
-    constexpr int VW = DPL >= 2 ? DPL / 2 : 1;  // 32-bit words of values per lane per key
-    uint32_t vraw[32][VW];
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      if (jj < nk) {
-        if constexpr (DPL >= 2) {
-#pragma unroll
-          for (int e = 0; e < VW; ++e)
-            vraw[jj][e] = reinterpret_cast<const uint32_t*>(vbase + (int64_t)jj * HD + lane * DPL)[e];
-        } else {
-          vraw[jj][0] = __half_as_ushort(vbase[(int64_t)jj * HD + lane]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < VW; ++e) vraw[jj][e] = 0u;
-      }
-    }
-    float s = -INFINITY;
-    if (j < ctx) {
-      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (int64_t)lane * HD);
-      uint4 kv[HD / 8];
-#pragma unroll
-      for (int c = 0; c < HD / 8; ++c) kv[c] = kr[c];
-      float dot = 0.f;
-#pragma unroll
-      for (int c = 0; c < HD / 8; ++c) {
-        const __half2* hv = reinterpret_cast<const __half2*>(&kv[c]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(hv[e]);
-          dot = fmaf(qs[8 * c + 2 * e], f.x, dot);
-          dot = fmaf(qs[8 * c + 2 * e + 1], f.y, dot);
-        }
-      }
-      s = dot;
-    }
-    const float mb = warp_max(s);
-    const float mn = fmaxf(m, mb);
-    const float p = (j < ctx) ? expf(s - mn) : 0.f;
-    const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
-    l = l * corr + warp_sum(p);
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] *= corr;
-    m = mn;
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      const float pj = __shfl_sync(0xffffffffu, p, jj);
-      if constexpr (DPL >= 2) {
-#pragma unroll
-        for (int e = 0; e < VW; ++e) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vraw[jj][e]));
-          acc[2 * e] = fmaf(pj, f.x, acc[2 * e]);
-          acc[2 * e + 1] = fmaf(pj, f.y, acc[2 * e + 1]);
-        }
-      } else {
-        acc[0] = fmaf(pj, __half2float(__ushort_as_half((unsigned short)vraw[jj][0])), acc[0]);
-      }
-    }
-  }
-  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
-  __syncthreads();
-  float M = -INFINITY;
-  for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w]);
-  float Lsum = 0.f;
-  float f[4];
-  for (int w = 0; w < 4; ++w) {
-    f[w] = (wm[w] == -INFINITY) ? 0.f : expf(wm[w] - M);
-    Lsum += wl[w] * f[w];
-  }
-  if (S == 1) {
-    for (int i = threadIdx.x; i < HD; i += blockDim.x) {
-      float v = 0.f;
-      for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
-      o[(int64_t)r * d + h * HD + i] = v / Lsum;
-      o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lsum);
-    }
-    return;
-  }
-  // split partial: (max, sum, unnormalised output) for this key range
-  float* mine = part + (((int64_t)r * g.H + h) * gridDim.z + z) * (HD + 2);
-  for (int i = threadIdx.x; i < HD; i += blockDim.x) {
-    float v = 0.f;
-    for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
-    mine[2 + i] = v;
-  }
-  if (threadIdx.x == 0) { mine[0] = M; mine[1] = Lsum; }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last_s = (atomicAdd(&counters[r * g.H + h], 1) == S - 1);
-  __syncthreads();
-  if (!last_s) return;
-  __threadfence();
-  const float* base = part + ((int64_t)r * g.H + h) * gridDim.z * (HD + 2);
-  float Mx = -INFINITY;
-  for (int zz = 0; zz < S; ++zz) Mx = fmaxf(Mx, __ldcg(base + zz * (HD + 2)));
-  float Lt = 0.f;
-  for (int zz = 0; zz < S; ++zz) {
-    const float mz = __ldcg(base + zz * (HD + 2));
-    Lt += __ldcg(base + zz * (HD + 2) + 1) * ((mz == -INFINITY) ? 0.f : expf(mz - Mx));
-  }
-  for (int i = threadIdx.x; i < HD; i += blockDim.x) {
-    float v = 0.f;
-    for (int zz = 0; zz < S; ++zz) {
-      const float mz = __ldcg(base + zz * (HD + 2));
-      v += __ldcg(base + zz * (HD + 2) + 2 + i) * ((mz == -INFINITY) ? 0.f : expf(mz - Mx));
-    }
-    o[(int64_t)r * d + h * HD + i] = v / Lt;
-    o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lt);
-  }
-  if (threadIdx.x == 0) counters[r * g.H + h] = 0;
-}
-
 // --------------------------------------------------- prefill attention ----
 //
 // Causal attention for blocks of consecutive prompt rows of one lane each: CTA
@@ -916,12 +720,21 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* 
 // peek_every == 0; a probe with delta < tau extends the streak, any other
 // probe resets it; the lane's loop finishes on streak >= patience or when l
 // reaches L_run.  One CTA per row.
+//
+// L warmup: when a warmup token's loop finishes at depth D below the lane's
+// requested L, the K/V it wrote at its position for iteration D (every body
+// layer) are copied into the slots of iterations D+1 .. L_req, so a later,
+// deeper token attends there to the deepest iteration that computed the
+// position (the pages do not say what it should read; this is the reading
+// taken).  Positions are written once, so the copy stays valid.
 __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ h,
                                    const float* __restrict__ h_in, int d, EEParams ee,
-                                   uint8_t* __restrict__ exit_mask_out, unsigned long long* __restrict__ lane_iters) {
+                                   uint8_t* __restrict__ exit_mask_out, unsigned long long* __restrict__ lane_iters,
+                                   WarmParams wp, KVGeom g, int n_pre, int n_loop_layers, int32_t* __restrict__ status) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ double red[32];
+  __shared__ int fill_from, fill_to;
   const int r = blockIdx.x;
   if (r >= rows.n[0]) return;
   const int ln = rows.lane[r];
@@ -940,21 +753,44 @@ __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, con
     num = block_sum_d(num, red);
     den = block_sum_d(den, red);
   }
-  if (threadIdx.x != 0) return;
-  bool ex = false;
-  if (probe) {
-    const bool below = (den > 0.0) && (sqrt(num / den) < ee.tau);
-    st.streak = below ? st.streak + 1 : 0;
-    ex = st.streak >= ee.patience;
+  if (threadIdx.x == 0) {
+    bool ex = false;
+    if (probe) {
+      const bool below = (den > 0.0) && (sqrt(num / den) < ee.tau);
+      st.streak = below ? st.streak + 1 : 0;
+      ex = st.streak >= ee.patience;
+    }
+    st.iter = l;
+    const bool fin = ex || l >= st.L_run;
+    if (fin) {
+      st.phase = PH_BOUNDARY;
+      st.depth = l;
+    }
+    if (exit_mask_out) exit_mask_out[ln] = fin ? 1 : 0;
+    if (lane_iters) atomicAdd(lane_iters, 1ull);
+    fill_from = (fin && warm_token(wp, st.taken) && l < st.L_req) ? l : 0;
+    fill_to = st.L_req;
   }
-  st.iter = l;
-  const bool fin = ex || l >= st.L_run;
-  if (fin) {
-    st.phase = PH_BOUNDARY;
-    st.depth = l;
+  __syncthreads();
+  if (fill_from == 0) return;
+  // copy K and V of this position from iteration fill_from into iterations fill_from+1 .. fill_to
+  const int pos = rows.pos[r];
+  const int hd = g.hd, per_head = 2 * hd;  // K then V elements of one head
+  const int per_slot = g.H * per_head;
+  const int total = (fill_to - fill_from) * n_loop_layers * per_slot;
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int e = i % per_slot, q = i / per_slot;
+    const int m = q % n_loop_layers, it = fill_from + 1 + q / n_loop_layers;
+    const int hh = e / per_head, k = e % per_head;
+    const int src_slot = n_pre + (fill_from - 1) * n_loop_layers + m;
+    const int dst_slot = n_pre + (it - 1) * n_loop_layers + m;
+    const __half* sp = kv_k_ptr(g, ln, src_slot, pos, hh, status);
+    __half* dp = kv_k_ptr(g, ln, dst_slot, pos, hh, status);
+    if (!sp || !dp) continue;
+    const int64_t v_off = (int64_t)g.H * g.page_tokens * hd;  // V row of the same head and position
+    if (k < hd) dp[k] = sp[k];
+    else dp[v_off + k - hd] = sp[v_off + k - hd];
   }
-  if (exit_mask_out) exit_mask_out[ln] = fin ? 1 : 0;
-  if (lane_iters) atomicAdd(lane_iters, 1ull);
 }
 
 // ------------------------------------------------------------- boundary ----
@@ -973,7 +809,7 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
                                      int32_t* __restrict__ argmax_out, int32_t* __restrict__ tokens_out,
                                      int32_t* __restrict__ depths_out, int n_new, MatView E, float* __restrict__ h,
                                      int d, int max_seq, int32_t mark_entered, int32_t* __restrict__ status,
-                                     unsigned long long* __restrict__ tok_count) {
+                                     unsigned long long* __restrict__ tok_count, WarmParams wp) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float sv[32];
@@ -1018,8 +854,9 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
         set_status(status, ST_BAD_POS);
         st.phase = PH_DONE;
       } else {
-        st.L_cap = st.depth;
-        st.L_run = min(st.L_req, st.L_cap);
+        if (!warm_token(wp, st.taken)) st.L_cap = st.depth;  // a warmup token's depth does not lower the cap
+        st.taken += 1;
+        st.L_run = warm_token(wp, st.taken) ? min(wp.L, st.L_req) : min(st.L_req, st.L_cap);
         st.pos += 1;
         st.iter = 0;
         st.streak = 0;
@@ -1037,7 +874,7 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
 // Teacher-forced token entry for masked lanes (see tl_embed_next).  One CTA per lane.
 __global__ void embed_next_kernel(LaneState* __restrict__ lanes, int n_lanes, const uint8_t* __restrict__ mask,
                                   const int32_t* __restrict__ tokens, MatView E, float* __restrict__ h, int d,
-                                  int max_seq, int32_t* __restrict__ status) {
+                                  int max_seq, int32_t* __restrict__ status, WarmParams wp) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ int tok_s, go_s;
@@ -1052,8 +889,9 @@ __global__ void embed_next_kernel(LaneState* __restrict__ lanes, int n_lanes, co
       if (st.pos + 1 >= max_seq) {
         set_status(status, ST_BAD_POS);
       } else {
-        st.L_cap = st.depth;
-        st.L_run = min(st.L_req, st.L_cap);
+        if (!warm_token(wp, st.taken)) st.L_cap = st.depth;
+        st.taken += 1;
+        st.L_run = warm_token(wp, st.taken) ? min(wp.L, st.L_req) : min(st.L_req, st.L_cap);
         st.pos += 1;
         st.iter = 0;
         st.streak = 0;
@@ -1113,6 +951,7 @@ __global__ void prefill_finish_batch_kernel(LaneState* __restrict__ lanes, const
     st.n_target = 0;
     st.token = -1;
     st.entered = 0;
+    st.taken = 0;
   }
 }
 

@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "host_util.h"
+#include "attn_decode.cuh"
 #include "gemv_stream.cuh"
 #include "kernels.cuh"
 #include "tc_gemm.cuh"
@@ -55,6 +56,11 @@ static bool cfg_valid(const tl_config* c) {
   if (c->kv_page_tokens < 32 || (c->kv_page_tokens & (c->kv_page_tokens - 1))) return false;
   if (c->kv_pool_pages < 0 || c->max_prefill_tokens < 0) return false;
   return true;
+}
+
+// TMA row coordinates into the KV pool are 32-bit signed.
+static bool kv_rows_ok(const tl_config* c, int64_t n_pages) {
+  return n_pages * 2 * c->n_heads * (int64_t)c->kv_page_tokens < (int64_t(1) << 31);
 }
 
 static size_t mat_bytes(const tl_config* c, int fmt, int64_t N, int64_t K) {
@@ -99,7 +105,6 @@ enum ProjPath { PATH_AUTO = 0, PATH_GEMV = 1, PATH_TC = 2 };
 // head GEMV: output features per warp (its registers hold that many raw chunks
 // and 8 row accumulators each)
 constexpr int head_rpw(int fmt) { return fmt == TL_FMT_INT4 ? 4 : 2; }
-constexpr int kAttnSplits = 8;   // largest split of the context in decode attention
 
 static int tc_nt(int max_rows) { return max_rows <= 64 ? 64 : (max_rows <= 128 ? 128 : 256); }
 
@@ -212,7 +217,7 @@ static Layout make_layout(const tl_config* c) {
   L.act_a16 = take(R * d * 2);
   L.act_o16 = take(R * d * 2);
   L.act_u16 = take(R * F * 2);
-  L.attn_part = take(lanes * c->n_heads * kAttnSplits * (hd + 2) * 4);
+  L.attn_part = take(lanes * c->n_heads * kAttnPieces * (hd + 2) * 4);
   L.attn_counters = take(lanes * c->n_heads * 4);
   L.part_val = take(lanes * L.n_parts * 4);
   L.part_idx = take(lanes * L.n_parts * 4);
@@ -274,9 +279,11 @@ struct tl_ctx {
   unsigned long long* counters;  // 0 lane iterations, 1 tokens, 2 kernels run inside conditional graph bodies
   int32_t* body_kernels;          // [stage][variant] kernels of each conditional body (graph ticks)
   EEParams ee{0.0, 2, 0, 1, 0};
+  WarmParams warm{0, 2};
   int n_sms = 148;
   int head_parts = 0;  // partial results per row written by the head projection
   CUtensorMap mhead;   // TMA map of the head's raw weight tiles
+  CUtensorMap kvmap;   // TMA map of the KV pool: rows of hd fp16, tiles of kAttnUK rows (swizzled)
   int32_t* head_nparts;  // device: partial count written by whichever head kernel ran
   // CUDA graph of one decode tick (captured on cap_stream, replayed on stream)
   cudaStream_t cap_stream = nullptr, cap_body = nullptr;
@@ -284,6 +291,7 @@ struct tl_ctx {
   int tick_lanes = 0, tick_new = 0;
   int32_t *tick_tok = nullptr, *tick_dep = nullptr;
   EEParams tick_ee{};
+  WarmParams tick_warm{};
   int64_t tick_launches = 0;
   bool graphs_enabled = true;
   bool pdl = true;  // programmatic dependent launch between consecutive kernels
@@ -566,18 +574,30 @@ int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int3
   return prof_stop(c, prof_kind);
 }
 
-int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
-  TL_TRY(prof_start(c, TL_PROF_ATTN));
-  // splits beyond what max_rows * heads needs to fill the GPU are never used
-  int ks = (kAttnCtaTarget + max_rows * c->cfg.n_heads - 1) / (max_rows * c->cfg.n_heads);
-  ks = ks < 1 ? 1 : (ks > kAttnSplits ? kAttnSplits : ks);
-  if (max_rows > 1) ks = kAttnSplits < 4 ? kAttnSplits : (ks < 4 ? 4 : ks);
-  dim3 grid(max_rows, c->cfg.n_heads, ks);
-  switch (c->hd) {
-    case 32: TL_TRY(launch_k(c, attn_decode_kernel<32>, dim3(grid), dim3(128), 0, c->act_qkv, c->act_o, c->act_o16, rows, c->kv, c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
-    case 64: TL_TRY(launch_k(c, attn_decode_kernel<64>, dim3(grid), dim3(128), 0, c->act_qkv, c->act_o, c->act_o16, rows, c->kv, c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
-    default: TL_TRY(launch_k(c, attn_decode_kernel<128>, dim3(grid), dim3(128), 0, c->act_qkv, c->act_o, c->act_o16, rows, c->kv, c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status)); break;
+template <int HD>
+int attn_launch_t(tl_ctx* c, const Rows& rows, int slot_base, int slot_stride) {
+  auto kern = attn_decode_kernel<HD>;
+  const int smem = attn_smem_bytes<HD>(c->cfg.max_lanes);
+  static int attr_smem[64] = {0};  // per instantiation and device: largest opt-in requested so far
+  const int dev = current_device();
+  if (smem > attr_smem[dev]) {
+    TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_smem[dev] = smem;
   }
+  return launch_k(c, kern, dim3(c->n_sms), dim3(AttnCfg<HD>::WARPS * 32), (size_t)smem, c->kvmap,
+                  (const float*)c->act_qkv, c->act_o, c->act_o16, rows, c->kv, (const float2*)c->rope, slot_base,
+                  slot_stride, c->attn_part, c->attn_counters, c->status);
+}
+
+// Decode attention (one query row per (row, head)) over the rows of `rows`.
+int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
+  (void)max_rows;
+  TL_TRY(prof_start(c, TL_PROF_ATTN));
+  int st;
+  if (c->hd == 32) st = attn_launch_t<32>(c, rows, slot_base, slot_stride);
+  else if (c->hd == 64) st = attn_launch_t<64>(c, rows, slot_base, slot_stride);
+  else st = attn_launch_t<128>(c, rows, slot_base, slot_stride);
+  TL_TRY(st);
   return prof_stop(c, TL_PROF_ATTN);
 }
 
@@ -719,8 +739,9 @@ int loop_iteration(tl_ctx* c, int max_rows, uint8_t* exit_mask, int path = PATH_
   for (int m = 0; m < Lb; ++m)
     TL_TRY(run_block(c, R, max_rows, c->h, R.lane, c->loop[m], c->cfg.n_pre + m, Lb, m == 0 ? c->h_in : nullptr,
                      false, path));
-  TL_TRY(launch_k(c, exit_update_kernel, dim3(max_rows), dim3(256), 0, R, c->lanes, c->h, c->h_in, c->cfg.d, c->ee, exit_mask,
-                                                      &c->counters[0]));
+  TL_TRY(launch_k(c, exit_update_kernel, dim3(max_rows), dim3(256), 0, R, c->lanes, (const float*)c->h,
+                  (const float*)c->h_in, c->cfg.d, c->ee, exit_mask, &c->counters[0], c->warm, c->kv, c->cfg.n_pre,
+                  c->cfg.n_loop_layers, c->status));
   c->steps++;
   return TL_OK;
 }
@@ -759,7 +780,8 @@ int head_core(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax,
               use_nrm ? &nrm : nullptr));
   TL_TRY(launch_k(c, head_finalize_kernel, dim3(max_rows), dim3(256), 0, B, c->lanes, c->part_val, c->part_idx, c->head_nparts, mode,
                                                         argmax, tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
-                                                        c->cfg.max_seq, mark_entered, c->status, &c->counters[1]));
+                                                        c->cfg.max_seq, mark_entered, c->status, &c->counters[1],
+                                                        c->warm));
   return TL_OK;
 }
 
@@ -837,6 +859,13 @@ int encode_all_maps(tl_ctx* c) {
       TL_TRY(encode_weight_map(&b.md, b.wd));
     }
   TL_TRY(encode_weight_map(&c->mhead, c->head));
+  {  // KV pool as rows of hd fp16: a page is [K: H x P rows][V: H x P rows]
+    const uint64_t pool_rows = (uint64_t)c->lay.n_pages * 2 * c->cfg.n_heads * c->cfg.kv_page_tokens;
+    const uint32_t cols = c->hd > 64 ? 64 : (uint32_t)c->hd;
+    TL_TRY(encode_2d(&c->kvmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->kv.pool, (uint64_t)c->hd, pool_rows,
+                     (uint64_t)c->hd * 2, cols, (uint32_t)kAttnUK,
+                     cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B));
+  }
   const __half* xs[3] = {c->act_a16, c->act_o16, c->act_u16};
   const int ks[3] = {c->cfg.d, c->cfg.d, c->cfg.ffn};
   const int nts[3] = {64, 128, 256};
@@ -853,7 +882,9 @@ int encode_all_maps(tl_ctx* c) {
 
 extern "C" int tl_workspace_bytes(const tl_config* cfg, size_t* out) {
   if (!cfg_valid(cfg) || !out) return TL_EINVAL;
-  *out = make_layout(cfg).total;
+  const Layout lay = make_layout(cfg);
+  if (!kv_rows_ok(cfg, lay.n_pages)) return TL_EINVAL;
+  *out = lay.total;
   return TL_OK;
 }
 
@@ -906,6 +937,7 @@ __global__ void lanes_init_kernel(LaneState* l, int n) {
 extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void* stream, tl_ctx** out) {
   if (!cfg_valid(cfg) || !dev_ws || !out || ((uintptr_t)dev_ws & 255)) return TL_EINVAL;
   Layout lay = make_layout(cfg);
+  if (!kv_rows_ok(cfg, lay.n_pages)) return TL_EINVAL;
   if (bytes < lay.total) return TL_ENOMEM;
   tl_ctx* c = new tl_ctx();
   c->cfg = *cfg;
@@ -1106,6 +1138,13 @@ extern "C" int tl_set_early_exit(tl_ctx* c, double tau, int32_t min_L, int32_t p
   return TL_OK;
 }
 
+extern "C" int tl_set_l_warmup(tl_ctx* c, int32_t warmup_tokens, int32_t warmup_L) {
+  if (!c || warmup_tokens < 0 || warmup_L < 1) return TL_EINVAL;
+  c->warm.tokens = warmup_tokens;
+  c->warm.L = warmup_L;
+  return TL_OK;
+}
+
 // Prompts of several lanes in one pass over the weights.  Every block runs
 // once on the rows of all lanes (the loop's iteration l on the lanes whose L
 // exceeds l: lanes are ordered by L, deepest first, so those rows are a prefix
@@ -1281,7 +1320,8 @@ extern "C" int tl_embed_next(tl_ctx* c, const uint8_t* dev_mask, const int32_t* 
   if (!c || !dev_tokens) return TL_EINVAL;
   if (!c->loaded) return TL_ESTATE;
   TL_TRY(launch_k(c, embed_next_kernel, dim3(c->cfg.max_lanes), dim3(256), 0, c->lanes, c->cfg.max_lanes, dev_mask, dev_tokens,
-                                                             c->embed, c->h, c->cfg.d, c->cfg.max_seq, c->status));
+                                                             c->embed, c->h, c->cfg.d, c->cfg.max_seq, c->status,
+                                                             c->warm));
   return pre_blocks_for_entered(c, c->cfg.max_lanes);
 }
 
@@ -1401,7 +1441,8 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
 
 static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
   if (c->tick_exec && c->tick_lanes == n_lanes && c->tick_new == n_new && c->tick_tok == tok_out &&
-      c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee))
+      c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee) && c->tick_warm.tokens == c->warm.tokens &&
+      c->tick_warm.L == c->warm.L)
     return TL_OK;
   if (c->tick_exec) {
     cudaGraphExecDestroy(c->tick_exec);
@@ -1434,6 +1475,7 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   c->tick_tok = tok_out;
   c->tick_dep = dep_out;
   c->tick_ee = c->ee;
+  c->tick_warm = c->warm;
   c->tick_launches = 1;  // the planning kernel outside the conditional bodies
   return TL_OK;
 }

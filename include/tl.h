@@ -220,6 +220,20 @@ int tl_prefill_batch(tl_ctx* ctx, int32_t n, const int32_t* lanes, const int32_t
  * tau <= 0 or patience == 0 disables it.  peek_every >= 1. */
 int tl_set_early_exit(tl_ctx* ctx, double tau, int32_t min_L, int32_t patience, int32_t peek_every);
 
+/* L warmup for all lanes ("Dynamic-L Inference", L scheduling: the first N
+ * tokens at a shallow depth, the rest at full depth; "CLI Reference",
+ * --l-warmup-tokens / --l-warmup-L): decode tokens 1..warmup_tokens after the
+ * prompt's token run min(warmup_L, L requested) iterations (early exit may
+ * stop them sooner) and do not lower the lane's cap; later tokens run min(L
+ * requested, cap) as usual.  A later token's deeper iteration l, at a
+ * position that a warmup token computed only to depth D < l, attends to that
+ * position's K/V of iteration D (the deepest iteration holding it; the pages
+ * do not say, this is the reading taken): when a warmup token's loop ends,
+ * its K/V are copied into the slots of the iterations above D.  warmup_tokens
+ * = 0 disables it (the default).  Takes effect for tokens entered afterwards.
+ * TL_EINVAL for warmup_tokens < 0 or warmup_L < 1. */
+int tl_set_l_warmup(tl_ctx* ctx, int32_t warmup_tokens, int32_t warmup_L);
+
 /* One loop step: every lane with dev_active_mask[lane] != 0 that is in its
  * loop phase runs its next loop iteration (all body layers), at its own
  * iteration index; then the device applies the early-exit rule.
@@ -283,7 +297,7 @@ int tl_set_graphs(tl_ctx* ctx, int32_t enabled);
 /* ------------------------------------------------- lane-state checkpoint -- */
 
 /* Bytes of a lane-state snapshot: the scheduling state and the fp32 hidden row
- * of every lane (max_lanes * (48 + 4 d)).  The KV cache is not part of it: a
+ * of every lane (max_lanes * (52 + 4 d)).  The KV cache is not part of it: a
  * decode started from a restored snapshot rewrites every position past the
  * saved ones before reading it, and positions at or before them are never
  * written by decode. */

@@ -53,7 +53,7 @@ def status_clean(m):
     return st
 
 
-def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None, prefill=None):
+def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None, prefill=None, warmup=(0, 2)):
     """Drive the CUDA path with the oracle's tokens (prefill, head, then
     embed_next + loop steps until every lane's loop finished, head again).
     prefill(i, lane) replaces the plain m.prefill of prompt i when given.
@@ -65,7 +65,8 @@ def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None, pr
     ee = ee or D.EarlyExit()
     n = len(prompts)
     lanes = list(range(n)) if lanes is None else lanes
-    ref = [D.generate_lane(W, prompts[i], Ls[i], n_new, ee) for i in range(n)]
+    ref = [D.generate_lane(W, prompts[i], Ls[i], n_new, ee, warmup_tokens=warmup[0], warmup_L=warmup[1])
+           for i in range(n)]
     V = W.shape.vocab
     max_lanes = m.cfg.max_lanes
     dev = m.device
@@ -76,6 +77,7 @@ def teacher_forced(m, W, prompts, Ls, n_new, ee=None, lanes=None, torch=None, pr
     exit_mask = torch.zeros(max_lanes, dtype=torch.uint8, device=dev)
     tok = torch.zeros(max_lanes, dtype=torch.int32, device=dev)
     m.set_early_exit(ee.tau, ee.min_L, ee.patience, ee.peek_every)
+    m.set_l_warmup(warmup[0], warmup[1])
     for i, ln in enumerate(lanes):
         if prefill is None:
             m.prefill(ln, prompts[i], Ls[i])

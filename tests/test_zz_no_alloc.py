@@ -18,7 +18,7 @@ from gpu_helpers import assert_logits_close, gpu_model, status_clean
 
 pytestmark = pytest.mark.gpu
 
-LANE_STATE_BYTES = 12 * 4  # int32 fields of one lane's scheduling state
+LANE_STATE_BYTES = 13 * 4  # int32 fields of one lane's scheduling state
 
 
 def _head_inputs(name, n_lanes, prompt_len, L):
