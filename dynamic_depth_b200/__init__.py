@@ -107,6 +107,10 @@ class LoopedLM:
     def set_early_exit(self, tau: float, min_L: int = 2, patience: int = 0, peek_every: int = 1):
         check(lib().tl_set_early_exit(self.h, float(tau), min_L, patience, peek_every), "tl_set_early_exit")
 
+    def set_early_exit_logit_margin(self, margin: float, min_L: int = 2, patience: int = 1, peek_every: int = 1):
+        check(lib().tl_set_early_exit_logit_margin(self.h, float(margin), min_L, patience, peek_every),
+              "tl_set_early_exit_logit_margin")
+
     def set_l_warmup(self, warmup_tokens: int, warmup_L: int = 2):
         check(lib().tl_set_l_warmup(self.h, warmup_tokens, warmup_L), "tl_set_l_warmup")
 

@@ -50,6 +50,7 @@ SIGNATURES = {
     "tl_prefill_batch": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                    C.c_int32, C.c_int32]),
     "tl_set_early_exit": (C.c_int, [C.c_void_p, C.c_double, C.c_int32, C.c_int32, C.c_int32]),
+    "tl_set_early_exit_logit_margin": (C.c_int, [C.c_void_p, C.c_double, C.c_int32, C.c_int32, C.c_int32]),
     "tl_set_l_warmup": (C.c_int, [C.c_void_p, C.c_int32, C.c_int32]),
     "tl_loop_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "tl_head_logits": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),

@@ -171,10 +171,8 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
   uint64_t* wfull = full + warp * STAGES;
   const int64_t head_rows = (int64_t)g.page_tokens;          // rows of one head's block inside a page
   const int64_t page_rows = (int64_t)2 * H * g.page_tokens;  // K then V
-  // TMA loads of flat unit u into stage s (lane 0 only)
-  auto issue = [&](int u, int s) {
-    int r, h, b;
-    locate(u, r, h, b);
+  // TMA loads of unit (r, h, b) into stage s (lane 0 only)
+  auto issue = [&](int r, int h, int b, int s) {
     const int ln = rows.lane[r];
     const int slot = slot_base + rows.iter[r] * slot_stride;
     const int p0 = b * UK;
@@ -197,16 +195,38 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
       tma_load_2d(smem_u32(st + (C::HALVES + t) * C::TILE_BYTES), &kvmap, t * C::COLS, (int)(y + H * head_rows), fb);
     }
   };
+  // the issue cursor runs ahead of the consumer over the same flat order
+  int ir = 0, ih = 0, ib = 0;
+  locate(u_begin, ir, ih, ib);
+  auto advance = [&](int& rr, int& hh, int& bb) {
+    if (++bb == (ubase[rr + 1] - ubase[rr]) / H) {
+      bb = 0;
+      if (++hh == H) {
+        hh = 0;
+        ++rr;
+      }
+    }
+  };
 
   const int n_units = u_end - u_begin;
   if (lane == 0)
-    for (int i = 0; i < min(STAGES, n_units); ++i) issue(u_begin + i, i);
+    for (int i = 0; i < min(STAGES, n_units); ++i) {
+      issue(ir, ih, ib, i);
+      advance(ir, ih, ib);
+    }
   __syncwarp();
 
-  const float scale = rsqrtf((float)HD);
+  // scores in the log2 domain: q carries log2(e) / sqrt(hd), so exp2 of differences gives the softmax weights
+  const float scale = rsqrtf((float)HD) * 1.4426950408889634f;
   // value-sum role of this lane: 16-byte chunk vc of the value row (tile vt, chunk vcc), key group kg
   const int vc = lane % LPR, kg = lane / LPR;
   const int vt = vc / CPT, vcc = vc % CPT;
+  // this lane's swizzled byte offsets: its key row's chunks (scores) and its value chunk of each key it sums
+  int koff[CPT], voff[UK / G];
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) koff[c] = swz_chunk<C::ROW_BYTES>(lane, c);
+#pragma unroll
+  for (int t = 0; t < UK / G; ++t) voff[t] = swz_chunk<C::ROW_BYTES>(kg + G * t, vcc);
   float q[HD];
   float m = -INFINITY, l = 0.f, acc[8];
   int r = 0, h = 0, b = 0, nu = 1, run_first = 0, ctx = 0, pos = 0, ln = 0;
@@ -292,7 +312,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
       const uint8_t* tile = st + t * C::TILE_BYTES;
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(tile + swz_chunk<C::ROW_BYTES>(lane, c));
+        const uint4 kv = *reinterpret_cast<const uint4*>(tile + koff[c]);
         const __half2* hv = reinterpret_cast<const __half2*>(&kv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -305,21 +325,23 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
     const bool valid = lane < nvalid;
     const float sc = valid ? dot : -INFINITY;
     const float mn = fmaxf(m, warp_max(sc));
-    const float p = valid ? expf(sc - mn) : 0.f;
-    const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
+    const float p = valid ? exp2f(sc - mn) : 0.f;
+    const float corr = (m == -INFINITY) ? 0.f : exp2f(m - mn);
     l = l * corr + warp_sum(p);
     m = mn;
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] *= corr;
     // value sum: keys kg, kg + G, ... of the unit, this lane's 8 dimensions
     {
+      // keys past nvalid have p = 0, but their stale bytes may not be finite: skip them
       const uint8_t* vtile = st + (C::HALVES + vt) * C::TILE_BYTES;
+      const bool full_unit = nvalid == UK;
 #pragma unroll
       for (int t = 0; t < UK / G; ++t) {
         const int j = kg + G * t;
         const float pj = __shfl_sync(0xffffffffu, p, j);
-        if (j < nvalid) {
-          const uint4 vv = *reinterpret_cast<const uint4*>(vtile + swz_chunk<C::ROW_BYTES>(j, vcc));
+        if (full_unit || j < nvalid) {
+          const uint4 vv = *reinterpret_cast<const uint4*>(vtile + voff[t]);
           const __half2* hv = reinterpret_cast<const __half2*>(&vv);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -333,7 +355,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
     // the stage is free: order this warp's reads before the next TMA write into it, then refill
     __syncwarp();
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (lane == 0 && i + STAGES < n_units) issue(u + STAGES, s);
+    if (lane == 0 && i + STAGES < n_units) {
+      issue(ir, ih, ib, s);
+      advance(ir, ih, ib);
+    }
     __syncwarp();
     // end of this warp's run over (r, h): write the output or a piece
     if (b == nu - 1 || i == n_units - 1) {
@@ -385,7 +410,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
           for (int e = 0; e < 8; ++e) outv[e] = 0.f;
           for (int z = 0; z < n_pieces; ++z) {
             const float mz = __ldcg(base + z * (HD + 2));
-            const float f = (mz == -INFINITY) ? 0.f : expf(mz - M);
+            const float f = (mz == -INFINITY) ? 0.f : exp2f(mz - M);
             Lt += __ldcg(base + z * (HD + 2) + 1) * f;
             if (kg == 0) {
 #pragma unroll

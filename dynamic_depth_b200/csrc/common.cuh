@@ -57,7 +57,14 @@ struct EEParams {
   int32_t patience;
   int32_t peek_every;
   int32_t enabled;
+  int32_t use_margin;  // 1: the probe's metric is the head's top-1 minus top-2 logit margin
+  double margin;       // margin mode: a probe succeeds when the margin is at least this
 };
+
+// Whether iteration l (1-based) of a token is a probe of the exit rule.
+__device__ __forceinline__ bool ee_probe(const EEParams& ee, int l) {
+  return ee.enabled && l > ee.min_L && ((l - ee.min_L - 1) % ee.peek_every) == 0;
+}
 
 // Compacted rows of one launch group: row r computes for lane row_lane[r] at
 // position row_pos[r], loop iteration row_iter[r] (0-based).

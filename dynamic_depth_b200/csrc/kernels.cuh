@@ -719,7 +719,10 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* 
 // (sums in fp64); probe at iteration l when l > min_L and (l - min_L - 1) %
 // peek_every == 0; a probe with delta < tau extends the streak, any other
 // probe resets it; the lane's loop finishes on streak >= patience or when l
-// reaches L_run.  One CTA per row.
+// reaches L_run.  In logit-margin mode ("CLI Reference",
+// --early-exit-logit-margin) the probe's metric is margin_lane[lane], the top-1
+// minus top-2 logit of the head at this iteration (margin_kernel), and it
+// succeeds when the margin is at least the threshold.  One CTA per row.
 //
 // L warmup: when a warmup token's loop finishes at depth D below the lane's
 // requested L, the K/V it wrote at its position for iteration D (every body
@@ -730,7 +733,8 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* 
 __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, const float* __restrict__ h,
                                    const float* __restrict__ h_in, int d, EEParams ee,
                                    uint8_t* __restrict__ exit_mask_out, unsigned long long* __restrict__ lane_iters,
-                                   WarmParams wp, KVGeom g, int n_pre, int n_loop_layers, int32_t* __restrict__ status) {
+                                   WarmParams wp, KVGeom g, int n_pre, int n_loop_layers, int32_t* __restrict__ status,
+                                   const float* __restrict__ margin_lane) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ double red[32];
@@ -740,9 +744,9 @@ __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, con
   const int ln = rows.lane[r];
   LaneState& st = lanes[ln];
   const int l = st.iter + 1;
-  const bool probe = ee.enabled && l > ee.min_L && ((l - ee.min_L - 1) % ee.peek_every) == 0;
+  const bool probe = ee_probe(ee, l);
   double num = 0.0, den = 0.0;
-  if (probe) {
+  if (probe && !ee.use_margin) {
     const float* a = h + (int64_t)ln * d;
     const float* b = h_in + (int64_t)ln * d;
     for (int k = threadIdx.x; k < d; k += blockDim.x) {
@@ -756,7 +760,8 @@ __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, con
   if (threadIdx.x == 0) {
     bool ex = false;
     if (probe) {
-      const bool below = (den > 0.0) && (sqrt(num / den) < ee.tau);
+      const bool below = ee.use_margin ? ((double)margin_lane[ln] >= ee.margin)
+                                       : ((den > 0.0) && (sqrt(num / den) < ee.tau));
       st.streak = below ? st.streak + 1 : 0;
       ex = st.streak >= ee.patience;
     }
@@ -790,6 +795,78 @@ __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, con
     const int64_t v_off = (int64_t)g.H * g.page_tokens * hd;  // V row of the same head and position
     if (k < hd) dp[k] = sp[k];
     else dp[v_off + k - hd] = sp[v_off + k - hd];
+  }
+}
+
+// ---------------------------------------------------- logit-margin probe ----
+//
+// Rows of the loop table whose iteration just run (lane's iter + 1) is a probe
+// of the exit rule, compacted in row order into `probe` (one CTA of 1024
+// threads; thread i looks at loop row i).
+__global__ void probe_rows_kernel(Rows loop, const LaneState* __restrict__ lanes, EEParams ee, Rows probe) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ int32_t cnt[32];
+  const int i = threadIdx.x, lane = i & 31, w = i >> 5;
+  const int n = loop.n[0];
+  int take = 0, ln = 0;
+  if (i < n) {
+    ln = loop.lane[i];
+    take = ee_probe(ee, lanes[ln].iter + 1);
+  }
+  const unsigned bal = __ballot_sync(0xffffffffu, take);
+  if (lane == 0) cnt[w] = __popc(bal);
+  __syncthreads();
+  if (w == 0) {
+    int v = cnt[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    cnt[lane] = v;
+  }
+  __syncthreads();
+  if (take) {
+    const int r = (w == 0 ? 0 : cnt[w - 1]) + __popc(bal & ((1u << lane) - 1u));
+    probe.lane[r] = ln;
+    probe.pos[r] = loop.pos[i];
+    probe.iter[r] = loop.iter[i];
+  }
+  if (i == 0) probe.n[0] = cnt[31];
+}
+
+// margin_lane[lane] = top-1 minus top-2 of logits[lane][0..V) for every probe
+// row (equal maxima give 0).  One CTA per row.
+__global__ void margin_kernel(Rows probe, const float* __restrict__ logits, int V, float* __restrict__ margin_lane) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ float s1[32], s2[32];
+  const int r = blockIdx.x;
+  if (r >= probe.n[0]) return;
+  const int ln = probe.lane[r];
+  const float* x = logits + (int64_t)ln * V;
+  float a1 = -INFINITY, a2 = -INFINITY;  // the two largest values seen (a multiset)
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float y = x[v];
+    if (y > a1) { a2 = a1; a1 = y; } else if (y > a2) { a2 = y; }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float b1 = __shfl_xor_sync(0xffffffffu, a1, off), b2 = __shfl_xor_sync(0xffffffffu, a2, off);
+    const float n1 = fmaxf(a1, b1), n2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+    a1 = n1;
+    a2 = n2;
+  }
+  if ((threadIdx.x & 31) == 0) { s1[threadIdx.x >> 5] = a1; s2[threadIdx.x >> 5] = a2; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+      const float n1 = fmaxf(a1, s1[w]), n2 = fmaxf(fminf(a1, s1[w]), fmaxf(a2, s2[w]));
+      a1 = n1;
+      a2 = n2;
+    }
+    margin_lane[ln] = a1 - a2;
   }
 }
 

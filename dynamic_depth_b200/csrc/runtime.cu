@@ -175,9 +175,9 @@ struct Layout {
   int n_slots, pages_per_seq, n_pages, max_rows, n_parts, max_prefill;
   size_t page_elems;
   std::vector<size_t> mat_off;  // per matrix
-  size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[4], act_a, act_qkv, act_q, act_o, act_u,
+  size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[5], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
-      mask_stage, pf_n, pf_tiles, pf_info,
+      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane,
       out_tok, out_dep, status, counters, body_kernels, alive, total;
 };
 
@@ -208,7 +208,7 @@ static Layout make_layout(const tl_config* c) {
   L.h = take(lanes * d * 4);
   L.h_in = take(lanes * d * 4);
   L.hrows = take((size_t)L.max_prefill * d * 4);
-  for (int i = 0; i < 4; ++i) L.rows[i] = take(4 + 3 * R * 4 + 16);
+  for (int i = 0; i < 5; ++i) L.rows[i] = take(4 + 3 * R * 4 + 16);
   L.act_a = take(R * d * 4);
   L.act_qkv = take(R * 3 * d * 4);
   L.act_q = take(R * d * 4);
@@ -227,6 +227,8 @@ static Layout make_layout(const tl_config* c) {
   L.pf_n = take((size_t)(c->L_max + 2) * 4);
   L.pf_tiles = take((R / 64 + lanes + 2) * 8);
   L.pf_info = take(lanes * 16);
+  L.probe_logits = take(lanes * (size_t)c->vocab * 4);
+  L.margin_lane = take(lanes * 4);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
@@ -263,7 +265,9 @@ struct tl_ctx {
   int32_t* page_table;
   LaneState* lanes;
   float *h, *h_in, *hrows;
-  Rows rows[4];  // 0 loop, 1 boundary, 2 entered, 3 prefill / mask
+  Rows rows[5];  // 0 loop, 1 boundary, 2 entered, 3 prefill / mask, 4 logit-margin probes
+  float* probe_logits;  // [lanes][vocab] head logits of the lanes probing in margin mode
+  float* margin_lane;   // [lanes] their top-1 minus top-2 margins
   float *act_a, *act_qkv, *act_q, *act_o, *act_u;
   __half *act_a16, *act_o16, *act_u16;
   float* attn_part;
@@ -278,7 +282,7 @@ struct tl_ctx {
   uint8_t* mask_stage;
   unsigned long long* counters;  // 0 lane iterations, 1 tokens, 2 kernels run inside conditional graph bodies
   int32_t* body_kernels;          // [stage][variant] kernels of each conditional body (graph ticks)
-  EEParams ee{0.0, 2, 0, 1, 0};
+  EEParams ee{0.0, 2, 0, 1, 0, 0, 0.0};
   WarmParams warm{0, 2};
   int n_sms = 148;
   int head_parts = 0;  // partial results per row written by the head projection
@@ -732,6 +736,35 @@ int build_rows(tl_ctx* c, int which, int sel, const uint8_t* mask, const int32_t
   return TL_OK;
 }
 
+// Logit-margin probes ("CLI Reference", --early-exit-logit-margin: a head
+// projection per peek): the loop rows whose iteration is a probe go into
+// rows[4]; the final norm and the head (the boundary stage's kernels) write
+// their logits, and margin_kernel reduces each to its top-1 minus top-2.  The
+// probe count is known only on the device, so unless the loop rows fit the
+// GEMV (then so do the probes) both head variants are launched and the one
+// that does not apply returns at once.
+int probe_head(tl_ctx* c, int max_rows, int path) {
+  const Rows& P = c->rows[4];
+  TL_TRY(launch_k(c, probe_rows_kernel, dim3(1), dim3(1024), 0, c->rows[0], (const LaneState*)c->lanes, c->ee, P));
+  const int ppath = path == PATH_GEMV ? PATH_GEMV : PATH_AUTO;
+  const float* X = nullptr;
+  GsNorm nrm{};
+  bool use_nrm = false;
+  TL_TRY(norm_for_proj(c, max_rows, ppath, P.n, c->h, P.lane, c->g_final, nullptr, c->head, 1, &X, &nrm, &use_nrm));
+  ProjOut o{};
+  o.epi = EPI_ARGMAX;
+  o.logits = c->probe_logits;
+  o.lmap = P.lane;
+  o.ldo = c->cfg.vocab;
+  o.part_val = c->part_val;
+  o.part_idx = c->part_idx;
+  o.n_parts_dev = c->head_nparts;
+  TL_TRY(proj(c, max_rows, ppath, X, 0, P.n, c->head, &c->mhead, nullptr, nullptr, o, nullptr, TL_PROF_HEAD,
+              use_nrm ? &nrm : nullptr));
+  return launch_k(c, margin_kernel, dim3(max_rows), dim3(256), 0, P, (const float*)c->probe_logits, c->cfg.vocab,
+                  c->margin_lane);
+}
+
 // One loop iteration for the lanes selected into rows[0].
 int loop_iteration(tl_ctx* c, int max_rows, uint8_t* exit_mask, int path = PATH_AUTO) {
   const Rows& R = c->rows[0];
@@ -739,9 +772,10 @@ int loop_iteration(tl_ctx* c, int max_rows, uint8_t* exit_mask, int path = PATH_
   for (int m = 0; m < Lb; ++m)
     TL_TRY(run_block(c, R, max_rows, c->h, R.lane, c->loop[m], c->cfg.n_pre + m, Lb, m == 0 ? c->h_in : nullptr,
                      false, path));
+  if (c->ee.enabled && c->ee.use_margin) TL_TRY(probe_head(c, max_rows, path));
   TL_TRY(launch_k(c, exit_update_kernel, dim3(max_rows), dim3(256), 0, R, c->lanes, (const float*)c->h,
                   (const float*)c->h_in, c->cfg.d, c->ee, exit_mask, &c->counters[0], c->warm, c->kv, c->cfg.n_pre,
-                  c->cfg.n_loop_layers, c->status));
+                  c->cfg.n_loop_layers, c->status, (const float*)c->margin_lane));
   c->steps++;
   return TL_OK;
 }
@@ -994,7 +1028,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->h = (float*)(w + lay.h);
   c->h_in = (float*)(w + lay.h_in);
   c->hrows = (float*)(w + lay.hrows);
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 5; ++i) {
     int32_t* base = (int32_t*)(w + lay.rows[i]);
     c->rows[i].n = base;
     c->rows[i].lane = base + 4;
@@ -1018,6 +1052,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->pf_n = (int32_t*)(w + lay.pf_n);
   c->pf_tiles = (int2*)(w + lay.pf_tiles);
   c->pf_info = (int32_t*)(w + lay.pf_info);
+  c->probe_logits = (float*)(w + lay.probe_logits);
+  c->margin_lane = (float*)(w + lay.margin_lane);
   c->mask_stage = (uint8_t*)(w + lay.mask_stage);
   c->out_tok = (int32_t*)(w + lay.out_tok);
   c->out_dep = (int32_t*)(w + lay.out_dep);
@@ -1056,7 +1092,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     if ((st = check_cuda(cudaMemsetAsync(c->counters, 0, 32, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->attn_counters, 0, (size_t)cfg->max_lanes * cfg->n_heads * 4, c->stream))) != TL_OK) break;
     if ((st = encode_all_maps(c)) != TL_OK) break;
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 5; ++i)
       if ((st = check_cuda(cudaMemsetAsync(c->rows[i].n, 0, 4, c->stream))) != TL_OK) break;
     if (st != TL_OK) break;
     if ((st = check_cuda(cudaHostAlloc((void**)&c->pinned_alive, kAliveRing * sizeof(int32_t), cudaHostAllocDefault))) != TL_OK) break;
@@ -1135,6 +1171,21 @@ extern "C" int tl_set_early_exit(tl_ctx* c, double tau, int32_t min_L, int32_t p
   c->ee.patience = patience;
   c->ee.peek_every = peek_every;
   c->ee.enabled = (tau > 0.0 && patience > 0) ? 1 : 0;
+  c->ee.use_margin = 0;
+  c->ee.margin = 0.0;
+  return TL_OK;
+}
+
+extern "C" int tl_set_early_exit_logit_margin(tl_ctx* c, double margin, int32_t min_L, int32_t patience,
+                                              int32_t peek_every) {
+  if (!c || peek_every < 1 || min_L < 0 || patience < 0) return TL_EINVAL;
+  c->ee.tau = 0.0;
+  c->ee.min_L = min_L;
+  c->ee.patience = patience;
+  c->ee.peek_every = peek_every;
+  c->ee.enabled = (margin > 0.0 && patience > 0) ? 1 : 0;
+  c->ee.use_margin = 1;
+  c->ee.margin = margin;
   return TL_OK;
 }
 
@@ -1345,7 +1396,7 @@ static int enqueue_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
 
 static bool same_ee(const EEParams& a, const EEParams& b) {
   return a.tau == b.tau && a.min_L == b.min_L && a.patience == b.patience && a.peek_every == b.peek_every &&
-         a.enabled == b.enabled;
+         a.enabled == b.enabled && a.use_margin == b.use_margin && a.margin == b.margin;
 }
 
 // Conditional node after the current position of the capture on `s`.

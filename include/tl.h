@@ -217,8 +217,22 @@ int tl_prefill_batch(tl_ctx* ctx, int32_t n, const int32_t* lanes, const int32_t
  * probe at iteration l when l > min_L and (l - min_L - 1) % peek_every == 0;
  * a probe with delta = ||h_l - h_{l-1}|| / ||h_{l-1}|| < tau extends the
  * streak, any other probe resets it; exit once streak >= patience.
- * tau <= 0 or patience == 0 disables it.  peek_every >= 1. */
+ * tau <= 0 or patience == 0 disables it.  peek_every >= 1.  Replaces the
+ * logit-margin mode. */
 int tl_set_early_exit(tl_ctx* ctx, double tau, int32_t min_L, int32_t patience, int32_t peek_every);
+
+/* Logit-margin early exit for all lanes ("CLI Reference",
+ * --early-exit-logit-margin, and its "Current Behavior" note that this is the
+ * mode that fires): the same probe schedule, streak and patience as
+ * tl_set_early_exit, but a probe's metric is the head's top-1 minus top-2
+ * logit (final RMSNorm and head projection of the lane's hidden state at that
+ * iteration, a full head pass per probe) and the probe succeeds when the
+ * margin is at least `margin` (the pages say the loop stops when the model is
+ * confidently predicting one token; "at least the threshold" is the reading
+ * taken).  Replaces the hidden-state mode; margin <= 0 or patience == 0
+ * disables early exit.  peek_every >= 1. */
+int tl_set_early_exit_logit_margin(tl_ctx* ctx, double margin, int32_t min_L, int32_t patience,
+                                   int32_t peek_every);
 
 /* L warmup for all lanes ("Dynamic-L Inference", L scheduling: the first N
  * tokens at a shallow depth, the rest at full depth; "CLI Reference",
