@@ -140,6 +140,14 @@ class LoopedLM:
               "tl_generate")
         return tok, dep
 
+    def speculate(self, lane: int, n_new: int, L_draft: int, L_verify: int, draft_ahead: int):
+        """Self-speculative greedy decode of a freshly prefilled lane: (tokens int32 [n_new], verify rounds)."""
+        tok = np.zeros(n_new, np.int32)
+        rounds = C.c_int32(0)
+        check(lib().tl_speculate(self.h, lane, n_new, L_draft, L_verify, draft_ahead, tok.ctypes.data,
+                                 C.byref(rounds)), "tl_speculate")
+        return tok, rounds.value
+
     def set_graphs(self, enabled: bool):
         check(lib().tl_set_graphs(self.h, 1 if enabled else 0), "tl_set_graphs")
 

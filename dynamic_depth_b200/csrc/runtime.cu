@@ -177,7 +177,7 @@ struct Layout {
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[5], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
-      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane,
+      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec,
       out_tok, out_dep, status, counters, body_kernels, alive, total;
 };
 
@@ -229,6 +229,7 @@ static Layout make_layout(const tl_config* c) {
   L.pf_info = take(lanes * 16);
   L.probe_logits = take(lanes * (size_t)c->vocab * 4);
   L.margin_lane = take(lanes * 4);
+  L.spec = take((lanes + 3 * L.max_prefill + 8) * 4);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
@@ -268,6 +269,7 @@ struct tl_ctx {
   Rows rows[5];  // 0 loop, 1 boundary, 2 entered, 3 prefill / mask, 4 logit-margin probes
   float* probe_logits;  // [lanes][vocab] head logits of the lanes probing in margin mode
   float* margin_lane;   // [lanes] their top-1 minus top-2 margins
+  int32_t* spec;        // speculation: [lanes] token per lane, then drafted, verify-input and verify tokens
   float *act_a, *act_qkv, *act_q, *act_o, *act_u;
   __half *act_a16, *act_o16, *act_u16;
   float* attn_part;
@@ -1054,6 +1056,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->pf_info = (int32_t*)(w + lay.pf_info);
   c->probe_logits = (float*)(w + lay.probe_logits);
   c->margin_lane = (float*)(w + lay.margin_lane);
+  c->spec = (int32_t*)(w + lay.spec);
   c->mask_stage = (uint8_t*)(w + lay.mask_stage);
   c->out_tok = (int32_t*)(w + lay.out_tok);
   c->out_dep = (int32_t*)(w + lay.out_dep);
@@ -1351,6 +1354,167 @@ extern "C" int tl_prefill_batch(tl_ctx* c, int32_t n, const int32_t* lanes, cons
     off += (size_t)T[i];
   }
   return prefill_impl(c, in, share_from, shared_tokens, nullptr);
+}
+
+// ------------------------------------------------------ self-speculation ----
+
+// Positions pos0 .. pos0 + k - 1 of one lane (their tokens already in
+// c->tok_stage) through embed, the pre blocks and L loop iterations as one
+// causal batch over the lane's own pages (the cache of earlier positions is
+// read, these positions' K/V rewritten for every slot they reach); the final
+// hidden rows are left in c->hrows.  The lane state is not touched.
+static int rerun_positions(tl_ctx* c, int lane, int pos0, int k, int L) {
+  const tl_config& cfg = c->cfg;
+  const int P = cfg.n_pre, Lb = cfg.n_loop_layers;
+  std::vector<int32_t> r_lane(k, lane), r_pos(k), r_iter(k, 0), stage_rows(L + 1, k);
+  stage_rows[L] = 0;
+  for (int i = 0; i < k; ++i) r_pos[i] = pos0 + i;
+  std::vector<int2> tiles;
+  for (int t0 = 0; t0 < k; t0 += 64) tiles.push_back(make_int2(t0, k - t0 < 64 ? k - t0 : 64));
+  const Rows& R = c->rows[3];
+  TL_CUDA(cudaMemcpyAsync(R.lane, r_lane.data(), k * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(R.pos, r_pos.data(), k * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(R.iter, r_iter.data(), k * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->pf_tiles, tiles.data(), tiles.size() * sizeof(int2), cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(c->pf_n, stage_rows.data(), (L + 1) * 4, cudaMemcpyHostToDevice, c->stream));
+  Rows Rs = R;
+  Rs.n = c->pf_n;
+  const int nt = (int)tiles.size();
+  TL_TRY(launch_k(c, embed_rows_kernel, dim3(k), dim3(256), 0, c->embed, (const int32_t*)c->tok_stage, k, cfg.d,
+                  c->hrows, c->status));
+  PendingAdd pend;
+  for (int b = 0; b < P; ++b)
+    TL_TRY(run_block(c, Rs, k, c->hrows, nullptr, c->pre[b], b, 0, nullptr, true, PATH_AUTO, c->pf_tiles, nt, &pend));
+  for (int l = 0; l < L; ++l) {
+    Rs.n = c->pf_n + l;
+    for (int m = 0; m < Lb; ++m)
+      TL_TRY(run_block(c, Rs, k, c->hrows, nullptr, c->loop[m], P + l * Lb + m, 0, nullptr, true, PATH_AUTO,
+                       c->pf_tiles, nt, &pend));
+  }
+  if (pend.add)
+    TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(pend.rows), dim3(256), 0, c->hrows, (const int32_t*)nullptr,
+                    (const int32_t*)(c->pf_n + L), cfg.d, (const float*)nullptr, cfg.rms_eps, (float*)nullptr,
+                    (float*)nullptr, (__half*)nullptr, (float*)nullptr, 0, 0, pend.add, pend.n));
+  c->prefill_tokens += k;
+  return TL_OK;
+}
+
+// Greedy head over hidden rows 0 .. k - 1 of c->hrows: dev_argmax[r] for each row.
+static int head_hrows(tl_ctx* c, int k, int32_t* dev_argmax) {
+  const Rows& T4 = c->rows[4];
+  std::vector<int32_t> ident(k);
+  for (int i = 0; i < k; ++i) ident[i] = i;
+  TL_CUDA(cudaMemcpyAsync(T4.lane, ident.data(), k * 4, cudaMemcpyHostToDevice, c->stream));
+  TL_CUDA(cudaMemcpyAsync(T4.n, &k, 4, cudaMemcpyHostToDevice, c->stream));
+  const float* X = nullptr;
+  GsNorm nrm{};
+  bool use_nrm = false;
+  TL_TRY(norm_for_proj(c, k, PATH_AUTO, T4.n, c->hrows, nullptr, c->g_final, nullptr, c->head, 1, &X, &nrm, &use_nrm));
+  ProjOut o{};
+  o.epi = EPI_ARGMAX;
+  o.lmap = T4.lane;
+  o.ldo = c->cfg.vocab;
+  o.part_val = c->part_val;
+  o.part_idx = c->part_idx;
+  o.n_parts_dev = c->head_nparts;
+  TL_TRY(proj(c, k, PATH_AUTO, X, 0, T4.n, c->head, &c->mhead, nullptr, nullptr, o, nullptr, TL_PROF_HEAD,
+              use_nrm ? &nrm : nullptr));
+  return launch_k(c, head_finalize_kernel, dim3(k), dim3(256), 0, T4, c->lanes, (const float*)c->part_val,
+                  (const int32_t*)c->part_idx, (const int32_t*)c->head_nparts, (int32_t)HEAD_ONLY, dev_argmax,
+                  (int32_t*)nullptr, (int32_t*)nullptr, 0, c->embed, c->h, c->cfg.d, c->cfg.max_seq, 0, c->status,
+                  (unsigned long long*)nullptr, c->warm);
+}
+
+static int speculate_impl(tl_ctx* c, int lane, int n_new, int Ld, int Lv, int ahead, int32_t* out, int32_t* rounds_out) {
+  const tl_config& cfg = c->cfg;
+  LaneState st{};
+  TL_CUDA(cudaMemcpyAsync(&st, c->lanes + lane, sizeof(st), cudaMemcpyDeviceToHost, c->stream));
+  TL_CUDA(cudaStreamSynchronize(c->stream));
+  if (st.phase != PH_BOUNDARY || st.taken != 0 || st.depth < Lv) return TL_ESTATE;
+  const int T = st.pos + 1;
+  if (T + n_new - 1 > cfg.max_seq) return TL_EINVAL;
+  int32_t* tok = c->spec;                   // [lanes] the token each lane takes next (embed input, head output)
+  int32_t* drafted = c->spec + cfg.max_lanes;  // [ahead]
+  int32_t* verify = drafted + c->lay.max_prefill;  // [ahead] the verify pass's greedy tokens
+  std::vector<uint8_t> mask(cfg.max_lanes, 0);
+  mask[lane] = 1;
+  TL_CUDA(cudaMemcpyAsync(c->mask_stage, mask.data(), cfg.max_lanes, cudaMemcpyHostToDevice, c->stream));
+  std::vector<int32_t> Lreq(cfg.max_lanes, Ld);
+  TL_CUDA(cudaMemcpyAsync(c->L_stage, Lreq.data(), cfg.max_lanes * 4, cudaMemcpyHostToDevice, c->stream));
+  // token 0 from the prompt's last position
+  TL_TRY(build_rows(c, 1, SEL_MASK, c->mask_stage, nullptr, nullptr, nullptr));
+  TL_TRY(head_stage(c, cfg.max_lanes, HEAD_ONLY, nullptr, tok, nullptr, nullptr, 0));
+  int32_t t0 = 0;
+  TL_CUDA(cudaMemcpyAsync(&t0, tok + lane, 4, cudaMemcpyDeviceToHost, c->stream));
+  TL_CUDA(cudaStreamSynchronize(c->stream));
+  std::vector<int32_t> tokens{t0};
+  std::vector<int32_t> hd(ahead), hv(ahead);
+  int rounds = 0;
+  while ((int)tokens.size() < n_new) {
+    ++rounds;
+    const int p0 = T + (int)tokens.size() - 1;  // position of the last token taken, not computed yet
+    const int k = std::min(ahead, n_new - (int)tokens.size());
+    TL_CUDA(cudaMemcpyAsync(tok + lane, &tokens.back(), 4, cudaMemcpyHostToDevice, c->stream));
+    // draft: one position at a time at L_draft, each greedy token fed straight back on the device
+    for (int j = 0; j < k; ++j) {
+      TL_TRY(launch_k(c, embed_next_kernel, dim3(cfg.max_lanes), dim3(256), 0, c->lanes, cfg.max_lanes,
+                      (const uint8_t*)c->mask_stage, (const int32_t*)tok, c->embed, c->h, cfg.d, cfg.max_seq, c->status,
+                      c->warm));
+      TL_TRY(pre_blocks_for_entered(c, cfg.max_lanes));
+      for (int l = 0; l < Ld; ++l) {
+        TL_TRY(build_rows(c, 0, SEL_LOOP, c->mask_stage, l == 0 ? c->L_stage : nullptr, nullptr, nullptr));
+        TL_TRY(loop_iteration(c, cfg.max_lanes, nullptr));
+      }
+      TL_TRY(build_rows(c, 1, SEL_MASK, c->mask_stage, nullptr, nullptr, nullptr));
+      TL_TRY(head_stage(c, cfg.max_lanes, HEAD_ONLY, nullptr, tok, nullptr, nullptr, 0));
+      TL_CUDA(cudaMemcpyAsync(drafted + j, tok + lane, 4, cudaMemcpyDeviceToDevice, c->stream));
+    }
+    // verify: the k positions together at L_verify, inputs = the last token taken, then the drafts
+    TL_CUDA(cudaMemcpyAsync(c->tok_stage, &tokens.back(), 4, cudaMemcpyHostToDevice, c->stream));
+    if (k > 1)
+      TL_CUDA(cudaMemcpyAsync(c->tok_stage + 1, drafted, (size_t)(k - 1) * 4, cudaMemcpyDeviceToDevice, c->stream));
+    TL_TRY(rerun_positions(c, lane, p0, k, Lv));
+    TL_TRY(head_hrows(c, k, verify));
+    TL_CUDA(cudaMemcpyAsync(hd.data(), drafted, (size_t)k * 4, cudaMemcpyDeviceToHost, c->stream));
+    TL_CUDA(cudaMemcpyAsync(hv.data(), verify, (size_t)k * 4, cudaMemcpyDeviceToHost, c->stream));
+    TL_CUDA(cudaStreamSynchronize(c->stream));
+    int taken = 0;
+    for (int j = 0; j < k; ++j) {
+      tokens.push_back(hv[j]);
+      ++taken;
+      if (hv[j] != hd[j]) break;
+    }
+    // the lane continues from the last kept position, computed at L_verify by the verify pass
+    const int32_t info[4] = {lane, taken - 1, p0 + taken - 1, Lv};
+    TL_CUDA(cudaMemcpyAsync(c->pf_info, info, sizeof(info), cudaMemcpyHostToDevice, c->stream));
+    TL_TRY(launch_k(c, prefill_finish_batch_kernel, dim3(1), dim3(256), 0, c->lanes, (const int32_t*)c->pf_info, 1,
+                    (const float*)c->hrows, c->h, cfg.d));
+  }
+  TL_CUDA(cudaStreamSynchronize(c->stream));
+  std::memcpy(out, tokens.data(), (size_t)n_new * 4);
+  if (rounds_out) *rounds_out = rounds;
+  return TL_OK;
+}
+
+extern "C" int tl_speculate(tl_ctx* c, int32_t lane, int32_t n_new, int32_t L_draft, int32_t L_verify,
+                            int32_t draft_ahead, int32_t* host_tokens_out, int32_t* host_rounds_out) {
+  if (!c || !host_tokens_out) return TL_EINVAL;
+  if (!c->loaded) return TL_ESTATE;
+  if (lane < 0 || lane >= c->cfg.max_lanes || n_new < 1 || L_draft < 1 || L_verify < 1 || draft_ahead < 1 ||
+      L_draft > c->cfg.L_max || L_verify > c->cfg.L_max || draft_ahead > c->lay.max_prefill ||
+      draft_ahead > c->cfg.max_lanes)
+    return TL_EINVAL;
+  if (c->lane_L[lane] == 0) return TL_ESTATE;
+  if (L_verify > c->lane_L[lane] || L_draft > c->lane_L[lane]) return TL_EKV;
+  // the oracle's speculation has no early exit and no warmup: both are off for its duration
+  const EEParams ee = c->ee;
+  const WarmParams wp = c->warm;
+  c->ee.enabled = 0;
+  c->warm.tokens = 0;
+  const int st = speculate_impl(c, lane, n_new, L_draft, L_verify, draft_ahead, host_tokens_out, host_rounds_out);
+  c->ee = ee;
+  c->warm = wp;
+  return st;
 }
 
 extern "C" int tl_loop_step(tl_ctx* c, const int32_t* dev_L, const uint8_t* dev_mask, uint8_t* dev_exit) {

@@ -299,6 +299,33 @@ int tl_generate(tl_ctx* ctx, const int32_t* host_prompts, int32_t n_lanes, int32
                 const int32_t* host_per_lane_L, int32_t n_new, int32_t* host_tokens_out,
                 int32_t* host_depths_out);
 
+/* Self-speculative greedy decode of one lane ("CLI Reference", speculate:
+ * --draft-loops, --verify-loops, --draft-ahead at temperature 0; the same
+ * weights and one KV cache serve both depths).  The lane must be at a
+ * boundary with no token taken since its prompt: freshly prefilled
+ * (tl_prefill / tl_prefill_batch) at L >= max(L_draft, L_verify), or left so
+ * by a previous tl_speculate.
+ * Its first token comes from the prompt's last position; then each round
+ * drafts up to draft_ahead tokens at L_draft, one position at a time (every
+ * greedy token fed back on the device), runs the drafted positions again at
+ * L_verify as one causal batch (embed, pre blocks, L_verify iterations,
+ * rewriting their K/V in every slot), keeps the drafted tokens up to the first
+ * one the verify pass's greedy choice differs from and takes the verify
+ * pass's token there, and continues from the last kept position.  With greedy
+ * choices the tokens are those of a plain decode at L_verify; the draft only
+ * decides how many positions one verify pass covers.  Early exit and L warmup
+ * are off for the call.  One host synchronisation per round.
+ *   host_tokens_out: int32 [n_new]; host_rounds_out: NULL or the number of
+ *   verify rounds.  Positions up to prompt length + n_new - 2 are written, so
+ *   that must stay below max_seq; draft_ahead <= max_lanes and <=
+ *   max_prefill_tokens.  Afterwards the lane is at its last kept position
+ *   with cap L_verify, as after a prompt: a following tl_decode or
+ *   tl_speculate starts there, so its first token is this call's last.
+ * TL_ESTATE if the lane is not at such a boundary; TL_EKV if a depth exceeds
+ * its cache; TL_EINVAL on bad arguments. */
+int tl_speculate(tl_ctx* ctx, int32_t lane, int32_t n_new, int32_t L_draft, int32_t L_verify, int32_t draft_ahead,
+                 int32_t* host_tokens_out, int32_t* host_rounds_out);
+
 /* Replay of decode ticks as CUDA graphs (default on): each tick of tl_decode /
  * tl_generate is one captured graph whose conditional nodes, set on the
  * device from the live row counts, skip empty stages and pick the CUDA-core or
