@@ -148,6 +148,9 @@ class LoopedLM:
                                  C.byref(rounds)), "tl_speculate")
         return tok, rounds.value
 
+    def set_cascade(self, enabled: bool):
+        check(lib().tl_set_cascade(self.h, 1 if enabled else 0), "tl_set_cascade")
+
     def set_graphs(self, enabled: bool):
         check(lib().tl_set_graphs(self.h, 1 if enabled else 0), "tl_set_graphs")
 

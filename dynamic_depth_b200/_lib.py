@@ -60,6 +60,7 @@ SIGNATURES = {
                               C.c_void_p]),
     "tl_speculate": (C.c_int, [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p,
                                C.c_void_p]),
+    "tl_set_cascade": (C.c_int, [C.c_void_p, C.c_int32]),
     "tl_set_graphs": (C.c_int, [C.c_void_p, C.c_int32]),
     "tl_lane_state_bytes": (C.c_int, [C.c_void_p, C.POINTER(C.c_size_t)]),
     "tl_lane_state_save": (C.c_int, [C.c_void_p, C.c_void_p]),

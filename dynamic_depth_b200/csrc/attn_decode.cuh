@@ -22,6 +22,13 @@
 // another.  Units per warp are raised when needed so a (row, head) never has
 // more than kAttnPieces pieces.
 //
+// Shared prefixes ("Benchmark Comparison" (measured benchmarks), section 2):
+// when lane_shared is given, a row whose lane maps lane_shared[lane] positions
+// of a shared prefix skips them (the cascade pass of attn_tc_kernel attended
+// all such rows against the prefix at once and left a partial per (row,
+// head) in casc); its output merges that partial with its own positions by
+// log-sum-exp.
+//
 // The unit that holds position pos is processed by exactly one warp: it
 // rotates that position's key, writes K and V to the cache for later steps and
 // patches them into its shared-memory copy of the unit (the TMA may have read
@@ -87,7 +94,8 @@ __global__ void __launch_bounds__(AttnCfg<HD>::WARPS * 32, 1)
 attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __restrict__ qkv, float* __restrict__ o,
                    __half* __restrict__ o16, Rows rows, KVGeom g, const float2* __restrict__ rope_cs, int slot_base,
                    int slot_stride, float* __restrict__ part, int32_t* __restrict__ counters,
-                   int32_t* __restrict__ status) {
+                   int32_t* __restrict__ status, const int32_t* __restrict__ lane_shared,
+                   const float* __restrict__ casc) {
   using C = AttnCfg<HD>;
   constexpr int UK = C::UK, STAGES = C::STAGES, WARPS = C::WARPS, HALF = HD / 2, LPR = C::LPR, G = C::G;
   constexpr int CPT = C::COLS / 8;  // 16-byte chunks per tile row
@@ -101,6 +109,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = g.H, d = H * HD;
+  // shared-prefix rows (lane_shared != null): their first lane_shared[lane] positions were attended by the
+  // cascade pass, whose partial (max, sum, output) in casc is merged in here; this kernel takes the rest
+  auto first_block = [&](int r) { return lane_shared ? lane_shared[rows.lane[r]] / UK : 0; };
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < WARPS * STAGES; ++i) mbar_init(smem_u32(&full[i]), 1);
@@ -115,7 +126,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
     const int r0 = threadIdx.x * per, r1 = min(n, r0 + per);
     int s = 0, mx = 0;
     for (int r = r0; r < r1; ++r) {
-      const int nu = (rows.pos[r] + UK) / UK;
+      const int nu = (rows.pos[r] + UK) / UK - first_block(r);
       s += nu;
       mx = max(mx, nu);
     }
@@ -136,7 +147,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
     int run = before + incl - s;
     for (int r = r0; r < r1; ++r) {
       ubase[r] = run * H;
-      run += (rows.pos[r] + UK) / UK;
+      run += (rows.pos[r] + UK) / UK - first_block(r);
     }
     if (threadIdx.x == blockDim.x - 1) ubase[n] = (before + incl) * H;
     __syncthreads();
@@ -175,7 +186,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
   auto issue = [&](int r, int h, int b, int s) {
     const int ln = rows.lane[r];
     const int slot = slot_base + rows.iter[r] * slot_stride;
-    const int p0 = b * UK;
+    const int p0 = (first_block(r) + b) * UK;
     const int pg = p0 >> g.page_shift;
     int page = -1;
     if (slot >= 0 && slot < g.n_slots && pg < g.pages_per_seq)
@@ -229,7 +240,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
   for (int t = 0; t < UK / G; ++t) voff[t] = swz_chunk<C::ROW_BYTES>(kg + G * t, vcc);
   float q[HD];
   float m = -INFINITY, l = 0.f, acc[8];
-  int r = 0, h = 0, b = 0, nu = 1, run_first = 0, ctx = 0, pos = 0, ln = 0;
+  int r = 0, h = 0, b = 0, nu = 1, run_first = 0, ctx = 0, pos = 0, ln = 0, fb = 0;
   locate(u_begin, r, h, b);
   bool aborted = false;
   int consumed = 0;
@@ -241,6 +252,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
       pos = rows.pos[r];
       ln = rows.lane[r];
       ctx = pos + 1;
+      fb = first_block(r);
       run_first = b;
       const float* src = qkv + (int64_t)r * 3 * d + h * HD;
       // lane l rotates pairs (l + 32 k, l + 32 k + HD/2); then every lane gathers the whole vector
@@ -270,10 +282,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
     if (!mbar_wait_warp(smem_u32(&wfull[s]), (i / STAGES) & 1, abort_flag)) { aborted = true; break; }
     consumed = i + 1;
     uint8_t* st = wring + s * C::UNIT_BYTES;
-    const int nvalid = min(UK, ctx - b * UK);
+    const int nvalid = min(UK, ctx - (fb + b) * UK);
     if (b == nu - 1) {
       // this unit holds position pos: rotate its key, append K/V to the cache, patch the staged copy
-      const int j = pos - b * UK;
+      const int j = pos - (fb + b) * UK;
       const float* src = qkv + (int64_t)r * 3 * d + h * HD;
       __half* kp = kv_k_ptr(g, ln, slot_base + rows.iter[r] * slot_stride, pos, h, status);
       __half* vp = kp ? kp + (int64_t)H * g.page_tokens * HD : nullptr;
@@ -373,7 +385,17 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
       const int dim0 = vc * 8;  // this lane's dimensions (lanes of key group 0 write)
       if (run_first == 0 && b == nu - 1) {
         if (kg == 0) {
-          const float inv = 1.f / l;
+          float Lt = l, fo = 1.f;
+          if (fb > 0) {  // merge the shared-prefix partial
+            const float* cp = casc + ((int64_t)r * H + h) * (HD + 2);
+            const float mc = cp[0], M = fmaxf(m, mc);
+            fo = exp2f(m - M);
+            const float fc = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+            Lt = l * fo + cp[1] * fc;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) tot[e] = tot[e] * fo + cp[2 + dim0 + e] * fc;
+          }
+          const float inv = 1.f / Lt;
           float4* op = reinterpret_cast<float4*>(o + (int64_t)r * d + h * HD + dim0);
           op[0] = make_float4(tot[0] * inv, tot[1] * inv, tot[2] * inv, tot[3] * inv);
           op[1] = make_float4(tot[4] * inv, tot[5] * inv, tot[6] * inv, tot[7] * inv);
@@ -403,18 +425,23 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
         if (last) {
           __threadfence();
           const float* base = part + (int64_t)(r * H + h) * kAttnPieces * (HD + 2);
+          // the pieces in order, then the shared-prefix partial when the row has one
+          const float* cp = fb > 0 ? casc + ((int64_t)r * H + h) * (HD + 2) : nullptr;
+          const int n_all = n_pieces + (cp ? 1 : 0);
+          auto piece_ptr = [&](int z) { return z < n_pieces ? base + z * (HD + 2) : cp; };
           float M = -INFINITY;
-          for (int z = 0; z < n_pieces; ++z) M = fmaxf(M, __ldcg(base + z * (HD + 2)));
+          for (int z = 0; z < n_all; ++z) M = fmaxf(M, __ldcg(piece_ptr(z)));
           float Lt = 0.f, outv[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) outv[e] = 0.f;
-          for (int z = 0; z < n_pieces; ++z) {
-            const float mz = __ldcg(base + z * (HD + 2));
+          for (int z = 0; z < n_all; ++z) {
+            const float* pz = piece_ptr(z);
+            const float mz = __ldcg(pz);
             const float f = (mz == -INFINITY) ? 0.f : exp2f(mz - M);
-            Lt += __ldcg(base + z * (HD + 2) + 1) * f;
+            Lt += __ldcg(pz + 1) * f;
             if (kg == 0) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) outv[e] += __ldcg(base + z * (HD + 2) + 2 + dim0 + e) * f;
+              for (int e = 0; e < 8; ++e) outv[e] += __ldcg(pz + 2 + dim0 + e) * f;
             }
           }
           if (kg == 0) {

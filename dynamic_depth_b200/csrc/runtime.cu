@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "host_util.h"
 #include "attn_decode.cuh"
+#include "attn_tc.cuh"
 #include "gemv_stream.cuh"
 #include "kernels.cuh"
 #include "tc_gemm.cuh"
@@ -177,7 +178,7 @@ struct Layout {
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[5], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
-      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec,
+      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec, lane_shared, casc,
       out_tok, out_dep, status, counters, body_kernels, alive, total;
 };
 
@@ -230,6 +231,8 @@ static Layout make_layout(const tl_config* c) {
   L.probe_logits = take(lanes * (size_t)c->vocab * 4);
   L.margin_lane = take(lanes * 4);
   L.spec = take((lanes + 3 * L.max_prefill + 8) * 4);
+  L.lane_shared = take(lanes * 4);
+  L.casc = take(lanes * c->n_heads * (hd + 2) * 4);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
@@ -270,6 +273,11 @@ struct tl_ctx {
   float* probe_logits;  // [lanes][vocab] head logits of the lanes probing in margin mode
   float* margin_lane;   // [lanes] their top-1 minus top-2 margins
   int32_t* spec;        // speculation: [lanes] token per lane, then drafted, verify-input and verify tokens
+  int32_t* lane_shared; // [lanes] shared-prefix positions each lane maps (device copy of h_lane_shared)
+  float* casc;          // [lanes][heads][hd + 2] shared-prefix attention partials of a decode step
+  std::vector<int32_t> h_lane_shared, h_lane_donor;
+  bool cascade_enabled = true;  // tl_set_cascade
+  bool cascade_active = false;  // enabled, and the lanes that share map one donor's prefix of one length
   float *act_a, *act_qkv, *act_q, *act_o, *act_u;
   __half *act_a16, *act_o16, *act_u16;
   float* attn_part;
@@ -298,6 +306,7 @@ struct tl_ctx {
   int32_t *tick_tok = nullptr, *tick_dep = nullptr;
   EEParams tick_ee{};
   WarmParams tick_warm{};
+  bool tick_cascade = false;
   int64_t tick_launches = 0;
   bool graphs_enabled = true;
   bool pdl = true;  // programmatic dependent launch between consecutive kernels
@@ -581,7 +590,17 @@ int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int3
 }
 
 template <int HD>
-int attn_launch_t(tl_ctx* c, const Rows& rows, int slot_base, int slot_stride) {
+int attn_tc_launch(tl_ctx* c, const AttnTcParams& p, dim3 grid) {
+  auto kern = attn_tc_kernel<HD>;
+  static uint64_t attr_done = 0;  // per instantiation: one bit per device
+  if (attr_needed(&attr_done)) {
+    TL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnTcCfg<HD>::SMEM));
+  }
+  return launch_k(c, kern, grid, dim3(256), (size_t)AttnTcCfg<HD>::SMEM, c->kvmap, p);
+}
+
+template <int HD>
+int attn_launch_t(tl_ctx* c, const Rows& rows, int slot_base, int slot_stride, bool cascade) {
   auto kern = attn_decode_kernel<HD>;
   const int smem = attn_smem_bytes<HD>(c->cfg.max_lanes);
   static int attr_smem[64] = {0};  // per instantiation and device: largest opt-in requested so far
@@ -592,17 +611,40 @@ int attn_launch_t(tl_ctx* c, const Rows& rows, int slot_base, int slot_stride) {
   }
   return launch_k(c, kern, dim3(c->n_sms), dim3(AttnCfg<HD>::WARPS * 32), (size_t)smem, c->kvmap,
                   (const float*)c->act_qkv, c->act_o, c->act_o16, rows, c->kv, (const float2*)c->rope, slot_base,
-                  slot_stride, c->attn_part, c->attn_counters, c->status);
+                  slot_stride, c->attn_part, c->attn_counters, c->status,
+                  cascade ? (const int32_t*)c->lane_shared : (const int32_t*)nullptr, (const float*)c->casc);
+}
+
+// Shared-prefix ("cascade") pass of a decode step: for every loop iteration
+// value, all rows whose lanes map the shared prefix attend to it together on
+// the tensor cores, 128 rows per CTA; partials go to c->casc.
+int cascade_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
+  AttnTcParams p{};
+  p.q = c->act_qkv;
+  p.rope = c->rope;
+  p.rows = rows;
+  p.mode = 1;
+  p.lane_shared = c->lane_shared;
+  p.chunks = (max_rows + 127) / 128;
+  p.casc = c->casc;
+  p.g = c->kv;
+  p.slot_base = slot_base;
+  p.slot_stride = slot_stride;
+  p.status = c->status;
+  const int groups = slot_stride > 0 ? c->cfg.L_max : 1;
+  const dim3 grid(groups * p.chunks, c->cfg.n_heads);
+  return c->hd == 64 ? attn_tc_launch<64>(c, p, grid) : attn_tc_launch<128>(c, p, grid);
 }
 
 // Decode attention (one query row per (row, head)) over the rows of `rows`.
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
-  (void)max_rows;
   TL_TRY(prof_start(c, TL_PROF_ATTN));
+  const bool cascade = c->cascade_active && c->hd >= 64;
+  if (cascade) TL_TRY(cascade_launch(c, max_rows, rows, slot_base, slot_stride));
   int st;
-  if (c->hd == 32) st = attn_launch_t<32>(c, rows, slot_base, slot_stride);
-  else if (c->hd == 64) st = attn_launch_t<64>(c, rows, slot_base, slot_stride);
-  else st = attn_launch_t<128>(c, rows, slot_base, slot_stride);
+  if (c->hd == 32) st = attn_launch_t<32>(c, rows, slot_base, slot_stride, false);
+  else if (c->hd == 64) st = attn_launch_t<64>(c, rows, slot_base, slot_stride, cascade);
+  else st = attn_launch_t<128>(c, rows, slot_base, slot_stride, cascade);
   TL_TRY(st);
   return prof_stop(c, TL_PROF_ATTN);
 }
@@ -621,13 +663,33 @@ int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot, 
   return TL_OK;
 }
 
+// Prompt rows per attention tile: 128 for the tensor-core kernel (head widths 64 and 128), 64 otherwise.
+int prompt_tile_rows(const tl_ctx* c) { return c->hd >= 64 ? 128 : 64; }
+
 int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot, const int2* tiles, int n_tiles) {
   TL_TRY(prof_start(c, TL_PROF_ATTN));
   int st;
-  switch (c->hd) {
-    case 32: st = attn_prefill_launch_hd<32>(c, max_rows, rows, slot, tiles, n_tiles); break;
-    case 64: st = attn_prefill_launch_hd<64>(c, max_rows, rows, slot, tiles, n_tiles); break;
-    default: st = attn_prefill_launch_hd<128>(c, max_rows, rows, slot, tiles, n_tiles); break;
+  if (c->hd >= 64 && tiles) {  // tensor cores: 128-row tiles (prompt_tile_rows)
+    AttnTcParams p{};
+    p.q = c->act_q;
+    p.rope = c->rope;
+    p.rows = rows;
+    p.tiles = tiles;
+    p.mode = 0;
+    p.o = c->act_o;
+    p.o16 = c->act_o16;
+    p.g = c->kv;
+    p.slot_base = slot;
+    p.slot_stride = 0;
+    p.status = c->status;
+    const dim3 grid(n_tiles, c->cfg.n_heads);
+    st = c->hd == 64 ? attn_tc_launch<64>(c, p, grid) : attn_tc_launch<128>(c, p, grid);
+  } else {
+    switch (c->hd) {
+      case 32: st = attn_prefill_launch_hd<32>(c, max_rows, rows, slot, tiles, n_tiles); break;
+      case 64: st = attn_prefill_launch_hd<64>(c, max_rows, rows, slot, tiles, n_tiles); break;
+      default: st = attn_prefill_launch_hd<128>(c, max_rows, rows, slot, tiles, n_tiles); break;
+    }
   }
   TL_TRY(st);
   return prof_stop(c, TL_PROF_ATTN);
@@ -839,6 +901,30 @@ void release_lane_pages(tl_ctx* c, int lane) {
     t[i] = -1;
   }
   c->lane_L[lane] = 0;
+  c->h_lane_shared[lane] = 0;
+  c->h_lane_donor[lane] = -1;
+}
+
+// Shared-prefix attention runs as a cascade when enabled and every lane that
+// maps shared pages maps the same donor's prefix of the same length (the
+// tensor-core pass reads one page list per loop iteration).  Copies the
+// per-lane lengths to the device.
+int update_cascade(tl_ctx* c) {
+  int donor = -1, len = 0;
+  bool one = true, any = false;
+  for (int i = 0; i < c->cfg.max_lanes; ++i) {
+    if (c->h_lane_shared[i] == 0) continue;
+    if (!any) {
+      donor = c->h_lane_donor[i];
+      len = c->h_lane_shared[i];
+      any = true;
+    } else if (c->h_lane_donor[i] != donor || c->h_lane_shared[i] != len) {
+      one = false;
+    }
+  }
+  c->cascade_active = c->cascade_enabled && any && one && c->hd >= 64;
+  return check_cuda(cudaMemcpyAsync(c->lane_shared, c->h_lane_shared.data(), (size_t)c->cfg.max_lanes * 4,
+                                    cudaMemcpyHostToDevice, c->stream));
 }
 
 // --------------------------------------------------------- tensor maps ----
@@ -1057,6 +1143,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->probe_logits = (float*)(w + lay.probe_logits);
   c->margin_lane = (float*)(w + lay.margin_lane);
   c->spec = (int32_t*)(w + lay.spec);
+  c->lane_shared = (int32_t*)(w + lay.lane_shared);
+  c->casc = (float*)(w + lay.casc);
   c->mask_stage = (uint8_t*)(w + lay.mask_stage);
   c->out_tok = (int32_t*)(w + lay.out_tok);
   c->out_dep = (int32_t*)(w + lay.out_dep);
@@ -1080,6 +1168,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->free_pages.reserve(lay.n_pages);
   for (int p = lay.n_pages - 1; p >= 0; --p) c->free_pages.push_back(p);
   c->lane_L.assign(cfg->max_lanes, 0);
+  c->h_lane_shared.assign(cfg->max_lanes, 0);
+  c->h_lane_donor.assign(cfg->max_lanes, -1);
   int st = TL_OK;
   do {
     const int half = c->hd / 2;
@@ -1092,6 +1182,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
       break;
     if ((st = check_cuda(cudaMemsetAsync(w + lay.page_table, 0xFF, per_lane * cfg->max_lanes * 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->status, 0, 4, c->stream))) != TL_OK) break;
+    if ((st = check_cuda(cudaMemsetAsync(c->lane_shared, 0, (size_t)cfg->max_lanes * 4, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->counters, 0, 32, c->stream))) != TL_OK) break;
     if ((st = check_cuda(cudaMemsetAsync(c->attn_counters, 0, (size_t)cfg->max_lanes * cfg->n_heads * 4, c->stream))) != TL_OK) break;
     if ((st = encode_all_maps(c)) != TL_OK) break;
@@ -1243,7 +1334,10 @@ static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t sh
   if (total > c->lay.max_prefill) return TL_EINVAL;
   // pages: slots of the pre blocks and of iterations 1..L, for every position up to max_seq
   for (int i = 0; i < n; ++i) release_lane_pages(c, in[i].lane);
-  if ((int64_t)c->free_pages.size() < need) return TL_ENOMEM;
+  if ((int64_t)c->free_pages.size() < need) {
+    update_cascade(c);
+    return TL_ENOMEM;
+  }
   const size_t per_lane = (size_t)c->lay.n_slots * pps;
   for (int i = 0; i < n; ++i) {
     const int used_slots = P + in[i].L * Lb;
@@ -1262,9 +1356,12 @@ static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t sh
         t[(size_t)sl * pps + pg] = id;
       }
     c->lane_L[in[i].lane] = in[i].L;
+    c->h_lane_shared[in[i].lane] = share_pages[i] * pt;
+    c->h_lane_donor[in[i].lane] = share_pages[i] > 0 ? share_from : -1;
     TL_CUDA(cudaMemcpyAsync(c->page_table + (size_t)in[i].lane * per_lane, t, per_lane * 4, cudaMemcpyHostToDevice,
                             c->stream));
   }
+  TL_TRY(update_cascade(c));
   // row table (deepest lanes first), tokens, attention tiles, per-lane finish info
   std::vector<int> order(n);
   for (int i = 0; i < n; ++i) order[i] = i;
@@ -1284,7 +1381,8 @@ static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t sh
       r_pos.push_back(pos0 + t);
       tok.push_back(p.tokens[pos0 + t]);
     }
-    for (int t0 = 0; t0 < Tn; t0 += 64) tiles.push_back(make_int2(row0 + t0, Tn - t0 < 64 ? Tn - t0 : 64));
+    const int tr = prompt_tile_rows(c);
+    for (int t0 = 0; t0 < Tn; t0 += tr) tiles.push_back(make_int2(row0 + t0, Tn - t0 < tr ? Tn - t0 : tr));
     info.insert(info.end(), {p.lane, row0 + Tn - 1, p.T - 1, p.L});
     rows_upto[k + 1] = (int64_t)r_lane.size();
     tiles_upto[k + 1] = (int64_t)tiles.size();
@@ -1370,7 +1468,8 @@ static int rerun_positions(tl_ctx* c, int lane, int pos0, int k, int L) {
   stage_rows[L] = 0;
   for (int i = 0; i < k; ++i) r_pos[i] = pos0 + i;
   std::vector<int2> tiles;
-  for (int t0 = 0; t0 < k; t0 += 64) tiles.push_back(make_int2(t0, k - t0 < 64 ? k - t0 : 64));
+  const int tr = prompt_tile_rows(c);
+  for (int t0 = 0; t0 < k; t0 += tr) tiles.push_back(make_int2(t0, k - t0 < tr ? k - t0 : tr));
   const Rows& R = c->rows[3];
   TL_CUDA(cudaMemcpyAsync(R.lane, r_lane.data(), k * 4, cudaMemcpyHostToDevice, c->stream));
   TL_CUDA(cudaMemcpyAsync(R.pos, r_pos.data(), k * 4, cudaMemcpyHostToDevice, c->stream));
@@ -1657,7 +1756,7 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
 static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
   if (c->tick_exec && c->tick_lanes == n_lanes && c->tick_new == n_new && c->tick_tok == tok_out &&
       c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee) && c->tick_warm.tokens == c->warm.tokens &&
-      c->tick_warm.L == c->warm.L)
+      c->tick_warm.L == c->warm.L && c->tick_cascade == c->cascade_active)
     return TL_OK;
   if (c->tick_exec) {
     cudaGraphExecDestroy(c->tick_exec);
@@ -1691,6 +1790,7 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   c->tick_dep = dep_out;
   c->tick_ee = c->ee;
   c->tick_warm = c->warm;
+  c->tick_cascade = c->cascade_active;
   c->tick_launches = 1;  // the planning kernel outside the conditional bodies
   return TL_OK;
 }
@@ -1829,6 +1929,12 @@ extern "C" int tl_profile_end(tl_ctx* c, int64_t* groups, double* total_ms) {
   }
   c->prof_mask = 0;
   return TL_OK;
+}
+
+extern "C" int tl_set_cascade(tl_ctx* c, int32_t enabled) {
+  if (!c) return TL_EINVAL;
+  c->cascade_enabled = enabled != 0;
+  return update_cascade(c);
 }
 
 extern "C" int tl_set_graphs(tl_ctx* c, int32_t enabled) {

@@ -385,13 +385,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
           }
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (t < ncols) {
-          float bv = bv_s[t];
-          int bi = bi_s[t];
+        for (int c = t; c < ncols; c += 128) {  // activation rows of the tile (up to NT = 256): 128 threads
+          float bv = bv_s[c];
+          int bi = bi_s[c];
           for (int w = 1; w < 4; ++w)
-            if (better(bv_s[w * NT + t], bi_s[w * NT + t], bv, bi)) { bv = bv_s[w * NT + t]; bi = bi_s[w * NT + t]; }
-          p.o.part_val[(int64_t)(n0 + t) * p.o.n_parts + blockIdx.x] = bv;
-          p.o.part_idx[(int64_t)(n0 + t) * p.o.n_parts + blockIdx.x] = bi;
+            if (better(bv_s[w * NT + c], bi_s[w * NT + c], bv, bi)) { bv = bv_s[w * NT + c]; bi = bi_s[w * NT + c]; }
+          p.o.part_val[(int64_t)(n0 + c) * p.o.n_parts + blockIdx.x] = bv;
+          p.o.part_idx[(int64_t)(n0 + c) * p.o.n_parts + blockIdx.x] = bi;
         }
         if (blockIdx.x == 0 && blockIdx.y == 0 && t == 0 && p.o.n_parts_dev) p.o.n_parts_dev[0] = p.o.n_parts;
       } else

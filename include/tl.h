@@ -326,6 +326,18 @@ int tl_generate(tl_ctx* ctx, const int32_t* host_prompts, int32_t n_lanes, int32
 int tl_speculate(tl_ctx* ctx, int32_t lane, int32_t n_new, int32_t L_draft, int32_t L_verify, int32_t draft_ahead,
                  int32_t* host_tokens_out, int32_t* host_rounds_out);
 
+/* Shared-prefix ("cascade") attention in decode steps (default on; "Benchmark
+ * Comparison" (measured benchmarks), section 2: one cached prefix serves many
+ * requests, and in a looped model every loop iteration of them).  When every
+ * lane that maps shared prefix pages (tl_prefill with share_prefix_from_lane)
+ * maps the same donor's prefix of the same length, each decode attention step
+ * first attends all such rows at one loop iteration to the prefix together
+ * on the tensor cores (head widths 64 and 128), reading each prefix page once
+ * per step instead of once per lane, and then each row's own positions; the
+ * two are merged by log-sum-exp.  Same result up to summation order.
+ * enabled = 0 attends every lane's whole context on its own. */
+int tl_set_cascade(tl_ctx* ctx, int32_t enabled);
+
 /* Replay of decode ticks as CUDA graphs (default on): each tick of tl_decode /
  * tl_generate is one captured graph whose conditional nodes, set on the
  * device from the live row counts, skip empty stages and pick the CUDA-core or
