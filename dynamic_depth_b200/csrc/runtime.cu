@@ -178,7 +178,7 @@ struct Layout {
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[5], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
-      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec, lane_shared, casc,
+      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec, lane_shared, casc, wstage,
       out_tok, out_dep, status, counters, body_kernels, alive, total;
 };
 
@@ -233,6 +233,8 @@ static Layout make_layout(const tl_config* c) {
   L.spec = take((lanes + 3 * L.max_prefill + 8) * 4);
   L.lane_shared = take(lanes * 4);
   L.casc = take(lanes * c->n_heads * (hd + 2) * 4);
+  // prompt batches wide enough for the persistent GEMM: one block's five matrices in fp16
+  L.wstage = take(L.max_prefill >= 512 ? (size_t)(4 * d * d + 3 * d * F) * 2 : 0);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
@@ -278,6 +280,9 @@ struct tl_ctx {
   std::vector<int32_t> h_lane_shared, h_lane_donor;
   bool cascade_enabled = true;  // tl_set_cascade
   bool cascade_active = false;  // enabled, and the lanes that share map one donor's prefix of one length
+  __half* wstage = nullptr;     // fp16 staging copy of one block's matrices for wide prompt batches
+  BlockW sblock{};              // views and TMA maps of that copy
+  const BlockW* staged_src = nullptr;  // the block whose matrices the copy holds
   float *act_a, *act_qkv, *act_q, *act_o, *act_u;
   __half *act_a16, *act_o16, *act_u16;
   float* attn_part;
@@ -525,6 +530,11 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   if (max_rows >= kWideRows && o.epi != EPI_ARGMAX) {
     p.kb_per_split = W.K / 64;
     const CUtensorMap& mxw = c->xmap[xsel][nmat == 1 ? 2 : 1];  // 256-row tiles, 128 for the gate/up pair
+    if (W.fmt == FMT_F16) {
+      if (o.epi == EPI_SWIGLU) return tc_wide_launch<2, FMT_F16, EPI_SWIGLU>(c, max_rows, mw, m2, mxw, p);
+      if (o.epi == EPI_RESID) return tc_wide_launch<1, FMT_F16, EPI_RESID>(c, max_rows, mw, m2, mxw, p);
+      return tc_wide_launch<1, FMT_F16, EPI_STORE>(c, max_rows, mw, m2, mxw, p);
+    }
     if (W.fmt == TL_FMT_INT4) {
       if (o.epi == EPI_SWIGLU) return tc_wide_launch<2, TL_FMT_INT4, EPI_SWIGLU>(c, max_rows, mw, m2, mxw, p);
       if (o.epi == EPI_RESID) return tc_wide_launch<1, TL_FMT_INT4, EPI_RESID>(c, max_rows, mw, m2, mxw, p);
@@ -746,6 +756,20 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   if (prompt) path = max_rows > kGemvMaxRows ? PATH_TC : PATH_GEMV;
   const int d = c->cfg.d, F = c->cfg.ffn;
   const bool defer = pend && prompt && max_rows >= kWideRows;
+  // prompt batches on the persistent GEMM read an fp16 copy of the block's matrices, made once per pass and
+  // block (the loop block once for all its iterations), instead of dequantising every tile again
+  const bool staged = prompt && max_rows >= kWideRows && c->wstage;
+  if (staged && c->staged_src != &w) {
+    const MatView* src[5] = {&w.wqkv, &w.wo, &w.wg, &w.wu, &w.wd};
+    const MatView* dst[5] = {&c->sblock.wqkv, &c->sblock.wo, &c->sblock.wg, &c->sblock.wu, &c->sblock.wd};
+    for (int i = 0; i < 5; ++i) {
+      const int64_t words = (int64_t)src[i]->N * src[i]->K / 8;
+      TL_TRY(launch_k(c, stage_f16_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, *src[i],
+                      const_cast<__half*>(reinterpret_cast<const __half*>(dst[i]->bf))));
+    }
+    c->staged_src = &w;
+  }
+  const BlockW& pw = staged ? c->sblock : w;  // the projections' matrices and maps
   const float* X = nullptr;
   GsNorm nrm{};
   bool use_nrm = false;
@@ -756,7 +780,7 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   o.epi = EPI_STORE;
   o.out = c->act_qkv;
   o.ldo = 3 * d;
-  TL_TRY(proj(c, max_rows, path, X, 0, rows.n, w.wqkv, &w.mqkv, nullptr, nullptr, o, nullptr, TL_PROF_PROJ,
+  TL_TRY(proj(c, max_rows, path, X, 0, rows.n, pw.wqkv, &pw.mqkv, nullptr, nullptr, o, nullptr, TL_PROF_PROJ,
               use_nrm ? &nrm : nullptr));
   if (prompt) {
     TL_TRY(launch_k(c, rope_kv_kernel, dim3(max_rows), dim3(d / 2), 0, c->act_qkv, c->act_q, rows, c->kv, c->rope,
@@ -774,16 +798,16 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
     r.out = c->act_q;
     r.ldo = d;
   }
-  TL_TRY(proj(c, max_rows, path, c->act_o, 1, rows.n, w.wo, &w.mo, nullptr, nullptr, r, nullptr));
+  TL_TRY(proj(c, max_rows, path, c->act_o, 1, rows.n, pw.wo, &pw.mo, nullptr, nullptr, r, nullptr));
   TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g2, nullptr, w.wg, 2, &X, &nrm, &use_nrm,
                        defer ? PendingAdd{c->act_q, rows.n, max_rows} : PendingAdd{}));
   ProjOut sw{};
   sw.epi = EPI_SWIGLU;
   sw.out = c->act_u;
   sw.ldo = F;
-  TL_TRY(proj(c, max_rows, path, X, 0, rows.n, w.wg, &w.mg, &w.wu, &w.mu, sw, c->act_u16, TL_PROF_PROJ,
+  TL_TRY(proj(c, max_rows, path, X, 0, rows.n, pw.wg, &pw.mg, &pw.wu, &pw.mu, sw, c->act_u16, TL_PROF_PROJ,
               use_nrm ? &nrm : nullptr));
-  TL_TRY(proj(c, max_rows, path, c->act_u, 2, rows.n, w.wd, &w.md, nullptr, nullptr, r, nullptr));
+  TL_TRY(proj(c, max_rows, path, c->act_u, 2, rows.n, pw.wd, &pw.md, nullptr, nullptr, r, nullptr));
   if (defer) *pend = PendingAdd{c->act_q, rows.n, max_rows};
   return TL_OK;
 }
@@ -981,6 +1005,14 @@ int encode_all_maps(tl_ctx* c) {
       TL_TRY(encode_weight_map(&b.md, b.wd));
     }
   TL_TRY(encode_weight_map(&c->mhead, c->head));
+  if (c->wstage) {  // the staging copy: fp16 tiles of 128 rows x 64 K, in the MMA's swizzled layout
+    BlockW& b = c->sblock;
+    const MatView* mv5[5] = {&b.wqkv, &b.wo, &b.wg, &b.wu, &b.wd};
+    CUtensorMap* mp5[5] = {&b.mqkv, &b.mo, &b.mg, &b.mu, &b.md};
+    for (int i = 0; i < 5; ++i)
+      TL_TRY(encode_2d(mp5[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv5[i]->bf, (uint64_t)mv5[i]->K, (uint64_t)mv5[i]->N,
+                       (uint64_t)mv5[i]->K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  }
   {  // KV pool as rows of hd fp16: a page is [K: H x P rows][V: H x P rows]
     const uint64_t pool_rows = (uint64_t)c->lay.n_pages * 2 * c->cfg.n_heads * c->cfg.kv_page_tokens;
     const uint32_t cols = c->hd > 64 ? 64 : (uint32_t)c->hd;
@@ -1145,6 +1177,22 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->spec = (int32_t*)(w + lay.spec);
   c->lane_shared = (int32_t*)(w + lay.lane_shared);
   c->casc = (float*)(w + lay.casc);
+  if (lay.max_prefill >= 512) {
+    c->wstage = (__half*)(w + lay.wstage);
+    const int64_t d = cfg->d, F = cfg->ffn;
+    const int64_t off[5] = {0, 3 * d * d, 4 * d * d, 4 * d * d + F * d, 4 * d * d + 2 * F * d};
+    const int64_t NN[5] = {3 * d, d, F, F, d}, KK[5] = {d, d, d, d, F};
+    MatView* mv5[5] = {&c->sblock.wqkv, &c->sblock.wo, &c->sblock.wg, &c->sblock.wu, &c->sblock.wd};
+    for (int i = 0; i < 5; ++i) {
+      MatView m{};
+      m.fmt = FMT_F16;
+      m.N = (int)NN[i];
+      m.K = (int)KK[i];
+      m.group = cfg->group;
+      m.bf = reinterpret_cast<const uint16_t*>(c->wstage + off[i]);
+      *mv5[i] = m;
+    }
+  }
   c->mask_stage = (uint8_t*)(w + lay.mask_stage);
   c->out_tok = (int32_t*)(w + lay.out_tok);
   c->out_dep = (int32_t*)(w + lay.out_dep);
@@ -1254,6 +1302,7 @@ extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
     TL_TRY(launch_k(c, int4_repack_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, (uint32_t*)m->q, words));
   }
   TL_CUDA(cudaStreamSynchronize(c->stream));
+  c->staged_src = nullptr;
   c->loaded = true;
   return TL_OK;
 }

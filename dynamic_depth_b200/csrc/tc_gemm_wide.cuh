@@ -31,13 +31,20 @@
 
 namespace tl {
 
+// Weights already in fp16 (a prompt pass's staging buffer, see stage_f16_kernel):
+// the weight tile arrives by TMA in the canonical layout and nothing is converted.
+constexpr int FMT_F16 = 2;
+
 template <int NMAT, int FMT>
 struct TcWideCfg {
   static constexpr int NT = 256 / NMAT;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = NT * 64 * 2;
-  static constexpr int RAW_BYTES = (FMT == TL_FMT_INT4) ? 128 * 32 : 128 * 128;
-  static constexpr int stage_bytes = NMAT * (A_BYTES + RAW_BYTES) + B_BYTES;
+  static constexpr int RAW_BYTES = (FMT == TL_FMT_INT4) ? 128 * 32 : (FMT == FMT_F16 ? 0 : 128 * 128);
+  // 64-wide k-blocks per pipeline stage (two per stage, with only two stages fitting, measured slower:
+  // 766 against 837 TFLOP/s on the 64 x 512-token prompt pass)
+  static constexpr int KPS = 1;
+  static constexpr int stage_bytes = NMAT * (KPS * A_BYTES + RAW_BYTES) + KPS * B_BYTES;
   static constexpr int LIMIT = 227 * 1024;  // opt-in shared memory per CTA
   static constexpr int RESERVE = 2048;      // 1024-byte alignment slack + barriers
   static constexpr int FIT = (LIMIT - RESERVE) / stage_bytes;
@@ -75,9 +82,10 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
   constexpr int NT = C::NT, STAGES = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_wide[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_wide) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = base;                                  // [STAGES][NMAT][A_BYTES] fp16 weight tiles
-  uint8_t* sB = sA + STAGES * NMAT * C::A_BYTES;       // [STAGES][B_BYTES] fp16 activation tiles
-  uint8_t* sRaw = sB + STAGES * C::B_BYTES;            // [STAGES][NMAT][RAW_BYTES]
+  constexpr int KPS = C::KPS;
+  uint8_t* sA = base;                                  // [STAGES][NMAT][KPS][A_BYTES] fp16 weight tiles
+  uint8_t* sB = sA + STAGES * NMAT * KPS * C::A_BYTES;  // [STAGES][KPS][B_BYTES] fp16 activation tiles
+  uint8_t* sRaw = sB + STAGES * KPS * C::B_BYTES;      // [STAGES][NMAT][RAW_BYTES]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + STAGES * NMAT * C::RAW_BYTES);
   uint64_t* full = bars;                  // TMA landed
   uint64_t* afull = bars + STAGES;        // weight tile converted
@@ -120,6 +128,7 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
   const int n_tiles = rows > p.skip_at_or_below ? (rows + NT - 1) / NT : 0;
   const int n_total = m_tiles * n_tiles;
   const int nkb = p.K / 64;
+  const int nks = (nkb + KPS - 1) / KPS;  // pipeline steps per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
@@ -128,16 +137,29 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
     bool ok = true;
     for (int t = blockIdx.x; t < n_total && ok; t += gridDim.x) {
       const int m0 = (t % m_tiles) * 128, n0 = (t / m_tiles) * NT;
-      for (int kb = 0; kb < nkb; ++kb, ++g) {
+      for (int ks = 0; ks < nks; ++ks, ++g) {
         const int s = g % STAGES, r = g / STAGES;
         if (r > 0 && !mbar_wait_warp(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) { ok = false; break; }
         if (elect_one()) {
           const uint32_t fb = smem_u32(&full[s]);
-          mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
-          const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
-          tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
-          if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
-          tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
+          const int nq = min(KPS, nkb - ks * KPS);  // k-blocks in this step
+          if constexpr (FMT == FMT_F16) {  // fp16 weight tiles straight into the MMA layout
+            mbar_expect_tx(fb, nq * (NMAT * C::A_BYTES + C::B_BYTES));
+            for (int q = 0; q < nq; ++q) {
+              const int kb = ks * KPS + q;
+              tma_load_2d(smem_u32(sA + ((s * NMAT + 0) * KPS + q) * C::A_BYTES), &mapW, kb * 64, m0, fb);
+              if constexpr (NMAT == 2)
+                tma_load_2d(smem_u32(sA + ((s * NMAT + 1) * KPS + q) * C::A_BYTES), &mapW2, kb * 64, m0, fb);
+              tma_load_2d(smem_u32(sB + (s * KPS + q) * C::B_BYTES), &mapX, kb * 64, n0, fb);
+            }
+          } else {
+            const int kb = ks;
+            mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
+            const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
+            tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
+            if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+            tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
+          }
         }
         __syncwarp();
       }
@@ -158,23 +180,26 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
       if (use > 0 && !mbar_wait_warp(smem_u32(&accempty[buf]), (use - 1) & 1, abort_flag)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t acc = tmem + (uint32_t)(buf * NMAT * NT);
-      for (int kb = 0; kb < nkb; ++kb, ++g) {
+      for (int ks = 0; ks < nks; ++ks, ++g) {
         const int s = g % STAGES, r = g / STAGES;
-        if (!mbar_wait_warp(smem_u32(&afull[s]), r & 1, abort_flag) ||
+        if ((FMT != FMT_F16 && !mbar_wait_warp(smem_u32(&afull[s]), r & 1, abort_flag)) ||
             !mbar_wait_warp(smem_u32(&full[s]), r & 1, abort_flag)) {
           ok = false;
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
+        const int nq = min(KPS, nkb - ks * KPS);
         if (elect_one()) {
+          for (int q = 0; q < nq; ++q) {
+            const uint32_t b_addr = smem_u32(sB + (s * KPS + q) * C::B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = umma_desc(b_addr + kk * 32);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bdesc = umma_desc(b_addr + kk * 32);
 #pragma unroll
-            for (int mat = 0; mat < NMAT; ++mat) {
-              const uint64_t adesc = umma_desc(smem_u32(sA + (s * NMAT + mat) * C::A_BYTES) + kk * 32);
-              umma_f16(acc + mat * NT, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+              for (int mat = 0; mat < NMAT; ++mat) {
+                const uint64_t adesc = umma_desc(smem_u32(sA + ((s * NMAT + mat) * KPS + q) * C::A_BYTES) + kk * 32);
+                umma_f16(acc + mat * NT, adesc, bdesc, idesc, (ks > 0 || q > 0 || kk > 0) ? 1u : 0u);
+              }
             }
           }
           umma_commit(smem_u32(&empty[s]));
@@ -184,7 +209,7 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
       if (ok && elect_one()) umma_commit(smem_u32(&accfull[buf]));
       __syncwarp();
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 8 && FMT != FMT_F16) {
     // ------------------------------------------------------------ convert
     const int tr = threadIdx.x - 128;  // weight row within the tile
     const int gpr = (FMT == TL_FMT_INT4) ? p.K / p.group : 0;
@@ -292,6 +317,28 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::TMEM_COLS)
                  : "memory");
   }
+}
+
+// A prompt pass's staging copy of one weight matrix: out [N][K] fp16 with
+// exactly the values the converting kernels above build in shared memory
+// (INT4: (u - 8) exact, times the fp16 group scale, rounded once; BF16: the
+// same value in fp16).  One thread per 8 consecutive elements.
+__global__ void stage_f16_kernel(MatView W, __half* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();  // the previous pass's GEMMs may still read this buffer
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-element word
+  const int64_t words = (int64_t)W.N * W.K / 8;
+  if (i >= words) return;
+  const int64_t n = i / (W.K / 8), w = i % (W.K / 8);
+  uint4 v;
+  if (W.fmt == TL_FMT_INT4) {
+    const uint32_t word = reinterpret_cast<const uint32_t*>(W.q)[i];
+    const __half sc = W.s[n * (W.K / W.group) + (8 * w) / W.group];
+    v = int4_word_to_half8(word, __halves2half2(sc, sc));
+  } else {
+    v = bf16x8_to_half8(reinterpret_cast<const uint4*>(W.bf)[i]);
+  }
+  reinterpret_cast<uint4*>(out)[i] = v;
 }
 
 }  // namespace tl
