@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "host_util.h"
 #include "attn_decode.cuh"
+#include "attn_split.cuh"
 #include "attn_tc.cuh"
 #include "gemv_stream.cuh"
 #include "kernels.cuh"
@@ -647,14 +648,31 @@ int cascade_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int
 }
 
 // Decode attention (one query row per (row, head)) over the rows of `rows`.
+// Decode attention over the rows of `rows`.  Steps with a shared-prefix
+// cascade take the balanced persistent kernel (which merges the cascade's
+// partials); the others the split-context kernel, whose small CTAs measured
+// faster around the neighbouring projections in CUDA-graph ticks (64 lanes:
+// 346 against 358 ms per decode pass; one lane at L = 8: 1,609 against 1,516
+// tokens/s), with the same per-kind kernel time.
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
   TL_TRY(prof_start(c, TL_PROF_ATTN));
   const bool cascade = c->cascade_active && c->hd >= 64;
-  if (cascade) TL_TRY(cascade_launch(c, max_rows, rows, slot_base, slot_stride));
   int st;
-  if (c->hd == 32) st = attn_launch_t<32>(c, rows, slot_base, slot_stride, false);
-  else if (c->hd == 64) st = attn_launch_t<64>(c, rows, slot_base, slot_stride, cascade);
-  else st = attn_launch_t<128>(c, rows, slot_base, slot_stride, cascade);
+  if (cascade) {
+    TL_TRY(cascade_launch(c, max_rows, rows, slot_base, slot_stride));
+    st = c->hd == 64 ? attn_launch_t<64>(c, rows, slot_base, slot_stride, true)
+                     : attn_launch_t<128>(c, rows, slot_base, slot_stride, true);
+  } else {
+    int ks = (kAttnCtaTarget + max_rows * c->cfg.n_heads - 1) / (max_rows * c->cfg.n_heads);
+    ks = ks < 1 ? 1 : (ks > kAttnPieces ? kAttnPieces : ks);
+    if (max_rows > 1) ks = ks < 4 ? 4 : ks;
+    const dim3 grid(max_rows, c->cfg.n_heads, ks);
+    switch (c->hd) {
+      case 32: st = launch_k(c, attn_split_kernel<32>, grid, dim3(128), 0, (const float*)c->act_qkv, c->act_o, c->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
+      case 64: st = launch_k(c, attn_split_kernel<64>, grid, dim3(128), 0, (const float*)c->act_qkv, c->act_o, c->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
+      default: st = launch_k(c, attn_split_kernel<128>, grid, dim3(128), 0, (const float*)c->act_qkv, c->act_o, c->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride, c->attn_part, c->attn_counters, c->status); break;
+    }
+  }
   TL_TRY(st);
   return prof_stop(c, TL_PROF_ATTN);
 }
@@ -803,7 +821,8 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
                        defer ? PendingAdd{c->act_q, rows.n, max_rows} : PendingAdd{}));
   ProjOut sw{};
   sw.epi = EPI_SWIGLU;
-  sw.out = c->act_u;
+  // only the tensor-core variant runs here: the down projection reads the fp16 copy alone
+  sw.out = (path == PATH_TC && max_rows > kGemvMaxRows) ? nullptr : c->act_u;
   sw.ldo = F;
   TL_TRY(proj(c, max_rows, path, X, 0, rows.n, pw.wg, &pw.mg, &pw.wu, &pw.mu, sw, c->act_u16, TL_PROF_PROJ,
               use_nrm ? &nrm : nullptr));

@@ -140,7 +140,7 @@ __device__ __forceinline__ void tc_emit(const TcParams& p, int row, int m, float
     o.out[(int64_t)row * o.ldo + m] = v;
   } else if constexpr (EPI == EPI_SWIGLU) {
     const float u = silu_f(v) * v2;
-    o.out[(int64_t)row * o.ldo + m] = u;
+    if (o.out) o.out[(int64_t)row * o.ldo + m] = u;
     if (p.out16) p.out16[(int64_t)row * o.ldo + m] = __float2half_rn(u);
   } else if constexpr (EPI == EPI_RESID) {
     const int hr = o.map ? o.map[row] : row;

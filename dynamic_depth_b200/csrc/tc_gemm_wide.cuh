@@ -9,8 +9,8 @@
 // overlaps the next tile's main loop: the TMEM accumulator is double
 // buffered (2 x 256 columns).
 //
-// Warp roles (384 threads; the producer and MMA warps run their loops with
-// all 32 lanes and let one elected lane issue): warp 0 issues the TMA loads (raw weight tile and
+// Warp roles (384 threads; one lane of the producer and of the MMA warp runs
+// the whole issue loop): warp 0 issues the TMA loads (raw weight tile and
 // fp16 activation tile per 64-wide k-block) into a ring of stages; warps 4-7
 // convert the raw weight tile to fp16 in the canonical K-major SWIZZLE_128B
 // layout (INT4: (u - 8) * scale rounded once to fp16, scales read from
@@ -132,15 +132,15 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
-    // the whole warp runs the loop (waits included); one elected lane issues
-    int g = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < n_total && ok; t += gridDim.x) {
-      const int m0 = (t % m_tiles) * 128, n0 = (t / m_tiles) * NT;
-      for (int ks = 0; ks < nks; ++ks, ++g) {
-        const int s = g % STAGES, r = g / STAGES;
-        if (r > 0 && !mbar_wait_warp(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) { ok = false; break; }
-        if (elect_one()) {
+    // one lane runs the whole producer loop
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_total && ok; t += gridDim.x) {
+        const int m0 = (t % m_tiles) * 128, n0 = (t / m_tiles) * NT;
+        for (int ks = 0; ks < nks; ++ks, ++g) {
+          const int s = g % STAGES, r = g / STAGES;
+          if (r > 0 && !mbar_wait(smem_u32(&empty[s]), (r - 1) & 1, abort_flag)) { ok = false; break; }
           const uint32_t fb = smem_u32(&full[s]);
           const int nq = min(KPS, nkb - ks * KPS);  // k-blocks in this step
           if constexpr (FMT == FMT_F16) {  // fp16 weight tiles straight into the MMA layout
@@ -161,35 +161,37 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
             tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
           }
         }
-        __syncwarp();
+      }
+      if (*abort_flag) {  // let copies already in flight land before the CTA leaves
+        for (int i = (g > STAGES ? g - STAGES : 0); i < g; ++i) {
+          volatile int32_t never = 0;
+          mbar_wait(smem_u32(&full[i % STAGES]), (i / STAGES) & 1, &never);
+        }
       }
     }
-    if (*abort_flag && lane == 0) {  // let copies already in flight land before the CTA leaves
-      for (int i = (g > STAGES ? g - STAGES : 0); i < g; ++i) {
-        volatile int32_t never = 0;
-        mbar_wait(smem_u32(&full[i % STAGES]), (i / STAGES) & 1, &never);
-      }
-    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
-    constexpr uint32_t idesc = umma_idesc_f16<NT>();
-    int g = 0, it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < n_total && ok; t += gridDim.x, ++it) {
-      const int buf = it & 1, use = it >> 1;
-      if (use > 0 && !mbar_wait_warp(smem_u32(&accempty[buf]), (use - 1) & 1, abort_flag)) break;
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t acc = tmem + (uint32_t)(buf * NMAT * NT);
-      for (int ks = 0; ks < nks; ++ks, ++g) {
-        const int s = g % STAGES, r = g / STAGES;
-        if ((FMT != FMT_F16 && !mbar_wait_warp(smem_u32(&afull[s]), r & 1, abort_flag)) ||
-            !mbar_wait_warp(smem_u32(&full[s]), r & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
+    // one lane runs the whole issue loop: no warp-wide step (shuffle, elect, sync) between k-blocks, so the
+    // next MMAs follow a completed barrier as closely as possible
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_f16<NT>();
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_total && ok; t += gridDim.x, ++it) {
+        const int buf = it & 1, use = it >> 1;
+        if (use > 0 && !mbar_wait(smem_u32(&accempty[buf]), (use - 1) & 1, abort_flag)) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int nq = min(KPS, nkb - ks * KPS);
-        if (elect_one()) {
+        const uint32_t acc = tmem + (uint32_t)(buf * NMAT * NT);
+        for (int ks = 0; ks < nks; ++ks, ++g) {
+          const int s = g % STAGES, r = g / STAGES;
+          if ((FMT != FMT_F16 && !mbar_wait(smem_u32(&afull[s]), r & 1, abort_flag)) ||
+              !mbar_wait(smem_u32(&full[s]), r & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const int nq = min(KPS, nkb - ks * KPS);
           for (int q = 0; q < nq; ++q) {
             const uint32_t b_addr = smem_u32(sB + (s * KPS + q) * C::B_BYTES);
 #pragma unroll
@@ -204,11 +206,10 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
           }
           umma_commit(smem_u32(&empty[s]));
         }
-        __syncwarp();
+        if (ok) umma_commit(smem_u32(&accfull[buf]));
       }
-      if (ok && elect_one()) umma_commit(smem_u32(&accfull[buf]));
-      __syncwarp();
     }
+    __syncwarp();
   } else if (warp >= 4 && warp < 8 && FMT != FMT_F16) {
     // ------------------------------------------------------------ convert
     const int tr = threadIdx.x - 128;  // weight row within the tile
