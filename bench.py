@@ -130,16 +130,21 @@ def loop_block_weight_bytes(sh) -> int:
     return sum(n * k // 2 + n * (k // g) * 2 for n, k in [(3 * d, d), (d, d), (F, d), (F, d), (d, F)])
 
 
-def schedule_units(sh, wl, depths):
+def schedule_units(sh, wl, depths, same_tick: bool = True):
     """Counts behind the algorithmic bytes, from the executed depth schedule.
 
-    Lane i runs one loop iteration in every tick k < S_i = sum of its decode
-    depths (the boundary stage of a tick feeds the same tick's loop), and takes
-    a new token (pre blocks) at tick 0 and whenever a token's loop finished."""
+    A lane takes a new token (head, embedding, pre blocks) in the boundary
+    stage of tick 0 and whenever a token's loop finished.  same_tick (the
+    library's entry_in_boundary): the token's first loop iteration runs in that
+    same boundary stage and the rest in the following ticks, so a token of
+    depth D spans D ticks; otherwise its D iterations run in the D ticks after
+    the boundary stage, D + 1 ticks per token.  The boundary stage and the
+    loop step of a tick run concurrently on disjoint lanes."""
     T, n_new = wl.prompt_len, wl.n_new
-    S_i = depths[:, 1:].sum(axis=1)
-    ticks = int(S_i.max()) + 1
-    loop_rows = np.array([(S_i > k).sum() for k in range(ticks)])
+    extra = 0 if same_tick else 1
+    span = (depths[:, 1:].astype(np.int64) + extra).sum(axis=1)
+    ticks = int(span.max()) + 1
+    loop_rows = np.zeros(ticks, dtype=np.int64)
     entered = np.zeros(ticks, dtype=np.int64)
     boundary = np.zeros(ticks, dtype=np.int64)
     kv_bytes_per_pos = 2 * sh.d * 2  # K and V, fp16
@@ -150,10 +155,12 @@ def schedule_units(sh, wl, depths):
         boundary[0] += 1
         for t in range(1, n_new):
             ctx = T + t  # the row at position T + t - 1 attends to positions 0 .. T + t - 1
+            D = int(depths[i, t])
             entered[tick] += 1
-            attn_bytes += (sh.n_pre + int(depths[i, t])) * ctx * kv_bytes_per_pos
-            attn_rows += sh.n_pre + int(depths[i, t])
-            tick += int(depths[i, t])
+            loop_rows[tick + extra:tick + extra + D] += 1
+            attn_bytes += (sh.n_pre + D) * ctx * kv_bytes_per_pos
+            attn_rows += sh.n_pre + D
+            tick += D + extra
             boundary[tick] += 1
     return {"ticks": ticks, "loop_rows": loop_rows, "entered": entered, "boundary": boundary,
             "attn_bytes": attn_bytes, "attn_rows": attn_rows}
@@ -263,7 +270,8 @@ def run_ours(args, rank, world, local_rank):
     depths = dep.cpu().numpy()
 
     # roofline of the dominant kernel kind, from the live event timings
-    units = schedule_units(sh, wl, depths)
+    same_tick = bool(st1["entry_in_boundary"])
+    units = schedule_units(sh, wl, depths, same_tick)
     groups, kind_ms = prof
     kinds = {}
     for k, name in ((1, "attention"), (2, "projections"), (3, "head")):
@@ -362,6 +370,8 @@ def run_ours(args, rank, world, local_rank):
         "lane_iterations_no_exit": int(sum(int(L) * (wl.n_new - 1) for L in Ls)),
         "depth_histogram": {int(k): int(v) for k, v in zip(*np.unique(depths[:, 1:], return_counts=True))},
         "ticks_per_step": units["ticks"],
+        "tick_layout": "entering lanes' first iteration in the boundary stage" if same_tick
+                       else "entering lanes join the loop step at the next tick",
         "early_exit_tokens": exited,
         "early_exit_fired": exited > 0,
         "kernel_time": kinds,

@@ -148,6 +148,10 @@ class LoopedLM:
                                  C.byref(rounds)), "tl_speculate")
         return tok, rounds.value
 
+    def set_tick_overlap(self, mode: int):
+        """0 automatic, 1 entering lanes iterate in the boundary stage, 2 they join at the next tick."""
+        check(lib().tl_set_tick_overlap(self.h, mode), "tl_set_tick_overlap")
+
     def set_cascade(self, enabled: bool):
         check(lib().tl_set_cascade(self.h, 1 if enabled else 0), "tl_set_cascade")
 

@@ -31,7 +31,7 @@ class TlStats(C.Structure):
     _fields_ = [
         ("loop_steps", C.c_int64), ("lane_iterations", C.c_int64), ("tokens_emitted", C.c_int64),
         ("prefill_tokens", C.c_int64), ("kernel_launches", C.c_int64), ("device_status", C.c_int32),
-        ("kv_pages_used", C.c_int32),
+        ("kv_pages_used", C.c_int32), ("entry_in_boundary", C.c_int32),
     ]
 
 
@@ -60,6 +60,7 @@ SIGNATURES = {
                               C.c_void_p]),
     "tl_speculate": (C.c_int, [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p,
                                C.c_void_p]),
+    "tl_set_tick_overlap": (C.c_int, [C.c_void_p, C.c_int32]),
     "tl_set_cascade": (C.c_int, [C.c_void_p, C.c_int32]),
     "tl_set_graphs": (C.c_int, [C.c_void_p, C.c_int32]),
     "tl_lane_state_bytes": (C.c_int, [C.c_void_p, C.POINTER(C.c_size_t)]),

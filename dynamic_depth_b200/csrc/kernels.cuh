@@ -150,8 +150,10 @@ __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, in
 // The three row tables of a decode tick from the lane states at its start,
 // in lane order, decided one stage ahead: boundary rows (loop finished: head,
 // token), entered rows (boundary lanes that will take a token and continue:
-// their pre blocks run at position pos + 1) and loop rows (lanes in their loop
-// plus the entering lanes at iteration 0).  Whether a boundary lane continues
+// their pre blocks and first loop iteration run at position pos + 1, in the
+// boundary stage) and loop rows (lanes already in their loop), so the
+// boundary stage and the loop step touch disjoint lanes and run
+// concurrently.  Whether a boundary lane continues
 // is fixed before its head runs, by the same test head_finalize_kernel applies
 // (n_emitted + 1 < n_target and pos + 1 < max_seq).  alive = lanes in their
 // loop or at a boundary.  With conditional graph nodes, sets the SWITCH value
@@ -179,7 +181,7 @@ __global__ void plan_tick_kernel(const LaneState* __restrict__ lanes, int n_lane
     const bool e = b && st.n_emitted + 1 < st.n_target && st.pos + 1 < max_seq;
     take[0] = b;
     take[1] = e;
-    take[2] = st.phase == PH_LOOP || e;
+    take[2] = st.phase == PH_LOOP;  // entering lanes join the loop at the next tick
     live = st.phase == PH_LOOP || b;
   }
   unsigned bal[3];
@@ -211,7 +213,7 @@ __global__ void plan_tick_kernel(const LaneState* __restrict__ lanes, int n_lane
   for (int t = 0; t < 3; ++t) {
     if (take[t]) {
       const int r = (w == 0 ? 0 : cnt[t][w - 1]) + __popc(bal[t] & below);
-      const bool fresh = t == 1 || (t == 2 && take[1]);  // entering: next position, iteration 0
+      const bool fresh = t == 1;  // entering: next position, iteration 0
       tab[t]->lane[r] = i;
       tab[t]->pos[r] = fresh ? pos + 1 : pos;
       tab[t]->iter[r] = fresh ? 0 : iter;

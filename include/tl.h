@@ -101,6 +101,9 @@ typedef struct tl_stats {
     int64_t kernel_launches;     /* kernels this library launched               */
     int32_t device_status;       /* last status word read back (0 = clean)      */
     int32_t kv_pages_used;
+    int32_t entry_in_boundary;   /* the last decode ran entering lanes' first loop
+                                    iteration in the boundary stage (1) or at the
+                                    next tick (0); see tl_set_tick_overlap      */
 } tl_stats;
 
 /* ---------------------------------------------------------------- sizes -- */
@@ -325,6 +328,21 @@ int tl_generate(tl_ctx* ctx, const int32_t* host_prompts, int32_t n_lanes, int32
  * its cache; TL_EINVAL on bad arguments. */
 int tl_speculate(tl_ctx* ctx, int32_t lane, int32_t n_new, int32_t L_draft, int32_t L_verify, int32_t draft_ahead,
                  int32_t* host_tokens_out, int32_t* host_rounds_out);
+
+/* Layout of a decode tick ("Depth-adaptive Inference of Looped Language
+ * Models via Continuous Depth Batching": boundary stages queued apart from
+ * loop steps, with scheduling overlapping GPU work).  Every tick runs two
+ * concurrent branches on disjoint lanes: the boundary stage (head, greedy
+ * token, embedding and pre blocks of the lanes whose loop finished) and one
+ * loop iteration of the lanes in their loop.  mode 1: a lane that takes a
+ * token also runs its first loop iteration in that boundary stage (a token
+ * costs its depth in ticks); mode 2: it joins the loop step at the next tick
+ * (one tick more per token, a shorter boundary stage); mode 0 (default)
+ * chooses per decode call: mode 2 for 32+ lanes with mean requested L of 6 or
+ * more, mode 1 otherwise.  Results per lane do not depend on it beyond the
+ * rounding differences of batch width (see tl_stats.entry_in_boundary).
+ * TL_EINVAL for other modes. */
+int tl_set_tick_overlap(tl_ctx* ctx, int32_t mode);
 
 /* Shared-prefix ("cascade") attention in decode steps (default on; "Benchmark
  * Comparison" (measured benchmarks), section 2: one cached prefix serves many

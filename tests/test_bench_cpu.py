@@ -46,6 +46,50 @@ def _simulate(depths, T, n_pre, d):
     return boundary, entered, loop_rows, attn
 
 
+def _simulate_next_tick(depths, T, n_pre, d):
+    """Entering lanes run their loop from the next tick on: each tick, the lanes
+    in their loop at its start run one iteration while the waiting lanes take a
+    token (concurrently, on disjoint lanes)."""
+    n, n_new = depths.shape
+    nxt, left, done = [1] * n, [0] * n, [False] * n
+    boundary, entered, loop_rows, attn = [], [], [], 0
+    while not all(done):
+        looping = [i for i in range(n) if not done[i] and left[i] > 0]
+        waiting = [i for i in range(n) if not done[i] and left[i] == 0]
+        for i in looping:
+            left[i] -= 1
+        b = e = 0
+        for i in waiting:
+            b += 1
+            if nxt[i] >= n_new:
+                done[i] = True
+                continue
+            e += 1
+            left[i] = int(depths[i, nxt[i]])
+            attn += (n_pre + left[i]) * (T + nxt[i]) * 4 * d
+            nxt[i] += 1
+        boundary.append(b)
+        entered.append(e)
+        loop_rows.append(len(looping))
+    return boundary, entered, loop_rows, attn
+
+
+def test_schedule_counts_match_a_tick_by_tick_simulation_next_tick_entry():
+    rng = np.random.Generator(np.random.PCG64(6))
+    n, n_new, T = 7, 6, 20
+    depths = rng.integers(1, 6, (n, n_new)).astype(np.int32)
+
+    class Wl:
+        prompt_len, n_new = T, 6
+    u = bench.schedule_units(S.M407, Wl, depths, same_tick=False)
+    b, e, rows, attn = _simulate_next_tick(depths, T, S.M407.n_pre, S.M407.d)
+    assert u["ticks"] == len(b)
+    assert list(u["boundary"]) == b
+    assert list(u["entered"]) == e
+    assert list(u["loop_rows"]) == rows
+    assert u["attn_bytes"] == attn
+
+
 def test_schedule_counts_match_a_tick_by_tick_simulation():
     rng = np.random.Generator(np.random.PCG64(5))
     n, n_new, T = 7, 6, 20

@@ -191,3 +191,21 @@ def test_m407_wide_decode_logits():
     for i in range(16):
         for t in range(3):
             assert_logits_close(lg[i, t], ref[i].logits[t], f"lane {i} token {t}")
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_tiny_tick_layouts_match_oracle(mode):
+    # both layouts of a decode tick (entering lanes' first iteration in the boundary stage, or at the next
+    # tick beside the other lanes' loop step) give each lane its own schedule and tokens
+    W = oracle_weights("tiny", 7)
+    P = S.prompts(16, 12, 512, seed=75)
+    Ls = [1, 2, 3, 4, 5, 6, 7, 8] * 2
+    m = gpu_model("tiny", 7, max_lanes=16, max_seq=32, L_max=8)
+    m.set_tick_overlap(mode)
+    tok, dep = m.generate(P, Ls, 7)
+    st = status_clean(m)
+    assert st["entry_in_boundary"] == (1 if mode == 1 else 0)
+    for i in range(16):
+        r = D.generate_lane(W, P[i], Ls[i], 7)
+        assert dep[i].tolist() == r.depths.tolist()
+        _check_tokens(r.tokens, r.logits, tok[i])
