@@ -346,8 +346,11 @@ struct tl_ctx {
   int overlap_mode = 0;   // tl_set_tick_overlap: 0 automatic, 1 entering lanes iterate in the boundary stage, 2 next tick
   int entry_iter = 1;     // resolved for the running decode: 1 = first iteration in the boundary stage
   int64_t tick_launches = 0;
+  int64_t tick_loop_kernels = 0;  // plain kernel nodes of a tick graph (outside conditional bodies)
   bool graphs_enabled = true;
   bool pdl = true;  // programmatic dependent launch between consecutive kernels
+  int prio = 0;     // launch priority of the next kernels (0: the stream's)
+  int prio_hi = 0;  // the device's highest priority: a decode tick's boundary stage
   // host state
   std::vector<int32_t> h_page_table;  // [lanes][slots][pages]
   std::vector<int32_t> refcount;      // per page
@@ -387,11 +390,20 @@ int launch_k(tl_ctx* c, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
   lc.blockDim = block;
   lc.dynamicSmemBytes = smem;
   lc.stream = c->stream;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  if (c->pdl) {
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (c->prio) {
+    at[na].id = cudaLaunchAttributePriority;
+    at[na].val.priority = c->prio;
+    ++na;
+  }
   lc.attrs = at;
-  lc.numAttrs = c->pdl ? 1 : 0;
+  lc.numAttrs = na;
   TL_CUDA(cudaLaunchKernelEx(&lc, kern, args...));
   return launch_err(c);
 }
@@ -500,15 +512,24 @@ int tc_launch_t(tl_ctx* c, const CUtensorMap& mw, const CUtensorMap& mw2, const 
   lc.blockDim = dim3(256, 1, 1);
   lc.dynamicSmemBytes = Cf::SMEM;
   lc.stream = c->stream;
-  cudaLaunchAttribute at[2];
+  cudaLaunchAttribute at[3];
   at[0].id = cudaLaunchAttributeClusterDimension;  // the split-K CTAs of a tile share a cluster
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = grid.z;
-  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = 1;
+  int na = 1;
+  if (c->pdl) {
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (c->prio) {
+    at[na].id = cudaLaunchAttributePriority;
+    at[na].val.priority = c->prio;
+    ++na;
+  }
   lc.attrs = at;
-  lc.numAttrs = c->pdl ? 2 : 1;
+  lc.numAttrs = na;
   TL_CUDA(cudaLaunchKernelEx(&lc, kern, mw, mw2, mx, p));
   return launch_err(c);
 }
@@ -1285,6 +1306,8 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
       c->n_sms = sms;
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess) c->prio_hi = hi;
     c->scr[0].gs_ctas = c->n_sms;
     c->scr[1].gs_ctas = c->n_sms;
     const GsChoice g = gs_plan(c->head.fmt, c->head.N, c->head.K, c->head.group, 1, c->n_sms);
@@ -1793,10 +1816,12 @@ static int plan_tick(tl_ctx* c, int n_lanes, const TickConds& tc) {
 static int enqueue_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
   TL_TRY(plan_tick(c, n_lanes, TickConds{}));
   c->sc = &c->scr[1];
+  c->prio = c->prio_hi;
   int st = head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_AUTO, 0);
   if (st == TL_OK) st = pre_blocks(c, n_lanes);
   if (st == TL_OK && c->entry_iter) st = loop_iteration(c, n_lanes, nullptr, PATH_AUTO, 2);
   c->sc = &c->scr[0];
+  c->prio = 0;
   TL_TRY(st);
   return loop_iteration(c, n_lanes, nullptr);
 }
@@ -1859,13 +1884,16 @@ static int capture_body(tl_ctx* c, cudaGraph_t body, int64_t* n_kernels, F fn) {
 // parameters.
 //   plan -+-> SWITCH { norm, head, argmax + token + embedding: GEMV | tensor cores }
 //         |     -> SWITCH { entering lanes: pre blocks + first loop iteration: GEMV | TC }  (boundary scratch)
-//         +-> SWITCH { loop body + exit rule of the other lanes: GEMV | tensor cores }    (main scratch)
+//         +-> loop body + exit rule of the other lanes: plain nodes (both variants) for a body of
+//             <= 2 layers, else SWITCH { GEMV | tensor cores }                            (main scratch)
 //   (the two branches join at the end of the tick: "Depth-adaptive Inference of Looped Language Models via
 //   Continuous Depth Batching", boundary stages queued apart from loop steps, overlapped with them)
 static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out, int32_t* kcount) {
   TickConds tc{};
-  for (int t = 0; t < 3; ++t) TL_TRY(new_handle(c->stream, &tc.h[t]));
-  tc.use = 7;
+  // a short loop body runs as plain kernel nodes (below), so its handle is not needed
+  const bool plain_loop = c->cfg.n_loop_layers <= 2;
+  for (int t = 0; t < (plain_loop ? 2 : 3); ++t) TL_TRY(new_handle(c->stream, &tc.h[t]));
+  tc.use = plain_loop ? 3 : 7;
   TL_TRY(plan_tick(c, n_lanes, tc));
   cudaGraph_t body[2];
   int64_t nk[2] = {0, 0};
@@ -1875,6 +1903,9 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
   TL_CUDA(cudaStreamWaitEvent(c->cap_stream2, c->fork_ev, 0));
   c->stream = c->cap_stream2;
   c->sc = &c->scr[1];
+  // the boundary stage's kernels at the device's highest priority: their CTAs are dispatched ahead of the
+  // loop step's pending ones
+  c->prio = c->prio_hi;
   // boundary rows -> head (CUDA-core GEMV for <= 8 rows, tensor cores above)
   TL_TRY(add_conditional(c->stream, tc.h[0], cudaGraphCondTypeSwitch, 2, body));
   TL_TRY(capture_body(c, body[0], &nk[0], [&] {
@@ -1901,12 +1932,27 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
   TL_CUDA(cudaEventRecord(c->join_ev, c->cap_stream2));
   c->stream = main_s;
   c->sc = &c->scr[0];
-  // loop rows -> loop body
-  TL_TRY(add_conditional(c->stream, tc.h[2], cudaGraphCondTypeSwitch, 2, body));
-  TL_TRY(capture_body(c, body[0], &nk[0], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_GEMV); }));
-  TL_TRY(capture_body(c, body[1], &nk[1], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_TC); }));
-  kcount[4] = (int32_t)nk[0];
-  kcount[5] = (int32_t)nk[1];
+  c->prio = 0;
+  // loop rows -> loop body.  The bodies of a graph's conditional nodes were measured to start one after
+  // another (each once the previous body's last kernel was launched), which kept this branch waiting for
+  // the boundary stage's head.  So a short body runs as plain kernel nodes, which start at once, with both
+  // projection variants captured (the one that does not apply to the device-side row count returns at
+  // once); a long body (the 24-layer one) keeps its conditional node, where doubling every projection's
+  // launches measured slower (7.0k against 7.9k tokens/s on 256 lanes).  Plain nodes for the boundary
+  // stage too measured slower again (2.0k against 1.8k tokens/s for one lane at L = 8).
+  c->tick_loop_kernels = 0;
+  kcount[4] = kcount[5] = 0;
+  if (plain_loop) {
+    const int64_t l0 = c->launches;
+    TL_TRY(loop_iteration(c, n_lanes, nullptr, PATH_AUTO));
+    c->tick_loop_kernels = c->launches - l0;
+  } else {
+    TL_TRY(add_conditional(c->stream, tc.h[2], cudaGraphCondTypeSwitch, 2, body));
+    TL_TRY(capture_body(c, body[0], &nk[0], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_GEMV); }));
+    TL_TRY(capture_body(c, body[1], &nk[1], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_TC); }));
+    kcount[4] = (int32_t)nk[0];
+    kcount[5] = (int32_t)nk[1];
+  }
   TL_CUDA(cudaStreamWaitEvent(c->stream, c->join_ev, 0));
   return TL_OK;
 }
@@ -1928,6 +1974,7 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   const int st = capture_tick(c, n_lanes, n_new, tok_out, dep_out, kcount);
   c->stream = saved;
   c->sc = &c->scr[0];
+  c->prio = 0;
   cudaGraph_t g = nullptr;
   const cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
   c->launches = l0;
@@ -1951,7 +1998,7 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   c->tick_warm = c->warm;
   c->tick_cascade = c->cascade_active;
   c->tick_entry = c->entry_iter;
-  c->tick_launches = 1;  // the planning kernel outside the conditional bodies
+  c->tick_launches = 1 + c->tick_loop_kernels;  // the planning kernel and the loop step's plain nodes
   return TL_OK;
 }
 
