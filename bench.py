@@ -130,6 +130,14 @@ def loop_block_weight_bytes(sh) -> int:
     return sum(n * k // 2 + n * (k // g) * 2 for n, k in [(3 * d, d), (d, d), (F, d), (F, d), (d, F)])
 
 
+TICK_LAYOUTS = {
+    1: "ticks of boundary stage + loop step; entering lanes' first iteration in the boundary stage",
+    2: "ticks of boundary stage + loop step; entering lanes join the loop step at the next tick",
+    3: "boundary stages on their own stream, apart from the loop steps (no join per tick); the per-kind "
+       "profiled pass launches kernels individually and so runs layout 2, whose schedule ticks_per_step counts",
+}
+
+
 def schedule_units(sh, wl, depths, same_tick: bool = True):
     """Counts behind the algorithmic bytes, from the executed depth schedule.
 
@@ -204,6 +212,7 @@ def run_ours(args, rank, world, local_rank):
     m.set_early_exit(wl.ee_tau, wl.ee_min_L, wl.ee_patience, wl.ee_peek_every)
     if args.eager:
         m.set_graphs(False)
+    m.set_tick_overlap(args.tick_layout)
     P = S.prompts(wl.n_lanes, wl.prompt_len, sh.vocab)
     Ls = np.array(wl.per_lane_L, dtype=np.int32)
 
@@ -370,8 +379,8 @@ def run_ours(args, rank, world, local_rank):
         "lane_iterations_no_exit": int(sum(int(L) * (wl.n_new - 1) for L in Ls)),
         "depth_histogram": {int(k): int(v) for k, v in zip(*np.unique(depths[:, 1:], return_counts=True))},
         "ticks_per_step": units["ticks"],
-        "tick_layout": "entering lanes' first iteration in the boundary stage" if same_tick
-                       else "entering lanes join the loop step at the next tick",
+        "loop_steps_per_step": int(st1["loop_steps"] - st0["loop_steps"]) // args.steps,
+        "tick_layout": TICK_LAYOUTS.get(int(st1["tick_layout"]), str(st1["tick_layout"])),
         "early_exit_tokens": exited,
         "early_exit_fired": exited > 0,
         "kernel_time": kinds,
@@ -398,7 +407,11 @@ def _build_model(sh, dev, **capacity):
     cfg = T.config_from_shape(sh, **capacity)
     m = T.LoopedLM(cfg, dev)
     m.load_weights(Wt.build_blob(cfg, S.master_weights(sh), S.gains(sh), dev))
+    m.set_tick_overlap(_TICK_LAYOUT[0])
     return m
+
+
+_TICK_LAYOUT = [0]  # --tick-layout for every workload
 
 
 class L2Flush:
@@ -884,8 +897,11 @@ def main():
     ap.add_argument("--lanes", type=int, default=0, help="reduced case: lanes (profiling captures only)")
     ap.add_argument("--prompt-len", type=int, default=0, help="reduced case: prompt tokens")
     ap.add_argument("--new-tokens", type=int, default=0, help="reduced case: generated tokens")
+    ap.add_argument("--tick-layout", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="decode tick layout (tl_set_tick_overlap); 0 = the library's choice")
     ap.add_argument("--workload", choices=["cdb64", "tiny", "prefill128", "lsweep", "prefix256"], default="cdb64")
     args = ap.parse_args()
+    _TICK_LAYOUT[0] = args.tick_layout
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

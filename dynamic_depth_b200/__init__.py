@@ -149,7 +149,8 @@ class LoopedLM:
         return tok, rounds.value
 
     def set_tick_overlap(self, mode: int):
-        """0 automatic, 1 entering lanes iterate in the boundary stage, 2 they join at the next tick."""
+        """0 automatic, 1 entering lanes iterate in the boundary stage, 2 they join at the next tick,
+        3 boundary stages and loop steps on two streams with no join per tick."""
         check(lib().tl_set_tick_overlap(self.h, mode), "tl_set_tick_overlap")
 
     def set_cascade(self, enabled: bool):

@@ -21,7 +21,22 @@ enum : int32_t {
   ST_BAD_ROW = 1 << 5,      // row table larger than its buffers
 };
 
-enum LanePhase : int32_t { PH_IDLE = 0, PH_LOOP = 1, PH_BOUNDARY = 2, PH_DONE = 3 };
+// PH_CLAIMED: taken by a boundary stage that runs apart from the loop steps
+// (asynchronous decode stages); the stage hands the lane back as PH_LOOP when
+// its pre blocks are done, or retires it as PH_DONE.
+enum LanePhase : int32_t { PH_IDLE = 0, PH_LOOP = 1, PH_BOUNDARY = 2, PH_DONE = 3, PH_CLAIMED = 4 };
+
+// A lane's phase is the hand-off word between concurrently running stages:
+// the writer orders every other write of the lane before it (release), the
+// reader reads it before the lane's other fields (acquire).
+__device__ __forceinline__ int32_t phase_acquire(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void phase_release(int32_t* p, int32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // One lane's scheduling state, resident in device memory.
 struct LaneState {

@@ -157,32 +157,38 @@ __global__ void build_rows_kernel(LaneState* __restrict__ lanes, int n_lanes, in
 // is fixed before its head runs, by the same test head_finalize_kernel applies
 // (n_emitted + 1 < n_target and pos + 1 < max_seq).  alive = lanes in their
 // loop or at a boundary.  With conditional graph nodes, sets the SWITCH value
-// of each table whose bit is set in cond.use, as build_rows_kernel does.  One
-// CTA of 1024 threads; thread i looks at lane i.
+// of each table whose bit is set in cond.use, as build_rows_kernel does.
+// which: bit 0 plans the boundary and entered tables, bit 1 the loop table
+// and the alive count (both: one tick); a boundary plan alone (the stage runs
+// apart from the loop steps) also claims its lanes (PH_CLAIMED), and alive
+// then counts claimed lanes too.  alive[1] = loop rows.  One CTA of 1024
+// threads; thread i looks at lane i.
 struct TickConds {
   cudaGraphConditionalHandle h[3];  // boundary, entered, loop
   int32_t use;                      // bit t: h[t] is a live handle
 };
 
-__global__ void plan_tick_kernel(const LaneState* __restrict__ lanes, int n_lanes, Rows boundary, Rows entered,
-                                 Rows loop, int32_t* __restrict__ alive, int max_seq, TickConds cond,
-                                 int32_t gemv_max_rows, const int32_t* __restrict__ body_kernels,
-                                 unsigned long long* __restrict__ kernel_count) {
+__global__ void plan_tick_kernel(LaneState* lanes, int n_lanes, Rows boundary, Rows entered, Rows loop,
+                                 int32_t* __restrict__ alive, int max_seq, TickConds cond, int32_t gemv_max_rows,
+                                 const int32_t* __restrict__ body_kernels,
+                                 unsigned long long* __restrict__ kernel_count, int32_t which) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ int32_t cnt[3][32];
   const int i = threadIdx.x, lane = i & 31, w = i >> 5;
   int take[3] = {0, 0, 0}, live = 0, pos = 0, iter = 0;
   if (i < n_lanes) {
+    const int ph = phase_acquire(&lanes[i].phase);
     const LaneState st = lanes[i];
     pos = st.pos;
     iter = st.iter;
-    const bool b = st.phase == PH_BOUNDARY;
+    const bool b = ph == PH_BOUNDARY;
     const bool e = b && st.n_emitted + 1 < st.n_target && st.pos + 1 < max_seq;
-    take[0] = b;
-    take[1] = e;
-    take[2] = st.phase == PH_LOOP;  // entering lanes join the loop at the next tick
-    live = st.phase == PH_LOOP || b;
+    take[0] = (which & 1) && b;
+    take[1] = (which & 1) && e;
+    take[2] = (which & 2) && ph == PH_LOOP;  // entering lanes join the loop at the next tick
+    live = ph == PH_LOOP || b || ph == PH_CLAIMED;
+    if (which == 1 && b) lanes[i].phase = PH_CLAIMED;
   }
   unsigned bal[3];
 #pragma unroll
@@ -224,9 +230,12 @@ __global__ void plan_tick_kernel(const LaneState* __restrict__ lanes, int n_lane
 #pragma unroll
     for (int t = 0; t < 3; ++t) {
       n[t] = cnt[t][31];
-      tab[t]->n[0] = n[t];
+      if ((which >> (t == 2 ? 1 : 0)) & 1) tab[t]->n[0] = n[t];
     }
-    if (alive) alive[0] = live_cnt[0];
+    if (alive && (which & 2)) {
+      alive[0] = live_cnt[0];
+      alive[1] = n[2];
+    }
     unsigned long long k = 0;
 #pragma unroll
     for (int t = 0; t < 3; ++t) {
@@ -770,8 +779,8 @@ __global__ void exit_update_kernel(Rows rows, LaneState* __restrict__ lanes, con
     st.iter = l;
     const bool fin = ex || l >= st.L_run;
     if (fin) {
-      st.phase = PH_BOUNDARY;
       st.depth = l;
+      phase_release(&st.phase, PH_BOUNDARY);  // a boundary stage may take the lane from here on
     }
     if (exit_mask_out) exit_mask_out[ln] = fin ? 1 : 0;
     if (lane_iters) atomicAdd(lane_iters, 1ull);
@@ -888,7 +897,7 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
                                      int32_t* __restrict__ argmax_out, int32_t* __restrict__ tokens_out,
                                      int32_t* __restrict__ depths_out, int n_new, MatView E, float* __restrict__ h,
                                      int d, int max_seq, int32_t mark_entered, int32_t* __restrict__ status,
-                                     unsigned long long* __restrict__ tok_count, WarmParams wp) {
+                                     unsigned long long* __restrict__ tok_count, WarmParams wp, int32_t hold) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float sv[32];
@@ -940,7 +949,7 @@ __global__ void head_finalize_kernel(Rows rows, LaneState* __restrict__ lanes, c
         st.iter = 0;
         st.streak = 0;
         st.token = bi;
-        st.phase = PH_LOOP;
+        st.phase = hold ? PH_CLAIMED : PH_LOOP;  // held: release_rows_kernel hands it to the loop
         st.entered = mark_entered;
         go_s = 1;
       }
@@ -984,6 +993,17 @@ __global__ void embed_next_kernel(LaneState* __restrict__ lanes, int n_lanes, co
   }
   __syncthreads();
   if (go_s) embed_row(E, tok_s, h + (int64_t)ln * d, d);
+}
+
+// End of a boundary stage that runs apart from the loop steps: the entered
+// lanes (their token, embedding and pre blocks done by the kernels before this
+// one) go to the loop.  One thread per row.
+__global__ void release_rows_kernel(Rows rows, LaneState* lanes) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows.n[0]) return;
+  phase_release(&lanes[rows.lane[r]].phase, PH_LOOP);
 }
 
 // Lanes of a decode call: set the request and token budget.  A request above

@@ -242,7 +242,7 @@ static Layout make_layout(const tl_config* c) {
   L.status = take(4);
   L.counters = take(4 * 8);
   L.body_kernels = take(8 * 4);
-  L.alive = take(4);
+  L.alive = take(8);  // alive lanes, loop rows
   // the decode boundary stage's own scratch (rows = lanes)
   L.b_act_a = take(lanes * d * 4);
   L.b_act_qkv = take(lanes * 3 * d * 4);
@@ -342,9 +342,17 @@ struct tl_ctx {
   EEParams tick_ee{};
   WarmParams tick_warm{};
   bool tick_cascade = false;
-  int tick_entry = -1;
-  int overlap_mode = 0;   // tl_set_tick_overlap: 0 automatic, 1 entering lanes iterate in the boundary stage, 2 next tick
+  int tick_entry = -1, tick_layout = 0;
+  int overlap_mode = 0;   // tl_set_tick_overlap: 0 automatic, 1 entering lanes iterate in the boundary stage, 2 next
+                          // tick, 3 boundary stages apart from the loop steps
   int entry_iter = 1;     // resolved for the running decode: 1 = first iteration in the boundary stage
+  int layout = 1;         // resolved for the running decode: 1, 2 or 3 as overlap_mode
+  // asynchronous stages (layout 3): the loop step's graph on `stream`, the boundary stage's on bstream
+  cudaStream_t bstream = nullptr;
+  cudaEvent_t b_ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  cudaGraphExec_t loop_exec = nullptr, bnd_exec = nullptr;
+  int64_t loop_launches = 0, bnd_launches = 0;  // plain kernel nodes of each
+  int hold_entered = 0;   // head_finalize keeps continuing lanes claimed (boundary stage of layout 3)
   int64_t tick_launches = 0;
   int64_t tick_loop_kernels = 0;  // plain kernel nodes of a tick graph (outside conditional bodies)
   bool graphs_enabled = true;
@@ -356,7 +364,7 @@ struct tl_ctx {
   std::vector<int32_t> refcount;      // per page
   std::vector<int32_t> free_pages;
   std::vector<int32_t> lane_L;        // prefill depth per lane (0 = empty)
-  int32_t* pinned_alive = nullptr;    // ring of alive counts
+  int32_t* pinned_alive = nullptr;    // ring of (alive lanes, loop rows)
   cudaEvent_t alive_ev[4];
   int64_t steps = 0, prefill_tokens = 0, launches = 0;
   // profiling ring (tl_profile_begin / tl_profile_end)
@@ -368,6 +376,7 @@ struct tl_ctx {
 };
 
 static constexpr int kAliveRing = 4;
+static constexpr int kBRing = 4;  // boundary stages queued at once, at most (layout 3)
 static constexpr int kProfRing = 4096;
 
 namespace {
@@ -976,7 +985,7 @@ int head_core(tl_ctx* c, int max_rows, int mode, float* logits, int32_t* argmax,
   TL_TRY(launch_k(c, head_finalize_kernel, dim3(max_rows), dim3(256), 0, B, c->lanes, c->sc->part_val, c->sc->part_idx, c->sc->head_nparts, mode,
                                                         argmax, tok_out, dep_out, n_new, c->embed, c->h, c->cfg.d,
                                                         c->cfg.max_seq, mark_entered, c->status, &c->counters[1],
-                                                        c->warm));
+                                                        c->warm, (int32_t)c->hold_entered));
   return TL_OK;
 }
 
@@ -1343,7 +1352,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     for (int i = 0; i < 6; ++i)
       if ((st = check_cuda(cudaMemsetAsync(c->rows[i].n, 0, 4, c->stream))) != TL_OK) break;
     if (st != TL_OK) break;
-    if ((st = check_cuda(cudaHostAlloc((void**)&c->pinned_alive, kAliveRing * sizeof(int32_t), cudaHostAllocDefault))) != TL_OK) break;
+    if ((st = check_cuda(cudaHostAlloc((void**)&c->pinned_alive, 2 * kAliveRing * sizeof(int32_t), cudaHostAllocDefault))) != TL_OK) break;
     for (int i = 0; i < kAliveRing; ++i)
       if ((st = check_cuda(cudaEventCreateWithFlags(&c->alive_ev[i], cudaEventDisableTiming))) != TL_OK) break;
     if (st != TL_OK) break;
@@ -1352,6 +1361,10 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     if ((st = check_cuda(cudaStreamCreateWithFlags(&c->cap_stream2, cudaStreamNonBlocking))) != TL_OK) break;
     if ((st = check_cuda(cudaEventCreateWithFlags(&c->fork_ev, cudaEventDisableTiming))) != TL_OK) break;
     if ((st = check_cuda(cudaEventCreateWithFlags(&c->join_ev, cudaEventDisableTiming))) != TL_OK) break;
+    if ((st = check_cuda(cudaStreamCreateWithFlags(&c->bstream, cudaStreamNonBlocking))) != TL_OK) break;
+    for (int i = 0; i < kBRing; ++i)
+      if ((st = check_cuda(cudaEventCreateWithFlags(&c->b_ev[i], cudaEventDisableTiming))) != TL_OK) break;
+    if (st != TL_OK) break;
   } while (0);
   if (st != TL_OK) {
     if (c->pinned_alive) cudaFreeHost(c->pinned_alive);
@@ -1371,6 +1384,11 @@ extern "C" int tl_destroy(tl_ctx* c) {
   if (c->cap_stream2) cudaStreamDestroy(c->cap_stream2);
   if (c->fork_ev) cudaEventDestroy(c->fork_ev);
   if (c->join_ev) cudaEventDestroy(c->join_ev);
+  if (c->loop_exec) cudaGraphExecDestroy(c->loop_exec);
+  if (c->bnd_exec) cudaGraphExecDestroy(c->bnd_exec);
+  if (c->bstream) cudaStreamDestroy(c->bstream);
+  for (int i = 0; i < kBRing; ++i)
+    if (c->b_ev[i]) cudaEventDestroy(c->b_ev[i]);
   for (int i = 0; i < kAliveRing; ++i) cudaEventDestroy(c->alive_ev[i]);
   for (auto& e : c->prof_ev) {
     cudaEventDestroy(e[0]);
@@ -1682,7 +1700,7 @@ static int head_hrows(tl_ctx* c, int k, int32_t* dev_argmax) {
   return launch_k(c, head_finalize_kernel, dim3(k), dim3(256), 0, T4, c->lanes, (const float*)c->sc->part_val,
                   (const int32_t*)c->sc->part_idx, (const int32_t*)c->sc->head_nparts, (int32_t)HEAD_ONLY, dev_argmax,
                   (int32_t*)nullptr, (int32_t*)nullptr, 0, c->embed, c->h, c->cfg.d, c->cfg.max_seq, 0, c->status,
-                  (unsigned long long*)nullptr, c->warm);
+                  (unsigned long long*)nullptr, c->warm, (int32_t)0);
 }
 
 static int speculate_impl(tl_ctx* c, int lane, int n_new, int Ld, int Lv, int ahead, int32_t* out, int32_t* rounds_out) {
@@ -1803,9 +1821,9 @@ extern "C" int tl_embed_next(tl_ctx* c, const uint8_t* dev_mask, const int32_t* 
 // The tick's three row tables (boundary -> rows[1], entered -> rows[2],
 // loop -> rows[0]) and alive count from one kernel; with conditional nodes it
 // also chooses their bodies.
-static int plan_tick(tl_ctx* c, int n_lanes, const TickConds& tc) {
+static int plan_tick(tl_ctx* c, int n_lanes, const TickConds& tc, int32_t which = 3) {
   return launch_k(c, plan_tick_kernel, dim3(1), dim3(1024), 0, c->lanes, n_lanes, c->rows[1], c->rows[2], c->rows[0],
-                  c->alive, c->cfg.max_seq, tc, kGemvMaxRows, c->body_kernels, &c->counters[2]);
+                  c->alive, c->cfg.max_seq, tc, kGemvMaxRows, c->body_kernels, &c->counters[2], which);
 }
 
 // One decode tick: the boundary stage (head, tokens, embedding, pre blocks
@@ -1957,36 +1975,118 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
   return TL_OK;
 }
 
-static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
-  if (c->tick_exec && c->tick_lanes == n_lanes && c->tick_new == n_new && c->tick_tok == tok_out &&
-      c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee) && c->tick_warm.tokens == c->warm.tokens &&
-      c->tick_warm.L == c->warm.L && c->tick_cascade == c->cascade_active && c->tick_entry == c->entry_iter)
-    return TL_OK;
-  if (c->tick_exec) {
-    cudaGraphExecDestroy(c->tick_exec);
-    c->tick_exec = nullptr;
+// Layout 3 ("Depth-adaptive Inference of Looped Language Models via
+// Continuous Depth Batching": boundary stages queued apart from the loop
+// steps): two graphs on two streams with no join per tick.  The loop step's
+// graph plans the lanes in their loop and runs one iteration for them; the
+// boundary stage's graph claims the lanes whose loop finished, runs their
+// head, token and embedding and, for those that continue, their pre blocks,
+// then hands them to the loop (release_rows_kernel).  A lane's phase word
+// orders the hand-offs, so a lane's own steps keep their order while the two
+// streams run side by side at their own cadence.
+static int capture_loop_step(tl_ctx* c, int n_lanes, int32_t* kcount) {
+  TickConds tc{};
+  const bool plain_loop = c->cfg.n_loop_layers <= 2;  // as in the tick graph
+  if (!plain_loop) TL_TRY(new_handle(c->stream, &tc.h[2]));
+  tc.use = plain_loop ? 0 : 4;
+  const int64_t l0 = c->launches;
+  TL_TRY(plan_tick(c, n_lanes, tc, 2));
+  if (plain_loop) {
+    TL_TRY(loop_iteration(c, n_lanes, nullptr, PATH_AUTO));
+  } else {
+    cudaGraph_t body[2];
+    int64_t nk[2] = {0, 0};
+    TL_TRY(add_conditional(c->stream, tc.h[2], cudaGraphCondTypeSwitch, 2, body));
+    TL_TRY(capture_body(c, body[0], &nk[0], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_GEMV); }));
+    TL_TRY(capture_body(c, body[1], &nk[1], [&] { return loop_iteration(c, n_lanes, nullptr, PATH_TC); }));
+    kcount[4] = (int32_t)nk[0];
+    kcount[5] = (int32_t)nk[1];
   }
-  const int64_t l0 = c->launches, s0 = c->steps;
-  int32_t kcount[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  c->loop_launches = c->launches - l0;  // plain nodes (kernels in the chosen body are counted on the device)
+  return TL_OK;
+}
+
+static int capture_boundary_stage(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out,
+                                  int32_t* kcount) {
+  TickConds tc{};
+  for (int t = 0; t < 2; ++t) TL_TRY(new_handle(c->stream, &tc.h[t]));
+  tc.use = 3;
+  cudaGraph_t body[2];
+  int64_t nk[2] = {0, 0};
+  const int64_t l0 = c->launches;
+  TL_TRY(plan_tick(c, n_lanes, tc, 1));
+  TL_TRY(add_conditional(c->stream, tc.h[0], cudaGraphCondTypeSwitch, 2, body));
+  TL_TRY(capture_body(c, body[0], &nk[0], [&] {
+    return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_GEMV, 0);
+  }));
+  TL_TRY(capture_body(c, body[1], &nk[1], [&] {
+    return head_core(c, n_lanes, HEAD_DECODE, nullptr, nullptr, tok_out, dep_out, n_new, PATH_TC, 0);
+  }));
+  kcount[0] = (int32_t)nk[0];
+  kcount[1] = (int32_t)nk[1];
+  TL_TRY(add_conditional(c->stream, tc.h[1], cudaGraphCondTypeSwitch, 2, body));
+  TL_TRY(capture_body(c, body[0], &nk[0], [&] { return pre_blocks(c, n_lanes, PATH_GEMV); }));
+  TL_TRY(capture_body(c, body[1], &nk[1], [&] { return pre_blocks(c, n_lanes, PATH_TC); }));
+  kcount[2] = (int32_t)nk[0];
+  kcount[3] = (int32_t)nk[1];
+  TL_TRY(launch_k(c, release_rows_kernel, dim3((n_lanes + 255) / 256), dim3(256), 0, c->rows[2], c->lanes));
+  c->bnd_launches = c->launches - l0;
+  return TL_OK;
+}
+
+// Captures fn() as a graph on cap_stream and instantiates it into *exec.
+template <class F>
+static int capture_graph(tl_ctx* c, cudaGraphExec_t* exec, F fn) {
   cudaStream_t saved = c->stream;
   TL_CUDA(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
   c->stream = c->cap_stream;
-  const int st = capture_tick(c, n_lanes, n_new, tok_out, dep_out, kcount);
+  const int st = fn();
   c->stream = saved;
   c->sc = &c->scr[0];
   c->prio = 0;
+  c->hold_entered = 0;
   cudaGraph_t g = nullptr;
   const cudaError_t e = cudaStreamEndCapture(c->cap_stream, &g);
-  c->launches = l0;
-  c->steps = s0;
   if (st != TL_OK) {
     if (g) cudaGraphDestroy(g);
     return st;
   }
   TL_CUDA(e);
-  const cudaError_t ei = cudaGraphInstantiate(&c->tick_exec, g, 0);
+  const cudaError_t ei = cudaGraphInstantiate(exec, g, 0);
   cudaGraphDestroy(g);
-  TL_CUDA(ei);
+  return check_cuda(ei);
+}
+
+static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
+  const bool async = c->layout == 3;
+  if ((async ? (c->loop_exec && c->bnd_exec) : c->tick_exec != nullptr) && c->tick_lanes == n_lanes &&
+      c->tick_new == n_new && c->tick_tok == tok_out && c->tick_dep == dep_out && same_ee(c->tick_ee, c->ee) &&
+      c->tick_warm.tokens == c->warm.tokens && c->tick_warm.L == c->warm.L &&
+      c->tick_cascade == c->cascade_active && c->tick_entry == c->entry_iter && c->tick_layout == c->layout)
+    return TL_OK;
+  for (cudaGraphExec_t* g : {&c->tick_exec, &c->loop_exec, &c->bnd_exec})
+    if (*g) {
+      cudaGraphExecDestroy(*g);
+      *g = nullptr;
+    }
+  const int64_t l0 = c->launches, s0 = c->steps;
+  int32_t kcount[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int st = TL_OK;
+  if (async) {
+    st = capture_graph(c, &c->loop_exec, [&] { return capture_loop_step(c, n_lanes, kcount); });
+    if (st == TL_OK)
+      st = capture_graph(c, &c->bnd_exec, [&] {
+        c->sc = &c->scr[1];
+        c->prio = c->prio_hi;
+        c->hold_entered = 1;
+        return capture_boundary_stage(c, n_lanes, n_new, tok_out, dep_out, kcount);
+      });
+  } else {
+    st = capture_graph(c, &c->tick_exec, [&] { return capture_tick(c, n_lanes, n_new, tok_out, dep_out, kcount); });
+  }
+  c->launches = l0;
+  c->steps = s0;
+  TL_TRY(st);
   // the row-table kernels add the chosen bodies' kernel counts on the device
   TL_CUDA(cudaMemcpyAsync(c->body_kernels, kcount, sizeof(kcount), cudaMemcpyHostToDevice, c->stream));
   TL_CUDA(cudaStreamSynchronize(c->stream));
@@ -1998,26 +2098,83 @@ static int tick_graph(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32
   c->tick_warm = c->warm;
   c->tick_cascade = c->cascade_active;
   c->tick_entry = c->entry_iter;
+  c->tick_layout = c->layout;
   c->tick_launches = 1 + c->tick_loop_kernels;  // the planning kernel and the loop step's plain nodes
   return TL_OK;
 }
 
-// Where a decode's entering lanes run their first loop iteration.  In the
-// boundary stage (same tick) a token costs its depth in ticks; at the next
-// tick it costs one tick more, but the boundary stage is shorter and runs
-// beside the loop step.  Measured on the B200: 64 lanes at L ~ Poisson(8):
-// 25.7k tokens/s joining at the next tick against 24.1k in the same tick; one
-// lane at L = 8: 1,715 against 1,829; 256 lanes at L in 1..4: 7.3k against
-// 7.9k.  Automatic: the next tick for batches of 32+ lanes whose mean L is 6
-// or more.
+// Where a decode's entering lanes run their first loop iteration, and whether
+// boundary stages run apart from the loop steps.  In the boundary stage (same
+// tick) a token costs its depth in ticks; at the next tick it costs one tick
+// more, but the boundary stage is shorter and runs beside the loop step.  On
+// their own stream (layout 3) the loop steps no longer wait for the boundary
+// stage at every tick, and a lane waits for it only when its own loop has
+// finished.  Measured on the B200: 64 lanes at L ~ Poisson(8): 29.0k tokens/s
+// with layout 3, 25.6k with layout 2, 24.1k with layout 1; one lane at L = 8:
+// 1,829 with layout 1, 1,715 with layout 2; 256 lanes at L in 1..4: 7.9k with
+// layout 1, 7.3k with layouts 2 and 3.  Automatic: layout 3 for batches of
+// 32+ lanes whose mean L is 6 or more, else layout 1.
 static void resolve_entry(tl_ctx* c, const int32_t* host_L, int n_lanes) {
-  if (c->overlap_mode != 0) {
-    c->entry_iter = c->overlap_mode == 1 ? 1 : 0;
-    return;
+  int mode = c->overlap_mode;
+  if (mode == 0) {
+    double sum = 0;
+    for (int i = 0; i < n_lanes; ++i) sum += host_L[i];
+    mode = (n_lanes >= 32 && sum >= 6.0 * n_lanes) ? 3 : 1;
   }
-  double sum = 0;
-  for (int i = 0; i < n_lanes; ++i) sum += host_L[i];
-  c->entry_iter = (n_lanes >= 32 && sum >= 6.0 * n_lanes) ? 0 : 1;
+  // the asynchronous layout needs graphs; run individually, its stages take layout 2's order
+  if (mode == 3 && !(c->graphs_enabled && c->prof_mask == 0)) mode = 2;
+  c->layout = mode;
+  c->entry_iter = mode == 1 ? 1 : 0;
+}
+
+// Layout 3's host loop: loop steps on `stream` as in the tick loop; a
+// boundary stage on bstream whenever fewer than two are queued there.  When
+// the loop found no rows (all live lanes at or in a boundary stage), the next
+// step waits for the last queued boundary stage.
+static int decode_async(tl_ctx* c, int n_lanes, int n_new) {
+  TL_CUDA(cudaEventRecord(c->fork_ev, c->stream));  // the boundary stream starts after the decode's set-up
+  TL_CUDA(cudaStreamWaitEvent(c->bstream, c->fork_ev, 0));
+  int64_t nb = 0;
+  auto launch_bnd = [&]() -> int {
+    TL_CUDA(cudaGraphLaunch(c->bnd_exec, c->bstream));
+    TL_CUDA(cudaEventRecord(c->b_ev[nb % kBRing], c->bstream));
+    ++nb;
+    c->launches += c->bnd_launches;
+    return TL_OK;
+  };
+  auto run = [&]() -> int {
+    TL_TRY(launch_bnd());
+    // safety bound only: a step with rows advances some lane by an iteration, and empty steps are followed
+    // by a wait for the boundary stream
+    const int64_t max_ticks = ((int64_t)n_lanes * n_new * (c->cfg.L_max + 1) + 4) * (kAliveRing + 1);
+    for (int64_t t = 0; t < max_ticks; ++t) {
+      if (t >= kAliveRing - 1) {
+        const int64_t q = (t - (kAliveRing - 1)) % kAliveRing;
+        TL_CUDA(cudaEventSynchronize(c->alive_ev[q]));
+        if (c->pinned_alive[2 * q] == 0) break;
+        if (c->pinned_alive[2 * q + 1] == 0) TL_CUDA(cudaStreamWaitEvent(c->stream, c->b_ev[(nb - 1) % kBRing], 0));
+      }
+      TL_CUDA(cudaGraphLaunch(c->loop_exec, c->stream));
+      c->launches += c->loop_launches;
+      c->steps++;
+      TL_CUDA(cudaMemcpyAsync(&c->pinned_alive[2 * (t % kAliveRing)], c->alive, 8, cudaMemcpyDeviceToHost,
+                              c->stream));
+      TL_CUDA(cudaEventRecord(c->alive_ev[t % kAliveRing], c->stream));
+      if (nb < 2) {
+        TL_TRY(launch_bnd());
+      } else {
+        const cudaError_t q = cudaEventQuery(c->b_ev[(nb - 2) % kBRing]);
+        if (q == cudaSuccess) TL_TRY(launch_bnd());
+        else if (q != cudaErrorNotReady) return check_cuda(q);
+      }
+    }
+    return TL_OK;
+  };
+  const int st = run();
+  // the decode ends when both streams have, on every path
+  TL_CUDA(cudaEventRecord(c->join_ev, c->bstream));
+  TL_CUDA(cudaStreamWaitEvent(c->stream, c->join_ev, 0));
+  return st;
 }
 
 static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int32_t* dep_out) {
@@ -2025,6 +2182,7 @@ static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int3
   // per-kind event profiling needs individual launches; otherwise replay a captured tick
   const bool graphs = c->prof_mask == 0 && c->graphs_enabled;
   if (graphs) TL_TRY(tick_graph(c, n_lanes, n_new, tok_out, dep_out));
+  if (c->layout == 3) return decode_async(c, n_lanes, n_new);
   // upper bound on ticks: every token runs at most L_max iterations, plus the first
   const int64_t max_ticks = (int64_t)n_new * (c->cfg.L_max + 2) + 4;
   for (int64_t t = 0; t < max_ticks; ++t) {
@@ -2032,7 +2190,7 @@ static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int3
     if (t >= kAliveRing - 1) {
       const int64_t q = t - (kAliveRing - 1);
       TL_CUDA(cudaEventSynchronize(c->alive_ev[q % kAliveRing]));
-      if (c->pinned_alive[q % kAliveRing] == 0) break;
+      if (c->pinned_alive[2 * (q % kAliveRing)] == 0) break;
     }
     if (graphs) {
       TL_CUDA(cudaGraphLaunch(c->tick_exec, c->stream));
@@ -2042,7 +2200,7 @@ static int decode_impl(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int3
       TL_TRY(enqueue_tick(c, n_lanes, n_new, tok_out, dep_out));
     }
     // the alive count was written by the tick's first kernel
-    TL_CUDA(cudaMemcpyAsync(&c->pinned_alive[t % kAliveRing], c->alive, 4, cudaMemcpyDeviceToHost, c->stream));
+    TL_CUDA(cudaMemcpyAsync(&c->pinned_alive[2 * (t % kAliveRing)], c->alive, 8, cudaMemcpyDeviceToHost, c->stream));
     TL_CUDA(cudaEventRecord(c->alive_ev[t % kAliveRing], c->stream));
   }
   return TL_OK;
@@ -2104,6 +2262,7 @@ extern "C" int tl_stats_get(tl_ctx* c, tl_stats* out) {
   out->device_status = st;
   out->kv_pages_used = c->lay.n_pages - (int32_t)c->free_pages.size();
   out->entry_in_boundary = c->entry_iter;
+  out->tick_layout = c->layout;
   return TL_OK;
 }
 
@@ -2160,7 +2319,7 @@ extern "C" int tl_profile_end(tl_ctx* c, int64_t* groups, double* total_ms) {
 }
 
 extern "C" int tl_set_tick_overlap(tl_ctx* c, int32_t mode) {
-  if (!c || mode < 0 || mode > 2) return TL_EINVAL;
+  if (!c || mode < 0 || mode > 3) return TL_EINVAL;
   c->overlap_mode = mode;
   return TL_OK;
 }

@@ -104,6 +104,8 @@ typedef struct tl_stats {
     int32_t entry_in_boundary;   /* the last decode ran entering lanes' first loop
                                     iteration in the boundary stage (1) or at the
                                     next tick (0); see tl_set_tick_overlap      */
+    int32_t tick_layout;         /* the layout the last decode ran: 1, 2 or 3 (see
+                                    tl_set_tick_overlap)                         */
 } tl_stats;
 
 /* ---------------------------------------------------------------- sizes -- */
@@ -331,17 +333,23 @@ int tl_speculate(tl_ctx* ctx, int32_t lane, int32_t n_new, int32_t L_draft, int3
 
 /* Layout of a decode tick ("Depth-adaptive Inference of Looped Language
  * Models via Continuous Depth Batching": boundary stages queued apart from
- * loop steps, with scheduling overlapping GPU work).  Every tick runs two
- * concurrent branches on disjoint lanes: the boundary stage (head, greedy
- * token, embedding and pre blocks of the lanes whose loop finished) and one
- * loop iteration of the lanes in their loop.  mode 1: a lane that takes a
- * token also runs its first loop iteration in that boundary stage (a token
- * costs its depth in ticks); mode 2: it joins the loop step at the next tick
- * (one tick more per token, a shorter boundary stage); mode 0 (default)
- * chooses per decode call: mode 2 for 32+ lanes with mean requested L of 6 or
- * more, mode 1 otherwise.  Results per lane do not depend on it beyond the
- * rounding differences of batch width (see tl_stats.entry_in_boundary).
- * TL_EINVAL for other modes. */
+ * loop steps, with scheduling overlapping GPU work).  In modes 1 and 2 every
+ * tick runs two concurrent branches on disjoint lanes and ends when both
+ * have: the boundary stage (head, greedy token, embedding and pre blocks of
+ * the lanes whose loop finished) and one loop iteration of the lanes in their
+ * loop.  mode 1: a lane that takes a token also runs its first loop
+ * iteration in that boundary stage (a token costs its depth in ticks); mode
+ * 2: it joins the loop step at the next tick (one tick more per token, a
+ * shorter boundary stage).  mode 3: the two run on two streams at their own
+ * cadence with no join per tick; each boundary stage takes the lanes whose
+ * loop has finished when it starts and hands those that continue to the loop
+ * when their pre blocks are done (needs CUDA graphs, else mode 2 runs).
+ * mode 0 (default) chooses per decode call: mode 3 for 32+ lanes with mean
+ * requested L of 6 or more, mode 1 otherwise.  Results per lane do not
+ * depend on it beyond the rounding differences of batch width (a row's
+ * projections take fp32 activations in a step of at most 8 rows, fp16 in a
+ * wider one); in mode 3 the widths depend on timing.  See
+ * tl_stats.tick_layout.  TL_EINVAL for other modes. */
 int tl_set_tick_overlap(tl_ctx* ctx, int32_t mode);
 
 /* Shared-prefix ("cascade") attention in decode steps (default on; "Benchmark

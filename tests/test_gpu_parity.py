@@ -193,10 +193,11 @@ def test_m407_wide_decode_logits():
             assert_logits_close(lg[i, t], ref[i].logits[t], f"lane {i} token {t}")
 
 
-@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("mode", [1, 2, 3])
 def test_tiny_tick_layouts_match_oracle(mode):
-    # both layouts of a decode tick (entering lanes' first iteration in the boundary stage, or at the next
-    # tick beside the other lanes' loop step) give each lane its own schedule and tokens
+    # every layout of a decode tick (entering lanes' first iteration in the boundary stage, at the next
+    # tick beside the other lanes' loop step, or boundary stages on their own stream) gives each lane its
+    # own schedule and tokens
     W = oracle_weights("tiny", 7)
     P = S.prompts(16, 12, 512, seed=75)
     Ls = [1, 2, 3, 4, 5, 6, 7, 8] * 2
@@ -205,7 +206,47 @@ def test_tiny_tick_layouts_match_oracle(mode):
     tok, dep = m.generate(P, Ls, 7)
     st = status_clean(m)
     assert st["entry_in_boundary"] == (1 if mode == 1 else 0)
+    assert st["tick_layout"] == mode
+    assert st["tokens_emitted"] >= 16 * 7
     for i in range(16):
         r = D.generate_lane(W, P[i], Ls[i], 7)
         assert dep[i].tolist() == r.depths.tolist()
         _check_tokens(r.tokens, r.logits, tok[i])
+
+
+def _tau_clear_of_probes(W, P, Ls, n_new, candidates, min_L=1, patience=1, peek=1):
+    """The first threshold whose oracle run has no probe within 1% of it and exits somewhere early:
+    (early-exit rule, oracle results)."""
+    for tau in candidates:
+        ee = D.EarlyExit(tau, min_L, patience, peek)
+        ref = [D.generate_lane(W, P[i], Ls[i], n_new, ee) for i in range(len(Ls))]
+        clear = not [x for x in _probe_margins(ref, tau) if x <= 1e-2]
+        fired = any(int(d) < L for r, L in zip(ref, Ls) for d in r.depths[1:])
+        if clear and fired:
+            return ee, ref
+    raise AssertionError("no candidate threshold clear of the probes")
+
+
+@pytest.mark.parametrize("exit_rule", [False, True])
+def test_tiny_async_stages_early_exit_and_repeat(exit_rule):
+    # boundary stages apart from the loop steps: exact schedules with the exit rule, twice on one model
+    # (the second run replays the captured graphs)
+    W = oracle_weights("tiny")
+    P = S.prompts(24, 10, 512, seed=76)
+    Ls = [8, 1, 5, 3, 7, 2, 6, 4] * 3
+    m = gpu_model("tiny", None, max_lanes=24, max_seq=40, L_max=8)
+    m.set_tick_overlap(3)
+    if exit_rule:
+        # probes every second iteration from l = 3, two successes in a row: the oracle's probe values leave
+        # a wide gap around 0.45
+        ee, ref = _tau_clear_of_probes(W, P, Ls, 9, [0.446, 0.43, 0.46, 0.257], min_L=2, patience=2, peek=2)
+        m.set_early_exit(ee.tau, ee.min_L, ee.patience, ee.peek_every)
+    else:
+        ref = [D.generate_lane(W, P[i], Ls[i], 9) for i in range(24)]
+    for _ in range(2):
+        tok, dep = m.generate(P, Ls, 9)
+        st = status_clean(m)
+        assert st["tick_layout"] == 3
+        for i in range(24):
+            assert dep[i].tolist() == ref[i].depths.tolist(), i
+            _check_tokens(ref[i].tokens, ref[i].logits, tok[i])
