@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace tl {
 
@@ -22,15 +23,71 @@ namespace tl {
 // (row, head, split): the key
 // blocks of 32 positions are divided into S contiguous ranges, S chosen on the
 // device from the live row count so that few rows still spread over the SMs
-// (S <= gridDim.z).  Inside a CTA warp w takes blocks w, w+4, ...: one key per
-// lane for the scores, then every lane owns hd/32 output dimensions for the
-// value sum (all 32 value loads of a block issued together); running max and
-// sum are merged across warps, and across splits by the last CTA of the
-// (row, head) to finish, in split order.  Requires kv_page_tokens >= 32.
+// (S <= gridDim.z).  Inside a CTA warp w takes blocks w, w+4, ..., streamed
+// through its own two-stage shared-memory ring: one key per lane for the
+// scores, then every lane owns hd/32 output dimensions for the value sum;
+// running max and sum are merged across warps, and across splits by the last
+// CTA of the (row, head) to finish, in split order.  Requires kv_page_tokens
+// >= 32 (a block lies in one page).
 // Working CTAs the context split aims for: four per SM on 148 SMs (a
 // larger target, 12 per SM, split the 64-row case in two and measured
 // slower: the split partials and their combine cost more than the waves save).
 constexpr int kAttnCtaTarget = 4 * 148;
+
+// Keys of one ring stage: 32 (one per lane), 16 at head dim 128 (two lanes
+// per key), so that a stage of keys is 4 KB or less at every head dim.
+template <int HD>
+constexpr int kAttnKeys = HD >= 128 ? 16 : 32;
+// Bytes of one stage's keys (or values) of one head.
+template <int HD>
+constexpr int kAttnBlockBytes = kAttnKeys<HD> * HD * 2;
+// Dynamic shared memory of attn_split_kernel: per warp, two stages of a block's keys and values.
+template <int HD>
+constexpr int kAttnSplitSmem = 4 * 2 * 2 * kAttnBlockBytes<HD>;
+
+extern __shared__ __align__(16) uint8_t attn_split_smem[];
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Stored position of 16-byte chunk c of key row r: the eight rows one
+// shared-memory access phase reads (lane = row) land in eight different bank
+// groups.
+template <int HD>
+__device__ __forceinline__ int attn_swz(int c, int r) {
+  return HD == 32 ? (c ^ ((r >> 1) & 3)) : (c ^ (r & 7));
+}
+
+// The keys and values of sub-block sb (positions sb*KEYS ..) of one head into
+// a ring stage: keys at row stride HD*2 bytes with swizzled chunks, then
+// values unswizzled; rows at or past ctx are zero-filled (no global read).
+// false when the page table has no page there (status set).
+template <int HD>
+__device__ __forceinline__ bool attn_issue_block(uint8_t* stage, const KVGeom& g, int ln, int slot, int sb, int ctx,
+                                                 int h, int32_t* status) {
+  constexpr int KEYS = kAttnKeys<HD>;
+  const __half* kbase = kv_k_ptr(g, ln, slot, sb * KEYS, h, status);
+  if (!kbase) return false;
+  const __half* vbase = kbase + (int64_t)g.H * g.page_tokens * HD;
+  const int lane = threadIdx.x & 31;
+  const int nk = min(KEYS, ctx - sb * KEYS);
+  constexpr int CPR = HD / 8;
+#pragma unroll
+  for (int q = lane; q < KEYS * CPR; q += 32) {
+    const int row = q / CPR, c = q % CPR;
+    const int bytes = row < nk ? 16 : 0;
+    cp_async16(stage + row * HD * 2 + attn_swz<HD>(c, row) * 16, kbase + row * HD + c * 8, bytes);
+    cp_async16(stage + kAttnBlockBytes<HD> + row * HD * 2 + c * 16, vbase + row * HD + c * 8, bytes);
+  }
+  return true;
+}
 
 template <int HD>
 __global__ void __launch_bounds__(128)
@@ -85,40 +142,37 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
   float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  for (int kb = b0 + warp; kb < b1; kb += 4) {
-    const __half* kbase = kv_k_ptr(g, ln, slot, kb * 32, h, status);
-    if (!kbase) break;
-    const __half* vbase = kbase + (int64_t)g.H * g.page_tokens * HD;
-    const int j = kb * 32 + lane;
-    const int nk = min(32, ctx - kb * 32);
-    // the block's values, loaded together with its keys (neither depends on the scores)
-    constexpr int VW = DPL >= 2 ? DPL / 2 : 1;  // 32-bit words of values per lane per key
-    uint32_t vraw[32][VW];
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      if (jj < nk) {
-        if constexpr (DPL >= 2) {
-#pragma unroll
-          for (int e = 0; e < VW; ++e)
-            vraw[jj][e] = reinterpret_cast<const uint32_t*>(vbase + (int64_t)jj * HD + lane * DPL)[e];
-        } else {
-          vraw[jj][0] = __half_as_ushort(vbase[(int64_t)jj * HD + lane]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < VW; ++e) vraw[jj][e] = 0u;
-      }
-    }
+  // Each warp streams its blocks through a two-stage shared-memory ring
+  // (cp.async, 16-byte chunks): the next block's keys and values are in
+  // flight while the current one is scored and summed.
+  constexpr int KEYS = kAttnKeys<HD>;
+  constexpr int LPK = 32 / KEYS;       // lanes per key (their partial dots are summed)
+  constexpr int CPL = HD / 8 / LPK;    // 16-byte chunks of a key row per lane
+  uint8_t* ring = attn_split_smem + (size_t)warp * 2 * 2 * kAttnBlockBytes<HD>;
+  const int key = lane % KEYS, half = lane / KEYS;
+  // the split's 32-position blocks b0 .. b1 as sub-blocks of KEYS positions
+  const int sb1 = min(b1 * (32 / KEYS), (ctx + KEYS - 1) / KEYS);
+  int sb = b0 * (32 / KEYS) + warp;
+  bool more = sb < sb1 && attn_issue_block<HD>(ring, g, ln, slot, sb, ctx, h, status);
+  cp_async_commit();
+  for (int stage = 0; more; stage ^= 1) {
+    const int sn = sb + 4;
+    const bool next = sn < sb1 && attn_issue_block<HD>(ring + (stage ^ 1) * 2 * kAttnBlockBytes<HD>, g, ln, slot, sn,
+                                                       ctx, h, status);
+    cp_async_commit();
+    cp_async_wait<1>();  // this sub-block's copies (each lane's own) have landed
+    __syncwarp();        // ... and every lane's are visible to the warp
+    const uint8_t* ks = ring + stage * 2 * kAttnBlockBytes<HD>;
+    const uint8_t* vs = ks + kAttnBlockBytes<HD>;
+    const int j = sb * KEYS + key;
     float s = -INFINITY;
-    if (j < ctx) {
-      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (int64_t)lane * HD);
-      uint4 kv[HD / 8];
-#pragma unroll
-      for (int c = 0; c < HD / 8; ++c) kv[c] = kr[c];
+    {
       float dot = 0.f;
 #pragma unroll
-      for (int c = 0; c < HD / 8; ++c) {
-        const __half2* hv = reinterpret_cast<const __half2*>(&kv[c]);
+      for (int cc = 0; cc < CPL; ++cc) {
+        const int c = half * CPL + cc;
+        const uint4 kv = *reinterpret_cast<const uint4*>(ks + key * HD * 2 + attn_swz<HD>(c, key) * 16);
+        const __half2* hv = reinterpret_cast<const __half2*>(&kv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __half22float2(hv[e]);
@@ -126,31 +180,42 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
           dot = fmaf(qs[8 * c + 2 * e + 1], f.y, dot);
         }
       }
-      s = dot;
+      if constexpr (LPK == 2) dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+      if (j < ctx) s = dot;
     }
     const float mb = warp_max(s);
     const float mn = fmaxf(m, mb);
-    const float p = (j < ctx) ? expf(s - mn) : 0.f;
+    const float p = (j < ctx && half == 0) ? expf(s - mn) : 0.f;  // one lane per key carries its weight
     const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
     l = l * corr + warp_sum(p);
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[e] *= corr;
     m = mn;
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
+#pragma unroll 8
+    for (int jj = 0; jj < KEYS; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      if constexpr (DPL >= 2) {
-#pragma unroll
-        for (int e = 0; e < VW; ++e) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vraw[jj][e]));
-          acc[2 * e] = fmaf(pj, f.x, acc[2 * e]);
-          acc[2 * e + 1] = fmaf(pj, f.y, acc[2 * e + 1]);
-        }
+      const uint8_t* vr = vs + jj * HD * 2 + lane * DPL * 2;  // rows past the context were zero-filled
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vr);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+        acc[0] = fmaf(pj, f0.x, acc[0]);
+        acc[1] = fmaf(pj, f0.y, acc[1]);
+        acc[2] = fmaf(pj, f1.x, acc[2]);
+        acc[3] = fmaf(pj, f1.y, acc[3]);
+      } else if constexpr (DPL == 2) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(vr));
+        acc[0] = fmaf(pj, f.x, acc[0]);
+        acc[1] = fmaf(pj, f.y, acc[1]);
       } else {
-        acc[0] = fmaf(pj, __half2float(__ushort_as_half((unsigned short)vraw[jj][0])), acc[0]);
+        acc[0] = fmaf(pj, __half2float(*reinterpret_cast<const __half*>(vr)), acc[0]);
       }
     }
+    __syncwarp();  // every lane is done with this stage before it is refilled
+    sb = sn;
+    more = next;
   }
+  cp_async_wait<0>();
   if (lane == 0) { wm[warp] = m; wl[warp] = l; }
 #pragma unroll
   for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];

@@ -716,6 +716,18 @@ int cascade_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int
 // faster around the neighbouring projections in CUDA-graph ticks (64 lanes:
 // 346 against 358 ms per decode pass; one lane at L = 8: 1,609 against 1,516
 // tokens/s), with the same per-kind kernel time.
+template <int HD>
+int attn_split_launch(tl_ctx* c, dim3 grid, const Rows& rows, int slot_base, int slot_stride) {
+  static uint64_t attr_done = 0;  // per instantiation: one bit per device
+  if (attr_needed(&attr_done)) {
+    TL_CUDA(cudaFuncSetAttribute(attn_split_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kAttnSplitSmem<HD>));
+  }
+  return launch_k(c, attn_split_kernel<HD>, grid, dim3(128), kAttnSplitSmem<HD>, (const float*)c->sc->act_qkv,
+                  c->sc->act_o, c->sc->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride,
+                  c->sc->attn_part, c->sc->attn_counters, c->status);
+}
+
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
   TL_TRY(prof_start(c, TL_PROF_ATTN));
   const bool cascade = c->cascade_active && c->hd >= 64;
@@ -730,9 +742,9 @@ int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int sl
     if (max_rows > 1) ks = ks < 4 ? 4 : ks;
     const dim3 grid(max_rows, c->cfg.n_heads, ks);
     switch (c->hd) {
-      case 32: st = launch_k(c, attn_split_kernel<32>, grid, dim3(128), 0, (const float*)c->sc->act_qkv, c->sc->act_o, c->sc->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride, c->sc->attn_part, c->sc->attn_counters, c->status); break;
-      case 64: st = launch_k(c, attn_split_kernel<64>, grid, dim3(128), 0, (const float*)c->sc->act_qkv, c->sc->act_o, c->sc->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride, c->sc->attn_part, c->sc->attn_counters, c->status); break;
-      default: st = launch_k(c, attn_split_kernel<128>, grid, dim3(128), 0, (const float*)c->sc->act_qkv, c->sc->act_o, c->sc->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride, c->sc->attn_part, c->sc->attn_counters, c->status); break;
+      case 32: st = attn_split_launch<32>(c, grid, rows, slot_base, slot_stride); break;
+      case 64: st = attn_split_launch<64>(c, grid, rows, slot_base, slot_stride); break;
+      default: st = attn_split_launch<128>(c, grid, rows, slot_base, slot_stride); break;
     }
   }
   TL_TRY(st);
