@@ -34,16 +34,20 @@ namespace tl {
 // slower: the split partials and their combine cost more than the waves save).
 constexpr int kAttnCtaTarget = 4 * 148;
 
-// Keys of one ring stage: 32 (one per lane), 16 at head dim 128 (two lanes
-// per key), so that a stage of keys is 4 KB or less at every head dim.
+// Keys of one ring stage: 16 (two lanes per key) from head dim 64, 32 (one
+// per lane) below.
 template <int HD>
-constexpr int kAttnKeys = HD >= 128 ? 16 : 32;
+constexpr int kAttnKeys = HD >= 64 ? 16 : 32;
 // Bytes of one stage's keys (or values) of one head.
 template <int HD>
 constexpr int kAttnBlockBytes = kAttnKeys<HD> * HD * 2;
-// Dynamic shared memory of attn_split_kernel: per warp, two stages of a block's keys and values.
+// Ring stages per warp: as many as 16 KB per warp holds (4 at head dims 32
+// and 64, 2 at 128), so a CTA takes 64 KB and three share an SM.
 template <int HD>
-constexpr int kAttnSplitSmem = 4 * 2 * 2 * kAttnBlockBytes<HD>;
+constexpr int kAttnStages = (8 * 1024) / kAttnBlockBytes<HD> >= 4 ? 4 : 2;
+// Dynamic shared memory of attn_split_kernel: per warp, its stages of keys and values.
+template <int HD>
+constexpr int kAttnSplitSmem = 4 * kAttnStages<HD> * 2 * kAttnBlockBytes<HD>;
 
 extern __shared__ __align__(16) uint8_t attn_split_smem[];
 
@@ -142,28 +146,35 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
   float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  // Each warp streams its blocks through a two-stage shared-memory ring
-  // (cp.async, 16-byte chunks): the next block's keys and values are in
-  // flight while the current one is scored and summed.
+  // Each warp streams its sub-blocks through a ring of NS shared-memory
+  // stages (cp.async, 16-byte chunks): NS - 1 sub-blocks' keys and values are
+  // in flight while the current one is scored and summed.
   constexpr int KEYS = kAttnKeys<HD>;
   constexpr int LPK = 32 / KEYS;       // lanes per key (their partial dots are summed)
   constexpr int CPL = HD / 8 / LPK;    // 16-byte chunks of a key row per lane
-  uint8_t* ring = attn_split_smem + (size_t)warp * 2 * 2 * kAttnBlockBytes<HD>;
+  constexpr int NS = kAttnStages<HD>;
+  constexpr int BB = kAttnBlockBytes<HD>;
+  uint8_t* ring = attn_split_smem + (size_t)warp * NS * 2 * BB;
   const int key = lane % KEYS, half = lane / KEYS;
-  // the split's 32-position blocks b0 .. b1 as sub-blocks of KEYS positions
+  // the split's 32-position blocks b0 .. b1 as sub-blocks of KEYS positions; this warp's are sb0, sb0 + 4, ...
   const int sb1 = min(b1 * (32 / KEYS), (ctx + KEYS - 1) / KEYS);
-  int sb = b0 * (32 / KEYS) + warp;
-  bool more = sb < sb1 && attn_issue_block<HD>(ring, g, ln, slot, sb, ctx, h, status);
-  cp_async_commit();
-  for (int stage = 0; more; stage ^= 1) {
-    const int sn = sb + 4;
-    const bool next = sn < sb1 && attn_issue_block<HD>(ring + (stage ^ 1) * 2 * kAttnBlockBytes<HD>, g, ln, slot, sn,
-                                                       ctx, h, status);
+  const int sb0 = b0 * (32 / KEYS) + warp;
+  int avail = sb0 < sb1 ? (sb1 - sb0 + 3) / 4 : 0;  // a sub-block without a page ends the range
+#pragma unroll
+  for (int i = 0; i < NS - 1; ++i) {
+    if (i < avail && !attn_issue_block<HD>(ring + i * 2 * BB, g, ln, slot, sb0 + 4 * i, ctx, h, status)) avail = i;
     cp_async_commit();
-    cp_async_wait<1>();  // this sub-block's copies (each lane's own) have landed
-    __syncwarp();        // ... and every lane's are visible to the warp
-    const uint8_t* ks = ring + stage * 2 * kAttnBlockBytes<HD>;
-    const uint8_t* vs = ks + kAttnBlockBytes<HD>;
+  }
+  for (int i = 0; i < avail; ++i) {
+    const int ip = i + NS - 1;
+    if (ip < avail && !attn_issue_block<HD>(ring + (ip % NS) * 2 * BB, g, ln, slot, sb0 + 4 * ip, ctx, h, status))
+      avail = ip;
+    cp_async_commit();
+    cp_async_wait<NS - 1>();  // sub-block i's copies (each lane's own) have landed
+    __syncwarp();             // ... and every lane's are visible to the warp
+    const int sb = sb0 + 4 * i;
+    const uint8_t* ks = ring + (i % NS) * 2 * BB;
+    const uint8_t* vs = ks + BB;
     const int j = sb * KEYS + key;
     float s = -INFINITY;
     {
@@ -212,8 +223,6 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
       }
     }
     __syncwarp();  // every lane is done with this stage before it is refilled
-    sb = sn;
-    more = next;
   }
   cp_async_wait<0>();
   if (lane == 0) { wm[warp] = m; wl[warp] = l; }
