@@ -827,9 +827,39 @@ def run_prefix256(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": None,
         "cpu_baseline": None,
-        "cpu_baseline_note": "the oracle would need ~10 TFLOP of fp64 work for the 1088-token prompt of one lane",
     })
+    if rank == 0 and not args.no_cpu_baseline:
+        v, dec_s, pr_s, cores, lane = oracle_prefix_sample(wl, 2)
+        out["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": f"lane {lane} (L=1): the {Tp}-token shared prefix and its {Ts}-token "
+                                         f"suffix at L=1 ({pr_s:.1f} s, excluded), then 2 greedy tokens in "
+                                         f"{dec_s:.1f} s; fp64 NumPy"}
     return out
+
+
+def oracle_prefix_sample(wl, n_tokens: int = 2):
+    """The fp64 oracle on a bounded sample of the shared-prefix workload: the
+    first lane with L = 1 (the 1024-token prefix and its suffix at L = 1, then
+    n_tokens greedy tokens).  Returns (decode tokens/s, seconds of decode,
+    seconds of prompt, cores, lane)."""
+    import oracle as O
+    from oracle import model as M
+    sh = wl.shape
+    W = O.build_weights(sh, S.master_weights(sh), S.gains(sh))
+    pre, suf = S.prefix_prompts(wl)
+    lane = next(i for i, L in enumerate(wl.per_lane_L) if int(L) == 1)
+    prompt = np.concatenate([pre, suf[lane]])
+    t0 = time.perf_counter()
+    h, cache = M.forward(W, prompt, 1, M.KVCache(sh, len(prompt) + n_tokens))
+    logits = M.head_logits(W, h[-1:])[0]
+    t1 = time.perf_counter()
+    pos = len(prompt)
+    for _ in range(n_tokens):
+        h, cache = M.forward(W, [int(M.argmax_lowest(logits))], 1, cache, pos0=pos)
+        logits = M.head_logits(W, h[-1:])[0]
+        pos += 1
+    t2 = time.perf_counter()
+    return n_tokens / (t2 - t1), t2 - t1, t1 - t0, len(os.sched_getaffinity(0)), lane
 
 
 # ---------------------------------------------------------- cpu / oracle ----

@@ -20,11 +20,12 @@ _FMT = {"int4": TL_FMT_INT4, "bf16": TL_FMT_BF16}
 
 def make_config(vocab, d, n_heads, ffn, n_pre, n_loop_layers, fmt_pre="int4", fmt_loop="int4",
                 fmt_embed_head="int4", group=128, rms_eps=1e-5, rope_base=1e4, *, max_lanes=1,
-                max_seq=256, L_max=32, kv_page_tokens=64, kv_pool_pages=0, max_prefill_tokens=0) -> TlConfig:
+                max_seq=256, L_max=32, kv_page_tokens=64, kv_pool_pages=0, max_prefill_tokens=0,
+                act_split=0) -> TlConfig:
     f = lambda x: _FMT[x] if isinstance(x, str) else int(x)  # noqa: E731
     return TlConfig(vocab, d, n_heads, ffn, n_pre, n_loop_layers, f(fmt_pre), f(fmt_loop), f(fmt_embed_head),
                     group, rms_eps, rope_base, max_lanes, max_seq, L_max, kv_page_tokens, kv_pool_pages,
-                    max_prefill_tokens)
+                    max_prefill_tokens, act_split)
 
 
 def config_from_shape(shape, **capacity) -> TlConfig:

@@ -24,6 +24,7 @@ class TlConfig(C.Structure):
         ("rms_eps", C.c_float), ("rope_base", C.c_float),
         ("max_lanes", C.c_int32), ("max_seq", C.c_int32), ("L_max", C.c_int32),
         ("kv_page_tokens", C.c_int32), ("kv_pool_pages", C.c_int32), ("max_prefill_tokens", C.c_int32),
+        ("act_split", C.c_int32),
     ]
 
 

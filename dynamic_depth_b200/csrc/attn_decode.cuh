@@ -95,7 +95,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
                    __half* __restrict__ o16, Rows rows, KVGeom g, const float2* __restrict__ rope_cs, int slot_base,
                    int slot_stride, float* __restrict__ part, int32_t* __restrict__ counters,
                    int32_t* __restrict__ status, const int32_t* __restrict__ lane_shared,
-                   const float* __restrict__ casc) {
+                   const float* __restrict__ casc, int split16) {
   using C = AttnCfg<HD>;
   constexpr int UK = C::UK, STAGES = C::STAGES, WARPS = C::WARPS, HALF = HD / 2, LPR = C::LPR, G = C::G;
   constexpr int CPT = C::COLS / 8;  // 16-byte chunks per tile row
@@ -399,10 +399,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
           float4* op = reinterpret_cast<float4*>(o + (int64_t)r * d + h * HD + dim0);
           op[0] = make_float4(tot[0] * inv, tot[1] * inv, tot[2] * inv, tot[3] * inv);
           op[1] = make_float4(tot[4] * inv, tot[5] * inv, tot[6] * inv, tot[7] * inv);
-          __half2 hv[4];
+          float ov[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) hv[e] = __floats2half2_rn(tot[2 * e] * inv, tot[2 * e + 1] * inv);
-          *reinterpret_cast<uint4*>(o16 + (int64_t)r * d + h * HD + dim0) = *reinterpret_cast<const uint4*>(hv);
+          for (int e = 0; e < 8; ++e) ov[e] = tot[e] * inv;
+          act16_put8(o16, r, d, h * HD + dim0, ov, split16);
         }
       } else {
         const int first_unit = ubase[r] + h * nu;  // flat index of block 0 of (r, h)
@@ -449,10 +449,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap kvmap, const float* __res
             float4* op = reinterpret_cast<float4*>(o + (int64_t)r * d + h * HD + dim0);
             op[0] = make_float4(outv[0] * inv, outv[1] * inv, outv[2] * inv, outv[3] * inv);
             op[1] = make_float4(outv[4] * inv, outv[5] * inv, outv[6] * inv, outv[7] * inv);
-            __half2 hv[4];
+            float ov[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) hv[e] = __floats2half2_rn(outv[2 * e] * inv, outv[2 * e + 1] * inv);
-            *reinterpret_cast<uint4*>(o16 + (int64_t)r * d + h * HD + dim0) = *reinterpret_cast<const uint4*>(hv);
+            for (int e = 0; e < 8; ++e) ov[e] = outv[e] * inv;
+            act16_put8(o16, r, d, h * HD + dim0, ov, split16);
           }
           if (lane == 0) counters[r * H + h] = 0;
         }

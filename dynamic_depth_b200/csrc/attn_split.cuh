@@ -97,7 +97,8 @@ template <int HD>
 __global__ void __launch_bounds__(128)
 attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
                    KVGeom g, const float2* __restrict__ rope_cs, int slot_base, int slot_stride,
-                   float* __restrict__ part, int32_t* __restrict__ counters, int32_t* __restrict__ status) {
+                   float* __restrict__ part, int32_t* __restrict__ counters, int32_t* __restrict__ status,
+                   int split16) {
   pdl_launch_dependents();
   pdl_wait();
   constexpr int DPL = HD / 32;  // output dims per lane
@@ -242,7 +243,7 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
       float v = 0.f;
       for (int w = 0; w < 4; ++w) v += wacc[w][i] * f[w];
       o[(int64_t)r * d + h * HD + i] = v / Lsum;
-      o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lsum);
+      act16_put(o16, r, d, h * HD + i, v / Lsum, split16);
     }
     return;
   }
@@ -275,7 +276,7 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
       v += __ldcg(base + zz * (HD + 2) + 2 + i) * ((mz == -INFINITY) ? 0.f : expf(mz - Mx));
     }
     o[(int64_t)r * d + h * HD + i] = v / Lt;
-    o16[(int64_t)r * d + h * HD + i] = __float2half_rn(v / Lt);
+    act16_put(o16, r, d, h * HD + i, v / Lt, split16);
   }
   if (threadIdx.x == 0) counters[r * g.H + h] = 0;
 }

@@ -59,7 +59,8 @@ struct AttnTcParams {
   int32_t chunks;                // mode 1: CTAs per loop iteration (128-row chunks of the rows)
   float* casc;                   // mode 1: [rows][H][hd + 2] partial (max, sum, output)
   float* o;                      // mode 0: output rows [rows][d]
-  __half* o16;
+  __half* o16;                   // mode 0: fp16 copy (hi and lo halves with split16)
+  int32_t split16;
   KVGeom g;
   int32_t slot_base, slot_stride;
   int32_t* status;
@@ -403,12 +404,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kvmap, AttnTcParams p) {
         if (p.mode == 0) {
           const float inv = 1.f / l;
           float* od = p.o + (int64_t)row * d + h * HD;
-          __half* oh = p.o16 + (int64_t)row * d + h * HD;
 #pragma unroll
-          for (int e = 0; e < HD; e += 4) {
-            *reinterpret_cast<float4*>(od + e) = make_float4(O[e] * inv, O[e + 1] * inv, O[e + 2] * inv, O[e + 3] * inv);
-            *reinterpret_cast<__half2*>(oh + e) = __floats2half2_rn(O[e] * inv, O[e + 1] * inv);
-            *reinterpret_cast<__half2*>(oh + e + 2) = __floats2half2_rn(O[e + 2] * inv, O[e + 3] * inv);
+          for (int e = 0; e < HD; e += 8) {
+            float ov[8];
+#pragma unroll
+            for (int f = 0; f < 8; ++f) ov[f] = O[e + f] * inv;
+            *reinterpret_cast<float4*>(od + e) = make_float4(ov[0], ov[1], ov[2], ov[3]);
+            *reinterpret_cast<float4*>(od + e + 4) = make_float4(ov[4], ov[5], ov[6], ov[7]);
+            act16_put8(p.o16, row, d, h * HD + e, ov, p.split16);
           }
         } else {
           float* dst = p.casc + ((int64_t)row * H + h) * (HD + 2);

@@ -29,6 +29,33 @@ enum LanePhase : int32_t { PH_IDLE = 0, PH_LOOP = 1, PH_BOUNDARY = 2, PH_DONE = 
 // A lane's phase is the hand-off word between concurrently running stages:
 // the writer orders every other write of the lane before it (release), the
 // reader reads it before the lane's other fields (acquire).
+// fp16 copy of an activation for the tensor cores, row `row` of a [rows][cols]
+// activation.  With split16 a row holds [hi | lo] (2 * cols halves): hi =
+// fp16(v), lo = fp16(v - hi); a projection that multiplies both halves by the
+// same weights and sums (a K of 2 * cols) sees the fp32 activation to within
+// ~2^-22 relative instead of fp16's 2^-11.
+__device__ __forceinline__ void act16_put(__half* base, int64_t row, int cols, int col, float v, int split16) {
+  __half* p = base + row * ((int64_t)cols << split16) + col;
+  const __half hi = __float2half_rn(v);
+  *p = hi;
+  if (split16) p[cols] = __float2half_rn(v - __half2float(hi));
+}
+
+// Eight consecutive columns col0 .. col0 + 7 (col0 a multiple of 8) as act16_put does, in 16-byte stores.
+__device__ __forceinline__ void act16_put8(__half* base, int64_t row, int cols, int col0, const float (&v)[8],
+                                           int split16) {
+  __half* p = base + row * ((int64_t)cols << split16) + col0;
+  __half2 hi[4], lo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    hi[e] = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+    const float2 f = __half22float2(hi[e]);
+    lo[e] = __floats2half2_rn(v[2 * e] - f.x, v[2 * e + 1] - f.y);
+  }
+  *reinterpret_cast<uint4*>(p) = *reinterpret_cast<const uint4*>(hi);
+  if (split16) *reinterpret_cast<uint4*>(p + cols) = *reinterpret_cast<const uint4*>(lo);
+}
+
 __device__ __forceinline__ int32_t phase_acquire(const int32_t* p) {
   int32_t v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -251,7 +251,8 @@ __global__ void plan_tick_kernel(LaneState* lanes, int n_lanes, Rows boundary, R
 // --------------------------------------------------------------- norms ----
 
 // out[r] = RMSNorm(h[map ? map[r] : r]) * g, fp32 (and an fp16 copy for the
-// tensor-core projections when out16 is given).  One CTA per row.  When h_in is
+// tensor-core projections when out16 is given, split into hi and lo halves
+// with split16, see act16_put).  One CTA per row.  When h_in is
 // given, also copies the source row there (indexed like h); when zero_rows is
 // given, clears row r of that [rows][zero_cols] accumulator, which the next
 // (split-K) projection adds into.  Does nothing more when the row count is
@@ -263,7 +264,8 @@ __global__ void rmsnorm_rows_kernel(float* __restrict__ h, const int32_t* __rest
                                     const int32_t* __restrict__ n_rows, int d, const float* __restrict__ g,
                                     float eps, float* __restrict__ out, float* __restrict__ h_in,
                                     __half* __restrict__ out16, float* __restrict__ zero_rows, int zero_cols,
-                                    int min_rows, const float* __restrict__ add, const int32_t* __restrict__ n_add) {
+                                    int min_rows, const float* __restrict__ add, const int32_t* __restrict__ n_add,
+                                    int split16) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float red[32];
@@ -285,7 +287,7 @@ __global__ void rmsnorm_rows_kernel(float* __restrict__ h, const int32_t* __rest
     const float v = x[k];
     const float y = v * inv * g[k];
     out[(int64_t)r * d + k] = y;
-    if (out16) out16[(int64_t)r * d + k] = __float2half_rn(y);
+    if (out16) act16_put(out16, r, d, k, y, split16);
     if (h_in) h_in[(int64_t)src * d + k] = v;
   }
   if (zero_rows)
@@ -588,7 +590,7 @@ __global__ void rope_kv_kernel(const float* __restrict__ qkv, float* __restrict_
 template <int HD>
 __global__ void __launch_bounds__(256)
 attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* __restrict__ o16, Rows rows,
-                    const int2* __restrict__ tiles, KVGeom g, int slot, int32_t* __restrict__ status) {
+                    const int2* __restrict__ tiles, KVGeom g, int slot, int32_t* __restrict__ status, int split16) {
   pdl_launch_dependents();
   pdl_wait();
   constexpr int BQ = 64, BK = 64, DPT = HD / 16;
@@ -719,7 +721,7 @@ attn_prefill_kernel(const float* __restrict__ q, float* __restrict__ o, __half* 
 #pragma unroll
     for (int j = 0; j < DPT; ++j) {
       o[(int64_t)(r0 + r) * d + h * HD + tx * DPT + j] = acc[i][j] * inv;
-      o16[(int64_t)(r0 + r) * d + h * HD + tx * DPT + j] = __float2half_rn(acc[i][j] * inv);
+      act16_put(o16, r0 + r, d, h * HD + tx * DPT + j, acc[i][j] * inv, split16);
     }
   }
 }

@@ -57,7 +57,22 @@ static bool cfg_valid(const tl_config* c) {
   if (c->max_lanes < 1 || c->max_lanes > 1024 || c->max_seq < 1 || c->L_max < 1) return false;
   if (c->kv_page_tokens < 32 || (c->kv_page_tokens & (c->kv_page_tokens - 1))) return false;
   if (c->kv_pool_pages < 0 || c->max_prefill_tokens < 0) return false;
+  if (c->act_split < 0 || c->act_split > 2) return false;
   return true;
+}
+
+// Split activations for the tensor cores (act16_put): on when asked, or
+// automatically when a token's path crosses more than kSplitDepth blocks.
+// Measured with the oracle on the 1.4B-class shape (24-layer body, L = 2, a
+// 1,088-position context): fp16 activations alone put the first token's
+// logits at relative L2 1.9e-3 from the fp64 result, fp16 K/V 1.2e-3, fp16
+// attention probabilities 0.9e-3, all three 2.4e-3 (the GPU: 2.39e-3),
+// against a bar of 2e-3; the 407M-class model at L = 32 (34 blocks) stays
+// at 1.5e-3 with fp16 activations.
+constexpr int kSplitDepth = 48;
+static int act_split_on(const tl_config* c) {
+  if (c->act_split != 0) return c->act_split == 1 ? 1 : 0;
+  return c->n_pre + c->L_max * c->n_loop_layers > kSplitDepth ? 1 : 0;
 }
 
 // TMA row coordinates into the KV pool are 32-bit signed.
@@ -217,9 +232,10 @@ static Layout make_layout(const tl_config* c) {
   L.act_q = take(R * d * 4);
   L.act_o = take(R * d * 4);
   L.act_u = take(R * F * 4);
-  L.act_a16 = take(R * d * 2);
-  L.act_o16 = take(R * d * 2);
-  L.act_u16 = take(R * F * 2);
+  const size_t s16 = (size_t)1 << act_split_on(c);  // [hi | lo] rows with split activations
+  L.act_a16 = take(R * d * 2 * s16);
+  L.act_o16 = take(R * d * 2 * s16);
+  L.act_u16 = take(R * F * 2 * s16);
   L.attn_part = take(lanes * c->n_heads * kAttnPieces * (hd + 2) * 4);
   L.attn_counters = take(lanes * c->n_heads * 4);
   L.part_val = take(lanes * L.n_parts * 4);
@@ -249,9 +265,9 @@ static Layout make_layout(const tl_config* c) {
   L.b_act_q = take(lanes * d * 4);
   L.b_act_o = take(lanes * d * 4);
   L.b_act_u = take(lanes * F * 4);
-  L.b_act_a16 = take(lanes * d * 2);
-  L.b_act_o16 = take(lanes * d * 2);
-  L.b_act_u16 = take(lanes * F * 2);
+  L.b_act_a16 = take(lanes * d * 2 * s16);
+  L.b_act_o16 = take(lanes * d * 2 * s16);
+  L.b_act_u16 = take(lanes * F * 2 * s16);
   L.b_attn_part = take(lanes * c->n_heads * kAttnPieces * (hd + 2) * 4);
   L.b_attn_counters = take(lanes * c->n_heads * 4);
   L.b_part_val = take(lanes * L.n_parts * 4);
@@ -299,6 +315,7 @@ struct tl_ctx {
   size_t ws_bytes;
   int hd;
   bool loaded = false;
+  int split16 = 0;  // tensor-core activation copies as [hi | lo] (act_split_on)
   MatView embed, head;
   std::vector<BlockW> pre, loop;
   const float* g_final;
@@ -576,7 +593,7 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
             const MatView* W2, const CUtensorMap* mw2, const ProjOut& o, __half* out16, int skip) {
   const int nmat = W2 ? 2 : 1;
   const int nt = tc_nt(max_rows);
-  const int S = o.epi == EPI_ARGMAX ? 1 : tc_splits(W.N, W.K, max_rows, nmat, W.fmt, W.group);
+  const int S = o.epi == EPI_ARGMAX ? 1 : tc_splits(W.N, W.K << c->split16, max_rows, nmat, W.fmt, W.group);
   dim3 grid((W.N + 127) / 128, (max_rows + nt - 1) / nt, S);
   TcParams p{};
   p.n_rows = n;
@@ -584,7 +601,9 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   p.N = W.N;
   p.K = W.K;
   p.group = W.group;
-  p.kb_per_split = (W.K / 64) / S;
+  p.kb_wrap = W.K / 64;
+  p.split16 = c->split16;
+  p.kb_per_split = ((W.K / 64) << c->split16) / S;
   p.scales = W.s;
   p.scales2 = W2 ? W2->s : nullptr;
   p.o = o;
@@ -592,7 +611,7 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
   p.status = c->status;
   const CUtensorMap& m2 = mw2 ? *mw2 : mw;
   if (max_rows >= kWideRows && o.epi != EPI_ARGMAX) {
-    p.kb_per_split = W.K / 64;
+    p.kb_per_split = (W.K / 64) << c->split16;
     const CUtensorMap& mxw = c->sc->xmap[xsel][nmat == 1 ? 2 : 1];  // 256-row tiles, 128 for the gate/up pair
     if (W.fmt == FMT_F16) {
       if (o.epi == EPI_SWIGLU) return tc_wide_launch<2, FMT_F16, EPI_SWIGLU>(c, max_rows, mw, m2, mxw, p);
@@ -686,7 +705,8 @@ int attn_launch_t(tl_ctx* c, const Rows& rows, int slot_base, int slot_stride, b
   return launch_k(c, kern, dim3(c->n_sms), dim3(AttnCfg<HD>::WARPS * 32), (size_t)smem, c->kvmap,
                   (const float*)c->sc->act_qkv, c->sc->act_o, c->sc->act_o16, rows, c->kv, (const float2*)c->rope, slot_base,
                   slot_stride, c->sc->attn_part, c->sc->attn_counters, c->status,
-                  cascade ? (const int32_t*)c->lane_shared : (const int32_t*)nullptr, (const float*)c->sc->casc);
+                  cascade ? (const int32_t*)c->lane_shared : (const int32_t*)nullptr, (const float*)c->sc->casc,
+                  c->split16);
 }
 
 // Shared-prefix ("cascade") pass of a decode step: for every loop iteration
@@ -726,7 +746,7 @@ int attn_split_launch(tl_ctx* c, dim3 grid, const Rows& rows, int slot_base, int
   }
   return launch_k(c, attn_split_kernel<HD>, grid, dim3(128), kAttnSplitSmem<HD>, (const float*)c->sc->act_qkv,
                   c->sc->act_o, c->sc->act_o16, rows, c->kv, (const float2*)c->rope, slot_base, slot_stride,
-                  c->sc->attn_part, c->sc->attn_counters, c->status);
+                  c->sc->attn_part, c->sc->attn_counters, c->status, c->split16);
 }
 
 int attn_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot_base, int slot_stride) {
@@ -762,7 +782,7 @@ int attn_prefill_launch_hd(tl_ctx* c, int max_rows, const Rows& rows, int slot, 
   }
   dim3 grid(tiles ? n_tiles : (max_rows + 63) / 64, c->cfg.n_heads);
   TL_TRY(launch_k(c, attn_prefill_kernel<HD>, dim3(grid), dim3(256), smem, c->sc->act_q, c->sc->act_o, c->sc->act_o16, rows,
-                  tiles, c->kv, slot, c->status));
+                  tiles, c->kv, slot, c->status, c->split16));
   return TL_OK;
 }
 
@@ -781,6 +801,7 @@ int attn_prefill_launch(tl_ctx* c, int max_rows, const Rows& rows, int slot, con
     p.mode = 0;
     p.o = c->sc->act_o;
     p.o16 = c->sc->act_o16;
+    p.split16 = c->split16;
     p.g = c->kv;
     p.slot_base = slot;
     p.slot_stride = 0;
@@ -829,7 +850,7 @@ int norm_for_proj(tl_ctx* c, int max_rows, int path, const int32_t* n, float* hb
     const int min_rows = (fused && path == PATH_AUTO) ? kGemvMaxRows : 0;  // <= 8 rows: the GEMV normalises
     const int grid = pend.rows > max_rows ? pend.rows : max_rows;
     TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(grid), dim3(256), 0, hbuf, map, n, c->cfg.d, g, c->cfg.rms_eps,
-                    c->sc->act_a, h_in, c->sc->act_a16, nullptr, 0, min_rows, pend.add, pend.n));
+                    c->sc->act_a, h_in, c->sc->act_a16, nullptr, 0, min_rows, pend.add, pend.n, c->split16));
   }
   return TL_OK;
 }
@@ -1121,8 +1142,9 @@ int encode_all_maps(tl_ctx* c) {
     const int nts[3] = {64, 128, 256};
     for (int x = 0; x < 3; ++x)
       for (int i = 0; i < 3; ++i)
-        TL_TRY(encode_2d(&sc.xmap[x][i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[x], (uint64_t)ks[x], (uint64_t)sc.rows,
-                         (uint64_t)ks[x] * 2, 64, nts[i], CU_TENSOR_MAP_SWIZZLE_128B));
+        TL_TRY(encode_2d(&sc.xmap[x][i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs[x], (uint64_t)ks[x] << c->split16,
+                         (uint64_t)sc.rows, ((uint64_t)ks[x] << c->split16) * 2, 64, nts[i],
+                         CU_TENSOR_MAP_SWIZZLE_128B));
   }
   return TL_OK;
 }
@@ -1198,6 +1220,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->ws = (char*)dev_ws;
   c->ws_bytes = bytes;
   c->hd = cfg->d / cfg->n_heads;
+  c->split16 = act_split_on(cfg);
   if (const char* e = std::getenv("TL_PDL")) c->pdl = std::strcmp(e, "0") != 0;
   char* w = c->ws;
   // weight views
@@ -1614,7 +1637,7 @@ static int prefill_impl(tl_ctx* c, const std::vector<PromptLane>& in, int32_t sh
   if (pend.add)  // the last block's residual (the norm kernel with no rows to normalise only adds)
     TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(pend.rows), dim3(256), 0, c->hrows, (const int32_t*)nullptr,
                     (const int32_t*)(c->pf_n + Lmax), cfg.d, (const float*)nullptr, cfg.rms_eps, (float*)nullptr,
-                    (float*)nullptr, (__half*)nullptr, (float*)nullptr, 0, 0, pend.add, pend.n));
+                    (float*)nullptr, (__half*)nullptr, (float*)nullptr, 0, 0, pend.add, pend.n, 0));
   TL_TRY(launch_k(c, prefill_finish_batch_kernel, dim3(n), dim3(256), 0, c->lanes, c->pf_info, n, c->hrows, c->h,
                   cfg.d));
   if (dev_hidden_out)
@@ -1685,7 +1708,7 @@ static int rerun_positions(tl_ctx* c, int lane, int pos0, int k, int L) {
   if (pend.add)
     TL_TRY(launch_k(c, rmsnorm_rows_kernel, dim3(pend.rows), dim3(256), 0, c->hrows, (const int32_t*)nullptr,
                     (const int32_t*)(c->pf_n + L), cfg.d, (const float*)nullptr, cfg.rms_eps, (float*)nullptr,
-                    (float*)nullptr, (__half*)nullptr, (float*)nullptr, 0, 0, pend.add, pend.n));
+                    (float*)nullptr, (__half*)nullptr, (float*)nullptr, 0, 0, pend.add, pend.n, 0));
   c->prefill_tokens += k;
   return TL_OK;
 }

@@ -36,6 +36,9 @@ struct TcParams {
   int32_t skip_at_or_below;
   int32_t N, K, group;
   int32_t kb_per_split;    // 64-wide k-blocks per split
+  int32_t kb_wrap;         // k-blocks of the weights, K / 64
+  int32_t split16;         // activation rows are [hi | lo] (see act16_put): 2 * kb_wrap k-blocks, block kb
+                           // multiplies weight block kb % kb_wrap
   const __half* scales;    // INT4: [N][K/group]
   const __half* scales2;   // second matrix (gate/up pair)
   ProjOut o;               // EPI_STORE / EPI_SWIGLU: o.out [rows][ldo]; EPI_RESID: o.h / o.map
@@ -141,7 +144,7 @@ __device__ __forceinline__ void tc_emit(const TcParams& p, int row, int m, float
   } else if constexpr (EPI == EPI_SWIGLU) {
     const float u = silu_f(v) * v2;
     if (o.out) o.out[(int64_t)row * o.ldo + m] = u;
-    if (p.out16) p.out16[(int64_t)row * o.ldo + m] = __float2half_rn(u);
+    if (p.out16) act16_put(p.out16, row, o.ldo, m, u, p.split16);
   } else if constexpr (EPI == EPI_RESID) {
     const int hr = o.map ? o.map[row] : row;
     o.h[(int64_t)hr * p.N + m] += v;
@@ -231,8 +234,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     for (int i = 0; i < pre; ++i) {
       const uint32_t fb = smem_u32(&full[i]);
       mbar_add_tx(fb, NMAT * C::RAW_BYTES);
-      const int kb = kb0 + i;
-      const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
+      const int kbw = (kb0 + i) % p.kb_wrap;
+      const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
       tma_load_2d(smem_u32(sRaw + (i * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
       if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (i * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
     }
@@ -264,7 +267,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
           mbar_expect_tx(fb, C::B_BYTES);
         } else {
           mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
-          const int wx = (FMT == TL_FMT_INT4) ? kb * 32 : kb * 64;
+          const int kbw = kb % p.kb_wrap;
+          const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
           tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
           if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
         }
@@ -308,10 +312,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     // ------------------------------------------------- convert + epilogue
     const int t = threadIdx.x - 128;  // weight row within the tile == TMEM lane
     const int q = warp - 4;
-    const int gfirst = (FMT == TL_FMT_INT4) ? (kb0 * 64) / p.group : 0;
+    // (split activations: the CTA's range may wrap around K, so all of the row's groups)
+    const int gfirst = (FMT == TL_FMT_INT4 && !p.split16) ? (kb0 * 64) / p.group : 0;
     if constexpr (FMT == TL_FMT_INT4) {
       // this row's group scales for the CTA's K range (while the first TMA is in flight)
-      const int glast = ((kb0 + nkb) * 64 - 1) / p.group;
+      const int glast = p.split16 ? p.K / p.group - 1 : ((kb0 + nkb) * 64 - 1) / p.group;
       for (int mat = 0; mat < NMAT; ++mat) {
         const __half* sc = mat == 0 ? p.scales : p.scales2;
         const int64_t rowoff = (int64_t)(m0 + t) * (p.K / p.group);
@@ -331,7 +336,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
           const uint4 w0 = *reinterpret_cast<const uint4*>(raw + t * 32);
           const uint4 w1 = *reinterpret_cast<const uint4*>(raw + t * 32 + 16);
           const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          const int kbase = (kb0 + i) * 64;
+          const int kbase = ((kb0 + i) % p.kb_wrap) * 64;
           const __half* srow = sSc + (mat * 128 + t) * TC_SC_MAX;
           if (p.group % 64 == 0) {  // the k-block lies inside one scale group
             const __half sc = srow[kbase / p.group - gfirst];

@@ -68,7 +68,17 @@ typedef enum tl_weight_fmt {
 /* Model and capacity.  d = n_heads * head_dim with head_dim 32, 64 or 128;
  * d and ffn multiples of 64 (the tensor-core projections take K in 64-wide
  * blocks); for INT4, group a multiple of 32 dividing d and ffn, with at
- * most 32 groups across d and across ffn. */
+ * most 32 groups across d and across ffn.
+ *
+ * act_split: the tensor-core projections (rows above 8) multiply fp16 copies
+ * of the activations.  Split, each copy is hi = fp16(x) and lo = fp16(x - hi)
+ * and the projection sums both products (twice the MMAs), which keeps the
+ * activations' fp32 precision to ~2^-22; single, one fp16 rounding (2^-11)
+ * per projection input.  Automatic: split when a token's path crosses more
+ * than 48 blocks (n_pre + L_max * n_loop_layers): the error of single fp16
+ * grows with depth, and at 96 blocks (a 24-layer body at L = 4) it takes the
+ * logits past relative L2 2e-3 from the exact model.  The few-row CUDA-core
+ * projections keep fp32 activations either way. */
 typedef struct tl_config {
     int32_t vocab;
     int32_t d;
@@ -89,6 +99,8 @@ typedef struct tl_config {
     int32_t kv_pool_pages;    /* pages in the pool; 0 = one per lane/slot/page    */
     int32_t max_prefill_tokens; /* prompt rows one prefill call computes, summed
                                    over its lanes; 0 = max_seq                   */
+    int32_t act_split;        /* activations for the tensor-core projections:
+                                 0 automatic, 1 split, 2 single fp16 (below)     */
 } tl_config;
 
 typedef struct tl_ctx tl_ctx;

@@ -117,13 +117,14 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, q_pos: np.ndarray, k_pos
     """Causal multi-head attention. q [T,H,hd], K/V [S,H,hd]; key s is visible to
     query t iff k_pos[s] <= q_pos[t].  Max-subtracted softmax, scale 1/sqrt(hd)."""
     hd = q.shape[-1]
-    scores = np.einsum("thd,shd->hts", q, K) / np.sqrt(hd)
+    # per head: scores = Q K^T [T, S], then softmax(scores) V [T, hd] (batched matrix products over heads)
+    scores = np.matmul(q.transpose(1, 0, 2), K.transpose(1, 2, 0)) / np.sqrt(hd)
     visible = k_pos[None, :] <= q_pos[:, None]
     scores = np.where(visible[None], scores, -np.inf)
     scores = scores - scores.max(axis=-1, keepdims=True)
     p = np.exp(scores)
     p = p / p.sum(axis=-1, keepdims=True)
-    return np.einsum("hts,shd->thd", p, V)
+    return np.matmul(p, V.transpose(1, 0, 2)).transpose(1, 0, 2)
 
 
 # ---------------------------------------------------------------- KV cache ----

@@ -18,7 +18,7 @@ from test_gpu_wide_paths import _compare, _teacher_forced_subset
 pytestmark = pytest.mark.gpu
 
 
-def _run(name, n, Tp, Ts, n_new, page, check, gain_seed=None, cascade=True, seed=131):
+def _run(name, n, Tp, Ts, n_new, page, check, gain_seed=None, cascade=True, seed=131, act_split=0):
     sh = S.SHAPES[name]
     rng = np.random.Generator(np.random.PCG64(seed))
     pre = rng.integers(0, sh.vocab, Tp).astype(np.int32)
@@ -27,7 +27,7 @@ def _run(name, n, Tp, Ts, n_new, page, check, gain_seed=None, cascade=True, seed
     prompts = [np.concatenate([pre, suf[i]]) for i in range(n)]
     donor = n
     m = gpu_model(name, gain_seed, max_lanes=n + 1, max_seq=Tp + Ts + n_new, L_max=4, kv_page_tokens=page,
-                  max_prefill_tokens=max(Tp + Ts, n * Ts))
+                  max_prefill_tokens=max(Tp + Ts, n * Ts), act_split=act_split)
     m.set_cascade(cascade)
     m.prefill(donor, pre, 4)
     m.prefill_batch(list(range(n)), prompts, Ls, share_from=donor, shared_tokens=Tp)
