@@ -123,7 +123,14 @@ enum ProjPath { PATH_AUTO = 0, PATH_GEMV = 1, PATH_TC = 2 };
 // and 8 row accumulators each)
 constexpr int head_rpw(int fmt) { return fmt == TL_FMT_INT4 ? 4 : 2; }
 
-static int tc_nt(int max_rows) { return max_rows <= 64 ? 64 : (max_rows <= 128 ? 128 : 256); }
+// Activation rows per tensor-core tile.  The gate/up pair stays at 128 above
+// 128 rows: its 256-row tile cannot split K (the pair's partial tiles would
+// need 256 KB of shared memory), which left a 256-row step with one CTA per
+// 128 weight rows (44 CTAs for a 5,632-wide FFN: 74 us per launch).
+static int tc_nt(int max_rows, int nmat = 1) {
+  if (max_rows <= 64) return 64;
+  return (max_rows <= 128 || nmat == 2) ? 128 : 256;
+}
 
 template <int NMAT, int FMT>
 static bool tc_split_ok(int nt) {
@@ -136,7 +143,7 @@ static bool tc_split_ok(int nt) {
 // keeps >= 2 k-blocks; its INT4 scale groups stay within TC_SC_MAX because the
 // configuration allows at most TC_SC_MAX - 1 groups over the whole K.
 static int tc_splits(int N, int K, int max_rows, int nmat, int fmt, int group) {
-  const int nt = tc_nt(max_rows);
+  const int nt = tc_nt(max_rows, nmat);
   const bool ok = nmat == 1 ? (fmt == TL_FMT_INT4 ? tc_split_ok<1, TL_FMT_INT4>(nt) : tc_split_ok<1, TL_FMT_BF16>(nt))
                             : (fmt == TL_FMT_INT4 ? tc_split_ok<2, TL_FMT_INT4>(nt) : tc_split_ok<2, TL_FMT_BF16>(nt));
   const int m_tiles = (N + 127) / 128, n_tiles = (max_rows + nt - 1) / nt;
@@ -592,7 +599,7 @@ constexpr int kWideRows = 512;
 int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& W, const CUtensorMap& mw,
             const MatView* W2, const CUtensorMap* mw2, const ProjOut& o, __half* out16, int skip) {
   const int nmat = W2 ? 2 : 1;
-  const int nt = tc_nt(max_rows);
+  const int nt = tc_nt(max_rows, nmat);
   const int S = o.epi == EPI_ARGMAX ? 1 : tc_splits(W.N, W.K << c->split16, max_rows, nmat, W.fmt, W.group);
   dim3 grid((W.N + 127) / 128, (max_rows + nt - 1) / nt, S);
   TcParams p{};
