@@ -37,8 +37,7 @@ struct TcParams {
   int32_t N, K, group;
   int32_t kb_per_split;    // 64-wide k-blocks per split
   int32_t kb_wrap;         // k-blocks of the weights, K / 64
-  int32_t split16;         // activation rows are [hi | lo] (see act16_put): 2 * kb_wrap k-blocks, block kb
-                           // multiplies weight block kb % kb_wrap
+  int32_t split16;         // activation rows are [hi | lo] (see act16_put): 2 * kb_wrap k-steps (below)
   const __half* scales;    // INT4: [N][K/group]
   const __half* scales2;   // second matrix (gate/up pair)
   ProjOut o;               // EPI_STORE / EPI_SWIGLU: o.out [rows][ldo]; EPI_RESID: o.h / o.map
@@ -47,6 +46,15 @@ struct TcParams {
 };
 
 constexpr int TC_SC_MAX = 33;  // scale groups per CTA row
+
+// k-step j of a projection: weight block tc_wblock, activation block
+// tc_xblock.  With split activations a weight block's hi and lo products run
+// back to back (steps 2w and 2w + 1), so its second read comes from L2 and a
+// CTA's k-steps cover a contiguous range of weight blocks.
+__device__ __forceinline__ int tc_wblock(const TcParams& p, int j) { return j >> p.split16; }
+__device__ __forceinline__ int tc_xblock(const TcParams& p, int j) {
+  return p.split16 ? (j & 1) * p.kb_wrap + (j >> 1) : j;
+}
 
 template <int NT, int NMAT, int FMT>
 struct TcCfg {
@@ -234,7 +242,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     for (int i = 0; i < pre; ++i) {
       const uint32_t fb = smem_u32(&full[i]);
       mbar_add_tx(fb, NMAT * C::RAW_BYTES);
-      const int kbw = (kb0 + i) % p.kb_wrap;
+      const int kbw = tc_wblock(p, kb0 + i);
       const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
       tma_load_2d(smem_u32(sRaw + (i * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
       if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (i * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
@@ -267,12 +275,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
           mbar_expect_tx(fb, C::B_BYTES);
         } else {
           mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
-          const int kbw = kb % p.kb_wrap;
+          const int kbw = tc_wblock(p, kb);
           const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
           tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
           if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
         }
-        tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
+        tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, tc_xblock(p, kb) * 64, n0, fb);
       }
       __syncwarp();
       issued = i + 1;
@@ -312,11 +320,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     // ------------------------------------------------- convert + epilogue
     const int t = threadIdx.x - 128;  // weight row within the tile == TMEM lane
     const int q = warp - 4;
-    // (split activations: the CTA's range may wrap around K, so all of the row's groups)
-    const int gfirst = (FMT == TL_FMT_INT4 && !p.split16) ? (kb0 * 64) / p.group : 0;
+    const int gfirst = (FMT == TL_FMT_INT4) ? (tc_wblock(p, kb0) * 64) / p.group : 0;
     if constexpr (FMT == TL_FMT_INT4) {
       // this row's group scales for the CTA's K range (while the first TMA is in flight)
-      const int glast = p.split16 ? p.K / p.group - 1 : ((kb0 + nkb) * 64 - 1) / p.group;
+      const int glast = ((tc_wblock(p, kb0 + nkb - 1) + 1) * 64 - 1) / p.group;
       for (int mat = 0; mat < NMAT; ++mat) {
         const __half* sc = mat == 0 ? p.scales : p.scales2;
         const int64_t rowoff = (int64_t)(m0 + t) * (p.K / p.group);
@@ -336,7 +343,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
           const uint4 w0 = *reinterpret_cast<const uint4*>(raw + t * 32);
           const uint4 w1 = *reinterpret_cast<const uint4*>(raw + t * 32 + 16);
           const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          const int kbase = ((kb0 + i) % p.kb_wrap) * 64;
+          const int kbase = tc_wblock(p, kb0 + i) * 64;
           const __half* srow = sSc + (mat * 128 + t) * TC_SC_MAX;
           if (p.group % 64 == 0) {  // the k-block lies inside one scale group
             const __half sc = srow[kbase / p.group - gfirst];

@@ -127,7 +127,7 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
   const int m_tiles = (p.N + 127) / 128;
   const int n_tiles = rows > p.skip_at_or_below ? (rows + NT - 1) / NT : 0;
   const int n_total = m_tiles * n_tiles;
-  const int nkb = p.kb_wrap << p.split16;  // activation k-blocks (split: [hi | lo], weights wrap around)
+  const int nkb = p.kb_wrap << p.split16;  // k-steps (split activations: two per weight block, tc_xblock)
   const int nks = (nkb + KPS - 1) / KPS;  // pipeline steps per tile
 
   if (warp == 0) {
@@ -146,19 +146,19 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
           if constexpr (FMT == FMT_F16) {  // fp16 weight tiles straight into the MMA layout
             mbar_expect_tx(fb, nq * (NMAT * C::A_BYTES + C::B_BYTES));
             for (int q = 0; q < nq; ++q) {
-              const int kb = ks * KPS + q, kbw = kb % p.kb_wrap;
+              const int kb = ks * KPS + q, kbw = tc_wblock(p, kb);
               tma_load_2d(smem_u32(sA + ((s * NMAT + 0) * KPS + q) * C::A_BYTES), &mapW, kbw * 64, m0, fb);
               if constexpr (NMAT == 2)
                 tma_load_2d(smem_u32(sA + ((s * NMAT + 1) * KPS + q) * C::A_BYTES), &mapW2, kbw * 64, m0, fb);
-              tma_load_2d(smem_u32(sB + (s * KPS + q) * C::B_BYTES), &mapX, kb * 64, n0, fb);
+              tma_load_2d(smem_u32(sB + (s * KPS + q) * C::B_BYTES), &mapX, tc_xblock(p, kb) * 64, n0, fb);
             }
           } else {
-            const int kb = ks, kbw = kb % p.kb_wrap;
+            const int kb = ks, kbw = tc_wblock(p, kb);
             mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
             const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
             tma_load_2d(smem_u32(sRaw + (s * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
             if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (s * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
-            tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, kb * 64, n0, fb);
+            tma_load_2d(smem_u32(sB + s * C::B_BYTES), &mapX, tc_xblock(p, kb) * 64, n0, fb);
           }
         }
       }
@@ -218,7 +218,7 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
     // INT4: this row's scales of a k-block, fetched one k-block ahead of their use
     auto fetch_scales = [&](int t, int kb_act, __half (&out)[NMAT][8]) {
       const int m = (t % m_tiles) * 128 + tr;
-      const int kb = kb_act % p.kb_wrap;
+      const int kb = tc_wblock(p, kb_act);
 #pragma unroll
       for (int mat = 0; mat < NMAT; ++mat) {
         const __half* sc = (mat == 0 ? p.scales : p.scales2) + (int64_t)m * gpr;
