@@ -34,17 +34,19 @@ namespace tl {
 // slower: the split partials and their combine cost more than the waves save).
 constexpr int kAttnCtaTarget = 4 * 148;
 
-// Keys of one ring stage: 16 (two lanes per key) from head dim 64, 32 (one
-// per lane) below.
+// Keys of one ring stage: 32 (one per lane) at head dim 32, 16 (two lanes per
+// key) at 64, 8 (four lanes per key) at 128: 2 KB of keys and 2 KB of values.
 template <int HD>
-constexpr int kAttnKeys = HD >= 64 ? 16 : 32;
+constexpr int kAttnKeys = HD >= 128 ? 8 : (HD >= 64 ? 16 : 32);
 // Bytes of one stage's keys (or values) of one head.
 template <int HD>
 constexpr int kAttnBlockBytes = kAttnKeys<HD> * HD * 2;
-// Ring stages per warp: as many as 16 KB per warp holds (4 at head dims 32
-// and 64, 2 at 128), so a CTA takes 64 KB and three share an SM.
+// Ring stages per warp: two, so a CTA takes 32 KB and six share an SM; the
+// CTAs of a 64-row step then run in about one wave.  Measured at 64 lanes
+// (hd 64): 34.0k tokens/s with 2 stages of 16 keys, 32.7k with 3, 31.5-32.0k
+// with 4 (three CTAs per SM); 8-key stages 33.0-33.6k.
 template <int HD>
-constexpr int kAttnStages = (8 * 1024) / kAttnBlockBytes<HD> >= 4 ? 4 : 2;
+constexpr int kAttnStages = 2;
 // Dynamic shared memory of attn_split_kernel: per warp, its stages of keys and values.
 template <int HD>
 constexpr int kAttnSplitSmem = 4 * kAttnStages<HD> * 2 * kAttnBlockBytes<HD>;
@@ -192,7 +194,8 @@ attn_split_kernel(const float* __restrict__ qkv, float* __restrict__ o, __half* 
           dot = fmaf(qs[8 * c + 2 * e + 1], f.y, dot);
         }
       }
-      if constexpr (LPK == 2) dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+      if constexpr (LPK >= 2) dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+      if constexpr (LPK >= 4) dot += __shfl_xor_sync(0xffffffffu, dot, 8);
       if (j < ctx) s = dot;
     }
     const float mb = warp_max(s);
