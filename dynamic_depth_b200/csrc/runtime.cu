@@ -70,6 +70,11 @@ static bool cfg_valid(const tl_config* c) {
 // against a bar of 2e-3; the 407M-class model at L = 32 (34 blocks) stays
 // at 1.5e-3 with fp16 activations.
 constexpr int kSplitDepth = 48;
+
+// Blocks whose matrices are BF16 (pre blocks first, then the loop body's layers).
+static int n_f16_blocks(const tl_config* c) {
+  return (c->fmt_pre == TL_FMT_BF16 ? c->n_pre : 0) + (c->fmt_loop == TL_FMT_BF16 ? c->n_loop_layers : 0);
+}
 static int act_split_on(const tl_config* c) {
   if (c->act_split != 0) return c->act_split == 1 ? 1 : 0;
   return c->n_pre + c->L_max * c->n_loop_layers > kSplitDepth ? 1 : 0;
@@ -144,8 +149,12 @@ static bool tc_split_ok(int nt) {
 // configuration allows at most TC_SC_MAX - 1 groups over the whole K.
 static int tc_splits(int N, int K, int max_rows, int nmat, int fmt, int group) {
   const int nt = tc_nt(max_rows, nmat);
-  const bool ok = nmat == 1 ? (fmt == TL_FMT_INT4 ? tc_split_ok<1, TL_FMT_INT4>(nt) : tc_split_ok<1, TL_FMT_BF16>(nt))
-                            : (fmt == TL_FMT_INT4 ? tc_split_ok<2, TL_FMT_INT4>(nt) : tc_split_ok<2, TL_FMT_BF16>(nt));
+  const bool ok = nmat == 1 ? (fmt == TL_FMT_INT4 ? tc_split_ok<1, TL_FMT_INT4>(nt)
+                                                 : (fmt == FMT_F16 ? tc_split_ok<1, FMT_F16>(nt)
+                                                                   : tc_split_ok<1, TL_FMT_BF16>(nt)))
+                            : (fmt == TL_FMT_INT4 ? tc_split_ok<2, TL_FMT_INT4>(nt)
+                                                 : (fmt == FMT_F16 ? tc_split_ok<2, FMT_F16>(nt)
+                                                                   : tc_split_ok<2, TL_FMT_BF16>(nt)));
   const int m_tiles = (N + 127) / 128, n_tiles = (max_rows + nt - 1) / nt;
   const int kb = K / 64;
   const int slots = (nmat == 1 && nt == 64) ? 296 : 148;
@@ -202,7 +211,7 @@ struct Layout {
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[6], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
       mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec, lane_shared, casc, wstage,
-      out_tok, out_dep, status, counters, body_kernels, alive, b_act_a, b_act_qkv, b_act_q, b_act_o, b_act_u,
+      f16blk, out_tok, out_dep, status, counters, body_kernels, alive, b_act_a, b_act_qkv, b_act_q, b_act_o, b_act_u,
       b_act_a16, b_act_o16, b_act_u16, b_attn_part, b_attn_counters, b_part_val, b_part_idx, b_casc, total;
 };
 
@@ -260,6 +269,9 @@ static Layout make_layout(const tl_config* c) {
   L.casc = take(lanes * c->n_heads * (hd + 2) * 4);
   // prompt batches wide enough for the persistent GEMM: one block's five matrices in fp16
   L.wstage = take(L.max_prefill >= 512 ? (size_t)(4 * d * d + 3 * d * F) * 2 : 0);
+  // BF16 blocks: a resident fp16 copy of every matrix (the same bytes per weight), so the tensor-core
+  // projections load weight tiles straight into the MMA layout instead of converting them every step
+  L.f16blk = take((size_t)n_f16_blocks(c) * (4 * d * d + 3 * d * F) * 2);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
   L.status = take(4);
@@ -288,6 +300,7 @@ struct BlockW {
   MatView wqkv, wo, wg, wu, wd;
   const float *g1, *g2;
   CUtensorMap mqkv, mo, mg, mu, md;  // TMA maps of the raw weight tiles
+  const BlockW* f16 = nullptr;       // BF16 blocks: the resident fp16 copy the tensor-core projections read
 };
 
 // Row-wise scratch of one stream of projection / attention / head kernels.  A
@@ -343,6 +356,7 @@ struct tl_ctx {
   bool cascade_active = false;  // enabled, and the lanes that share map one donor's prefix of one length
   __half* wstage = nullptr;     // fp16 staging copy of one block's matrices for wide prompt batches
   BlockW sblock{};              // views and TMA maps of that copy
+  std::vector<BlockW> blk16;    // resident fp16 copies of BF16 blocks (see BlockW::f16)
   const BlockW* staged_src = nullptr;  // the block whose matrices the copy holds
   int32_t *tok_stage, *L_stage, *out_tok, *out_dep, *status, *alive;
   int32_t* pf_n;     // prompt batches: row count of each stage (stage l = loop iteration l)
@@ -635,6 +649,12 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
     return tc_wide_launch<1, TL_FMT_BF16, EPI_STORE>(c, max_rows, mw, m2, mxw, p);
   }
   const CUtensorMap& mx = c->sc->xmap[xsel][nt == 64 ? 0 : (nt == 128 ? 1 : 2)];
+  if (W.fmt == FMT_F16) {  // (block matrices only: the head keeps its own format)
+    if (o.epi == EPI_ARGMAX) return TL_EINVAL;
+    if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, FMT_F16, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);
+    if (o.epi == EPI_RESID) return tc_launch_nt<1, FMT_F16, EPI_RESID>(c, nt, mw, m2, mx, p, grid);
+    return tc_launch_nt<1, FMT_F16, EPI_STORE>(c, nt, mw, m2, mx, p, grid);
+  }
   if (W.fmt == TL_FMT_INT4) {
     if (o.epi == EPI_ARGMAX) return tc_launch_nt<1, TL_FMT_INT4, EPI_ARGMAX>(c, nt, mw, m2, mx, p, grid);
     if (o.epi == EPI_SWIGLU) return tc_launch_nt<2, TL_FMT_INT4, EPI_SWIGLU>(c, nt, mw, m2, mx, p, grid);
@@ -654,9 +674,18 @@ int tc_proj(tl_ctx* c, int max_rows, int xsel, const int32_t* n, const MatView& 
 // caller knows which applies (prompts, or a graph branch chosen on the
 // device), and only that one is launched.  nrm: see small_rows_proj (the
 // tensor-core variant reads the fp16 copy of a separate norm kernel).
+// tw (optional): the matrices and maps the tensor-core variant reads instead (a BF16 block's resident
+// fp16 copy; the GEMV keeps the exact BF16 weights).
+struct TcTwin {
+  const MatView* W;
+  const CUtensorMap* mw;
+  const MatView* W2;
+  const CUtensorMap* mw2;
+};
+
 int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int32_t* n, const MatView& W,
          const CUtensorMap* mw, const MatView* W2, const CUtensorMap* mw2, ProjOut o, __half* out16,
-         int prof_kind = TL_PROF_PROJ, const GsNorm* nrm = nullptr) {
+         int prof_kind = TL_PROF_PROJ, const GsNorm* nrm = nullptr, const TcTwin* tw = nullptr) {
   const MatView& w2 = W2 ? *W2 : W;
   TL_TRY(prof_start(c, prof_kind));
   const bool argmax = o.epi == EPI_ARGMAX;
@@ -684,7 +713,11 @@ int proj(tl_ctx* c, int max_rows, int path, const float* X, int xsel, const int3
   }
   if (use_tc) {
     if (argmax) o.n_parts = (W.N + 127) / 128;  // one partial per 128-row tile
-    TL_TRY(tc_proj(c, max_rows, xsel, n, W, *mw, W2, mw2, o, out16, path == PATH_AUTO ? kGemvMaxRows : 0));
+    if (tw)
+      TL_TRY(tc_proj(c, max_rows, xsel, n, *tw->W, *tw->mw, tw->W2, tw->mw2, o, out16,
+                     path == PATH_AUTO ? kGemvMaxRows : 0));
+    else
+      TL_TRY(tc_proj(c, max_rows, xsel, n, W, *mw, W2, mw2, o, out16, path == PATH_AUTO ? kGemvMaxRows : 0));
   }
   return prof_stop(c, prof_kind);
 }
@@ -879,7 +912,7 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   const bool defer = pend && prompt && max_rows >= kWideRows;
   // prompt batches on the persistent GEMM read an fp16 copy of the block's matrices, made once per pass and
   // block (the loop block once for all its iterations), instead of dequantising every tile again
-  const bool staged = prompt && max_rows >= kWideRows && c->wstage;
+  const bool staged = prompt && max_rows >= kWideRows && c->wstage && !w.f16;
   if (staged && c->staged_src != &w) {
     const MatView* src[5] = {&w.wqkv, &w.wo, &w.wg, &w.wu, &w.wd};
     const MatView* dst[5] = {&c->sblock.wqkv, &c->sblock.wo, &c->sblock.wg, &c->sblock.wu, &c->sblock.wd};
@@ -891,6 +924,12 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
     c->staged_src = &w;
   }
   const BlockW& pw = staged ? c->sblock : w;  // the projections' matrices and maps
+  // a BF16 block's tensor-core variants read its resident fp16 copy
+  const BlockW* tb = w.f16;
+  const TcTwin t_qkv{tb ? &tb->wqkv : nullptr, tb ? &tb->mqkv : nullptr, nullptr, nullptr};
+  const TcTwin t_o{tb ? &tb->wo : nullptr, tb ? &tb->mo : nullptr, nullptr, nullptr};
+  const TcTwin t_gu{tb ? &tb->wg : nullptr, tb ? &tb->mg : nullptr, tb ? &tb->wu : nullptr, tb ? &tb->mu : nullptr};
+  const TcTwin t_d{tb ? &tb->wd : nullptr, tb ? &tb->md : nullptr, nullptr, nullptr};
   const float* X = nullptr;
   GsNorm nrm{};
   bool use_nrm = false;
@@ -902,7 +941,7 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   o.out = c->sc->act_qkv;
   o.ldo = 3 * d;
   TL_TRY(proj(c, max_rows, path, X, 0, rows.n, pw.wqkv, &pw.mqkv, nullptr, nullptr, o, nullptr, TL_PROF_PROJ,
-              use_nrm ? &nrm : nullptr));
+              use_nrm ? &nrm : nullptr, tb ? &t_qkv : nullptr));
   if (prompt) {
     TL_TRY(launch_k(c, rope_kv_kernel, dim3(max_rows), dim3(d / 2), 0, c->sc->act_qkv, c->sc->act_q, rows, c->kv, c->rope,
                     slot_base, slot_stride, nullptr, c->status));
@@ -919,7 +958,8 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
     r.out = c->sc->act_q;
     r.ldo = d;
   }
-  TL_TRY(proj(c, max_rows, path, c->sc->act_o, 1, rows.n, pw.wo, &pw.mo, nullptr, nullptr, r, nullptr));
+  TL_TRY(proj(c, max_rows, path, c->sc->act_o, 1, rows.n, pw.wo, &pw.mo, nullptr, nullptr, r, nullptr, TL_PROF_PROJ,
+              nullptr, tb ? &t_o : nullptr));
   TL_TRY(norm_for_proj(c, max_rows, path, rows.n, hbuf, map, w.g2, nullptr, w.wg, 2, &X, &nrm, &use_nrm,
                        defer ? PendingAdd{c->sc->act_q, rows.n, max_rows} : PendingAdd{}));
   ProjOut sw{};
@@ -928,8 +968,9 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   sw.out = (path == PATH_TC && max_rows > kGemvMaxRows) ? nullptr : c->sc->act_u;
   sw.ldo = F;
   TL_TRY(proj(c, max_rows, path, X, 0, rows.n, pw.wg, &pw.mg, &pw.wu, &pw.mu, sw, c->sc->act_u16, TL_PROF_PROJ,
-              use_nrm ? &nrm : nullptr));
-  TL_TRY(proj(c, max_rows, path, c->sc->act_u, 2, rows.n, pw.wd, &pw.md, nullptr, nullptr, r, nullptr));
+              use_nrm ? &nrm : nullptr, tb ? &t_gu : nullptr));
+  TL_TRY(proj(c, max_rows, path, c->sc->act_u, 2, rows.n, pw.wd, &pw.md, nullptr, nullptr, r, nullptr, TL_PROF_PROJ,
+              nullptr, tb ? &t_d : nullptr));
   if (defer) *pend = PendingAdd{c->sc->act_q, rows.n, max_rows};
   return TL_OK;
 }
@@ -1128,6 +1169,13 @@ int encode_all_maps(tl_ctx* c) {
       TL_TRY(encode_weight_map(&b.md, b.wd));
     }
   TL_TRY(encode_weight_map(&c->mhead, c->head));
+  for (BlockW& b : c->blk16) {  // fp16 tiles of 128 rows x 64 K, in the MMA's swizzled layout
+    const MatView* mv5[5] = {&b.wqkv, &b.wo, &b.wg, &b.wu, &b.wd};
+    CUtensorMap* mp5[5] = {&b.mqkv, &b.mo, &b.mg, &b.mu, &b.md};
+    for (int i = 0; i < 5; ++i)
+      TL_TRY(encode_2d(mp5[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv5[i]->bf, (uint64_t)mv5[i]->K, (uint64_t)mv5[i]->N,
+                       (uint64_t)mv5[i]->K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  }
   if (c->wstage) {  // the staging copy: fp16 tiles of 128 rows x 64 K, in the MMA's swizzled layout
     BlockW& b = c->sblock;
     const MatView* mv5[5] = {&b.wqkv, &b.wo, &b.wg, &b.wu, &b.wd};
@@ -1256,6 +1304,28 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     BlockW bw{mv[1 + 5 * b], mv[2 + 5 * b], mv[3 + 5 * b], mv[4 + 5 * b], mv[5 + 5 * b],
               gains + (size_t)(2 * b) * cfg->d, gains + (size_t)(2 * b + 1) * cfg->d};
     (b < cfg->n_pre ? c->pre : c->loop).push_back(bw);
+  }
+  {  // resident fp16 copies of the BF16 blocks, in block order (filled by tl_load_weights)
+    const int64_t d = cfg->d, F = cfg->ffn;
+    const int64_t off[5] = {0, 3 * d * d, 4 * d * d, 4 * d * d + F * d, 4 * d * d + 2 * F * d};
+    const int64_t NN[5] = {3 * d, d, F, F, d}, KK[5] = {d, d, d, d, F};
+    c->blk16.reserve(nb);  // (BlockW::f16 points into it)
+    __half* base = (__half*)(w + lay.f16blk);
+    for (int b = 0; b < nb; ++b) {
+      BlockW& src = b < cfg->n_pre ? c->pre[b] : c->loop[b - cfg->n_pre];
+      if (src.wqkv.fmt != TL_FMT_BF16) continue;
+      BlockW cp = src;
+      MatView* mv5[5] = {&cp.wqkv, &cp.wo, &cp.wg, &cp.wu, &cp.wd};
+      for (int i = 0; i < 5; ++i) {
+        mv5[i]->fmt = FMT_F16;
+        mv5[i]->N = (int)NN[i];
+        mv5[i]->K = (int)KK[i];
+        mv5[i]->bf = reinterpret_cast<const uint16_t*>(base + off[i]);
+      }
+      base += 4 * d * d + 3 * d * F;
+      c->blk16.push_back(cp);
+      src.f16 = &c->blk16.back();
+    }
   }
   c->g_final = gains + (size_t)(2 * nb) * cfg->d;
   c->rope = (float2*)(w + lay.rope);
@@ -1474,6 +1544,18 @@ extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
     const int64_t words = (int64_t)m->N * m->K / 8;
     TL_TRY(launch_k(c, int4_repack_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, (uint32_t*)m->q, words));
   }
+  // the resident fp16 copies of the BF16 blocks (the conversion the tensor-core kernels applied per tile)
+  for (auto* v : {&c->pre, &c->loop})
+    for (const BlockW& bw : *v) {
+      if (!bw.f16) continue;
+      const MatView* src[5] = {&bw.wqkv, &bw.wo, &bw.wg, &bw.wu, &bw.wd};
+      const MatView* dst[5] = {&bw.f16->wqkv, &bw.f16->wo, &bw.f16->wg, &bw.f16->wu, &bw.f16->wd};
+      for (int i = 0; i < 5; ++i) {
+        const int64_t words = (int64_t)src[i]->N * src[i]->K / 8;
+        TL_TRY(launch_k(c, stage_f16_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, *src[i],
+                        const_cast<__half*>(reinterpret_cast<const __half*>(dst[i]->bf))));
+      }
+    }
   TL_CUDA(cudaStreamSynchronize(c->stream));
   c->staged_src = nullptr;
   c->loaded = true;

@@ -47,6 +47,11 @@ struct TcParams {
 
 constexpr int TC_SC_MAX = 33;  // scale groups per CTA row
 
+// Weights already in fp16 (see stage_f16_kernel: a prompt pass's staging
+// buffer, or the resident copy of a BF16 model's blocks): the weight tile
+// arrives by TMA in the canonical MMA layout and nothing is converted.
+constexpr int FMT_F16 = 2;
+
 // k-step j of a projection: weight block tc_wblock, activation block
 // tc_xblock.  With split activations a weight block's hi and lo products run
 // back to back (steps 2w and 2w + 1), so its second read comes from L2 and a
@@ -60,7 +65,7 @@ template <int NT, int NMAT, int FMT>
 struct TcCfg {
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = NT * 64 * 2;
-  static constexpr int RAW_BYTES = (FMT == TL_FMT_INT4) ? 128 * 32 : 128 * 128;
+  static constexpr int RAW_BYTES = (FMT == TL_FMT_INT4) ? 128 * 32 : (FMT == FMT_F16 ? 0 : 128 * 128);
   static constexpr int SC_BYTES = (FMT == TL_FMT_INT4) ? NMAT * 128 * TC_SC_MAX * 2 : 0;
   static constexpr int stage_bytes = NMAT * (A_BYTES + RAW_BYTES) + B_BYTES;
   static constexpr int fixed = SC_BYTES + 256 + 1024;
@@ -73,11 +78,11 @@ struct TcCfg {
   static constexpr bool SPLIT_OK = NMAT * NT * 128 * 4 <= STAGES * stage_bytes;
   static_assert(STAGES >= 2, "tile does not fit in shared memory");
   // TMEM is allocated before the programmatic-dependency wait, so a CTA may
-  // allocate while a CTA of the previous kernel on its SM still has to.  The
-  // smallest tile uses ~95 KB of shared memory, so any tile holding more than
-  // 64 columns must leave no room for a second tensor-core CTA on its SM; two
-  // 64-column CTAs fit TMEM's 512 columns together.
-  static_assert(TMEM_COLS <= 64 || SMEM > 133 * 1024, "TMEM could be oversubscribed by co-resident CTAs");
+  // allocate while a CTA of the previous kernel on its SM still has to.  Any
+  // tile holding more than 64 columns must leave no room for a second
+  // tensor-core CTA on its SM (two CTAs above 114 KB exceed the SM's 228 KB);
+  // two 64-column CTAs fit TMEM's 512 columns together.
+  static_assert(TMEM_COLS <= 64 || SMEM > 114 * 1024, "TMEM could be oversubscribed by co-resident CTAs");
 };
 
 // K-major, SWIZZLE_128B canonical layout: 8-row groups 1024 B apart.
@@ -250,11 +255,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < pre; ++i) {
       const uint32_t fb = smem_u32(&full[i]);
-      mbar_add_tx(fb, NMAT * C::RAW_BYTES);
       const int kbw = tc_wblock(p, kb0 + i);
-      const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
-      tma_load_2d(smem_u32(sRaw + (i * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
-      if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (i * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+      if constexpr (FMT == FMT_F16) {  // straight into the MMA's A tiles
+        mbar_add_tx(fb, NMAT * C::A_BYTES);
+        tma_load_2d(smem_u32(sA + (i * NMAT + 0) * C::A_BYTES), &mapW, kbw * 64, m0, fb);
+        if constexpr (NMAT == 2) tma_load_2d(smem_u32(sA + (i * NMAT + 1) * C::A_BYTES), &mapW2, kbw * 64, m0, fb);
+      } else {
+        mbar_add_tx(fb, NMAT * C::RAW_BYTES);
+        const int wx = (FMT == TL_FMT_INT4) ? kbw * 32 : kbw * 64;
+        tma_load_2d(smem_u32(sRaw + (i * NMAT + 0) * C::RAW_BYTES), &mapW, wx, m0, fb);
+        if constexpr (NMAT == 2) tma_load_2d(smem_u32(sRaw + (i * NMAT + 1) * C::RAW_BYTES), &mapW2, wx, m0, fb);
+      }
     }
   }
   pdl_wait();
@@ -282,6 +293,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
       if (elect_one()) {
         if (i < pre) {
           mbar_expect_tx(fb, C::B_BYTES);
+        } else if constexpr (FMT == FMT_F16) {
+          mbar_expect_tx(fb, NMAT * C::A_BYTES + C::B_BYTES);
+          const int kbw = tc_wblock(p, kb);
+          tma_load_2d(smem_u32(sA + (s * NMAT + 0) * C::A_BYTES), &mapW, kbw * 64, m0, fb);
+          if constexpr (NMAT == 2) tma_load_2d(smem_u32(sA + (s * NMAT + 1) * C::A_BYTES), &mapW2, kbw * 64, m0, fb);
         } else {
           mbar_expect_tx(fb, NMAT * C::RAW_BYTES + C::B_BYTES);
           const int kbw = tc_wblock(p, kb);
@@ -305,7 +321,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
     constexpr uint32_t idesc = umma_idesc_f16<NT>();
     for (int i = 0; i < nkb; ++i) {
       const int s = i % STAGES, r = i / STAGES;
-      if (!mbar_wait_warp(smem_u32(&afull[s]), r & 1, abort_flag)) break;
+      if (FMT != FMT_F16 && !mbar_wait_warp(smem_u32(&afull[s]), r & 1, abort_flag)) break;
       if (!mbar_wait_warp(smem_u32(&full[s]), r & 1, abort_flag)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
@@ -341,7 +357,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__
       }
     }
     bool ok = true;
-    for (int i = 0; i < nkb && ok; ++i) {
+    for (int i = 0; i < (FMT == FMT_F16 ? 0 : nkb) && ok; ++i) {  // (fp16 weights: nothing to convert)
       const int s = i % STAGES, r = i / STAGES;
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), r & 1, abort_flag))) { ok = false; break; }
 #pragma unroll

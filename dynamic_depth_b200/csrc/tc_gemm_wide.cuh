@@ -31,10 +31,6 @@
 
 namespace tl {
 
-// Weights already in fp16 (a prompt pass's staging buffer, see stage_f16_kernel):
-// the weight tile arrives by TMA in the canonical layout and nothing is converted.
-constexpr int FMT_F16 = 2;
-
 template <int NMAT, int FMT>
 struct TcWideCfg {
   static constexpr int NT = 256 / NMAT;
