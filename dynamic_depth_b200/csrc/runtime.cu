@@ -71,10 +71,10 @@ static bool cfg_valid(const tl_config* c) {
 // at 1.5e-3 with fp16 activations.
 constexpr int kSplitDepth = 48;
 
-// Blocks whose matrices are BF16 (pre blocks first, then the loop body's layers).
-static int n_f16_blocks(const tl_config* c) {
-  return (c->fmt_pre == TL_FMT_BF16 ? c->n_pre : 0) + (c->fmt_loop == TL_FMT_BF16 ? c->n_loop_layers : 0);
-}
+// Blocks with a resident fp16 copy of their matrices: all of them (pre blocks
+// first, then the loop body's layers).  The tensor-core projections read the
+// copy; the few-row GEMV reads the INT4 or BF16 weights themselves.
+static int n_f16_blocks(const tl_config* c) { return c->n_pre + c->n_loop_layers; }
 static int act_split_on(const tl_config* c) {
   if (c->act_split != 0) return c->act_split == 1 ? 1 : 0;
   return c->n_pre + c->L_max * c->n_loop_layers > kSplitDepth ? 1 : 0;
@@ -210,7 +210,7 @@ struct Layout {
   std::vector<size_t> mat_off;  // per matrix
   size_t gains, rope, page_table, kv, lanes, h, h_in, hrows, rows[6], act_a, act_qkv, act_q, act_o, act_u,
       act_a16, act_o16, act_u16, attn_part, attn_counters, part_val, part_idx, tok_stage, L_stage,
-      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec, lane_shared, casc, wstage,
+      mask_stage, pf_n, pf_tiles, pf_info, probe_logits, margin_lane, spec, lane_shared, casc,
       f16blk, out_tok, out_dep, status, counters, body_kernels, alive, b_act_a, b_act_qkv, b_act_q, b_act_o, b_act_u,
       b_act_a16, b_act_o16, b_act_u16, b_attn_part, b_attn_counters, b_part_val, b_part_idx, b_casc, total;
 };
@@ -268,9 +268,10 @@ static Layout make_layout(const tl_config* c) {
   L.lane_shared = take(lanes * 4);
   L.casc = take(lanes * c->n_heads * (hd + 2) * 4);
   // prompt batches wide enough for the persistent GEMM: one block's five matrices in fp16
-  L.wstage = take(L.max_prefill >= 512 ? (size_t)(4 * d * d + 3 * d * F) * 2 : 0);
-  // BF16 blocks: a resident fp16 copy of every matrix (the same bytes per weight), so the tensor-core
-  // projections load weight tiles straight into the MMA layout instead of converting them every step
+  // a resident fp16 copy of every block matrix (BF16: the same bytes per weight; INT4: four times, 100 MB
+  // at the 407M-class shape), so the tensor-core projections load weight tiles straight into the MMA layout
+  // instead of converting them every step (64 lanes: 33.8k -> 36.0k tokens/s; 1.4B-class BF16, 256 lanes:
+  // 5.9k -> 8.6k)
   L.f16blk = take((size_t)n_f16_blocks(c) * (4 * d * d + 3 * d * F) * 2);
   L.out_tok = take(lanes * (size_t)c->max_seq * 4);
   L.out_dep = take(lanes * (size_t)c->max_seq * 4);
@@ -300,7 +301,7 @@ struct BlockW {
   MatView wqkv, wo, wg, wu, wd;
   const float *g1, *g2;
   CUtensorMap mqkv, mo, mg, mu, md;  // TMA maps of the raw weight tiles
-  const BlockW* f16 = nullptr;       // BF16 blocks: the resident fp16 copy the tensor-core projections read
+  const BlockW* f16 = nullptr;       // the resident fp16 copy the tensor-core projections read
 };
 
 // Row-wise scratch of one stream of projection / attention / head kernels.  A
@@ -354,10 +355,7 @@ struct tl_ctx {
   std::vector<int32_t> h_lane_shared, h_lane_donor;
   bool cascade_enabled = true;  // tl_set_cascade
   bool cascade_active = false;  // enabled, and the lanes that share map one donor's prefix of one length
-  __half* wstage = nullptr;     // fp16 staging copy of one block's matrices for wide prompt batches
-  BlockW sblock{};              // views and TMA maps of that copy
-  std::vector<BlockW> blk16;    // resident fp16 copies of BF16 blocks (see BlockW::f16)
-  const BlockW* staged_src = nullptr;  // the block whose matrices the copy holds
+  std::vector<BlockW> blk16;    // resident fp16 copies of the blocks (see BlockW::f16)
   int32_t *tok_stage, *L_stage, *out_tok, *out_dep, *status, *alive;
   int32_t* pf_n;     // prompt batches: row count of each stage (stage l = loop iteration l)
   int2* pf_tiles;    // prompt batches: attention tiles (first row, rows)
@@ -910,21 +908,7 @@ int run_block(tl_ctx* c, const Rows& rows, int max_rows, float* hbuf, const int3
   if (prompt) path = max_rows > kGemvMaxRows ? PATH_TC : PATH_GEMV;
   const int d = c->cfg.d, F = c->cfg.ffn;
   const bool defer = pend && prompt && max_rows >= kWideRows;
-  // prompt batches on the persistent GEMM read an fp16 copy of the block's matrices, made once per pass and
-  // block (the loop block once for all its iterations), instead of dequantising every tile again
-  const bool staged = prompt && max_rows >= kWideRows && c->wstage && !w.f16;
-  if (staged && c->staged_src != &w) {
-    const MatView* src[5] = {&w.wqkv, &w.wo, &w.wg, &w.wu, &w.wd};
-    const MatView* dst[5] = {&c->sblock.wqkv, &c->sblock.wo, &c->sblock.wg, &c->sblock.wu, &c->sblock.wd};
-    for (int i = 0; i < 5; ++i) {
-      const int64_t words = (int64_t)src[i]->N * src[i]->K / 8;
-      TL_TRY(launch_k(c, stage_f16_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, *src[i],
-                      const_cast<__half*>(reinterpret_cast<const __half*>(dst[i]->bf))));
-    }
-    c->staged_src = &w;
-  }
-  const BlockW& pw = staged ? c->sblock : w;  // the projections' matrices and maps
-  // a BF16 block's tensor-core variants read its resident fp16 copy
+  const BlockW& pw = w;  // the GEMV's matrices; the tensor-core variants read the block's resident fp16 copy
   const BlockW* tb = w.f16;
   const TcTwin t_qkv{tb ? &tb->wqkv : nullptr, tb ? &tb->mqkv : nullptr, nullptr, nullptr};
   const TcTwin t_o{tb ? &tb->wo : nullptr, tb ? &tb->mo : nullptr, nullptr, nullptr};
@@ -1176,14 +1160,6 @@ int encode_all_maps(tl_ctx* c) {
       TL_TRY(encode_2d(mp5[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv5[i]->bf, (uint64_t)mv5[i]->K, (uint64_t)mv5[i]->N,
                        (uint64_t)mv5[i]->K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
   }
-  if (c->wstage) {  // the staging copy: fp16 tiles of 128 rows x 64 K, in the MMA's swizzled layout
-    BlockW& b = c->sblock;
-    const MatView* mv5[5] = {&b.wqkv, &b.wo, &b.wg, &b.wu, &b.wd};
-    CUtensorMap* mp5[5] = {&b.mqkv, &b.mo, &b.mg, &b.mu, &b.md};
-    for (int i = 0; i < 5; ++i)
-      TL_TRY(encode_2d(mp5[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv5[i]->bf, (uint64_t)mv5[i]->K, (uint64_t)mv5[i]->N,
-                       (uint64_t)mv5[i]->K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
-  }
   {  // KV pool as rows of hd fp16: a page is [K: H x P rows][V: H x P rows]
     const uint64_t pool_rows = (uint64_t)c->lay.n_pages * 2 * c->cfg.n_heads * c->cfg.kv_page_tokens;
     const uint32_t cols = c->hd > 64 ? 64 : (uint32_t)c->hd;
@@ -1305,7 +1281,7 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
               gains + (size_t)(2 * b) * cfg->d, gains + (size_t)(2 * b + 1) * cfg->d};
     (b < cfg->n_pre ? c->pre : c->loop).push_back(bw);
   }
-  {  // resident fp16 copies of the BF16 blocks, in block order (filled by tl_load_weights)
+  {  // resident fp16 copies of the blocks, in block order (filled by tl_load_weights)
     const int64_t d = cfg->d, F = cfg->ffn;
     const int64_t off[5] = {0, 3 * d * d, 4 * d * d, 4 * d * d + F * d, 4 * d * d + 2 * F * d};
     const int64_t NN[5] = {3 * d, d, F, F, d}, KK[5] = {d, d, d, d, F};
@@ -1313,7 +1289,6 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
     __half* base = (__half*)(w + lay.f16blk);
     for (int b = 0; b < nb; ++b) {
       BlockW& src = b < cfg->n_pre ? c->pre[b] : c->loop[b - cfg->n_pre];
-      if (src.wqkv.fmt != TL_FMT_BF16) continue;
       BlockW cp = src;
       MatView* mv5[5] = {&cp.wqkv, &cp.wo, &cp.wg, &cp.wu, &cp.wd};
       for (int i = 0; i < 5; ++i) {
@@ -1375,22 +1350,6 @@ extern "C" int tl_create(const tl_config* cfg, void* dev_ws, size_t bytes, void*
   c->spec = (int32_t*)(w + lay.spec);
   c->lane_shared = (int32_t*)(w + lay.lane_shared);
   c->sc->casc = (float*)(w + lay.casc);
-  if (lay.max_prefill >= 512) {
-    c->wstage = (__half*)(w + lay.wstage);
-    const int64_t d = cfg->d, F = cfg->ffn;
-    const int64_t off[5] = {0, 3 * d * d, 4 * d * d, 4 * d * d + F * d, 4 * d * d + 2 * F * d};
-    const int64_t NN[5] = {3 * d, d, F, F, d}, KK[5] = {d, d, d, d, F};
-    MatView* mv5[5] = {&c->sblock.wqkv, &c->sblock.wo, &c->sblock.wg, &c->sblock.wu, &c->sblock.wd};
-    for (int i = 0; i < 5; ++i) {
-      MatView m{};
-      m.fmt = FMT_F16;
-      m.N = (int)NN[i];
-      m.K = (int)KK[i];
-      m.group = cfg->group;
-      m.bf = reinterpret_cast<const uint16_t*>(c->wstage + off[i]);
-      *mv5[i] = m;
-    }
-  }
   c->mask_stage = (uint8_t*)(w + lay.mask_stage);
   c->out_tok = (int32_t*)(w + lay.out_tok);
   c->out_dep = (int32_t*)(w + lay.out_dep);
@@ -1544,7 +1503,7 @@ extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
     const int64_t words = (int64_t)m->N * m->K / 8;
     TL_TRY(launch_k(c, int4_repack_kernel, dim3((unsigned)((words + 255) / 256)), dim3(256), 0, (uint32_t*)m->q, words));
   }
-  // the resident fp16 copies of the BF16 blocks (the conversion the tensor-core kernels applied per tile)
+  // the blocks' resident fp16 copies (the conversion the tensor-core kernels applied per tile)
   for (auto* v : {&c->pre, &c->loop})
     for (const BlockW& bw : *v) {
       if (!bw.f16) continue;
@@ -1557,7 +1516,6 @@ extern "C" int tl_load_weights(tl_ctx* c, const void* blob, size_t bytes) {
       }
     }
   TL_CUDA(cudaStreamSynchronize(c->stream));
-  c->staged_src = nullptr;
   c->loaded = true;
   return TL_OK;
 }

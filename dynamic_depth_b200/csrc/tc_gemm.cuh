@@ -47,9 +47,9 @@ struct TcParams {
 
 constexpr int TC_SC_MAX = 33;  // scale groups per CTA row
 
-// Weights already in fp16 (see stage_f16_kernel: a prompt pass's staging
-// buffer, or the resident copy of a BF16 model's blocks): the weight tile
-// arrives by TMA in the canonical MMA layout and nothing is converted.
+// Weights already in fp16 (a block's resident copy, see stage_f16_kernel): the
+// weight tile arrives by TMA in the canonical MMA layout and nothing is
+// converted.
 constexpr int FMT_F16 = 2;
 
 // k-step j of a projection: weight block tc_wblock, activation block

@@ -317,13 +317,13 @@ tc_gemm_wide_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_const
   }
 }
 
-// A prompt pass's staging copy of one weight matrix: out [N][K] fp16 with
-// exactly the values the converting kernels above build in shared memory
+// The resident fp16 copy of one block matrix (made at weight load): out [N][K]
+// fp16 with exactly the values the converting kernels build in shared memory
 // (INT4: (u - 8) exact, times the fp16 group scale, rounded once; BF16: the
 // same value in fp16).  One thread per 8 consecutive elements.
 __global__ void stage_f16_kernel(MatView W, __half* __restrict__ out) {
   pdl_launch_dependents();
-  pdl_wait();  // the previous pass's GEMMs may still read this buffer
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 8-element word
   const int64_t words = (int64_t)W.N * W.K / 8;
   if (i >= words) return;
