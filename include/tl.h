@@ -358,9 +358,11 @@ int tl_speculate(tl_ctx* ctx, int32_t lane, int32_t n_new, int32_t L_draft, int3
  * when their pre blocks are done (needs CUDA graphs, else mode 2 runs).
  * mode 0 (default) chooses per decode call: mode 3 for 32+ lanes with mean
  * requested L of 6 or more, mode 1 otherwise.  Results per lane do not
- * depend on it beyond the rounding differences of batch width (a row's
- * projections take fp32 activations in a step of at most 8 rows, fp16 in a
- * wider one); in mode 3 the widths depend on timing.  See
+ * depend on it beyond the rounding differences of batch width: in a decode
+ * of more than 8 lanes the loop steps always run on the tensor cores (fp16
+ * activation copies), while a boundary stage of at most 8 rows takes fp32
+ * activations and a wider one fp16, and attention's context split follows
+ * the step's row count; in mode 3 the widths depend on timing.  See
  * tl_stats.tick_layout.  TL_EINVAL for other modes. */
 int tl_set_tick_overlap(tl_ctx* ctx, int32_t mode);
 
