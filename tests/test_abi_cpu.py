@@ -86,7 +86,8 @@ def test_workspace_grows_with_capacity_and_kv_formula():
                                          ("ffn", 544),  # a multiple of 32 but not of 64
                                          ("ffn", 2048),  # 64 scale groups of 32 across ffn
                                          ("kv_page_tokens", 16), ("max_lanes", 0), ("max_lanes", 2048),
-                                         ("L_max", 0), ("fmt_loop", 7), ("max_prefill_tokens", -1)])
+                                         ("L_max", 0), ("fmt_loop", 7), ("max_prefill_tokens", -1),
+                                         ("act_split", 3), ("act_split", -1)])
 def test_invalid_configs_rejected(field, value):
     cfg = T.config_from_shape(S.TINY, max_lanes=2, max_seq=64, L_max=4)
     setattr(cfg, field, value)
@@ -122,3 +123,41 @@ def test_prompt_rows_may_exceed_one_sequence():
     cfg = T.config_from_shape(S.TINY, max_lanes=8, max_seq=64, L_max=4, max_prefill_tokens=512)
     small = T.config_from_shape(S.TINY, max_lanes=8, max_seq=64, L_max=4)
     assert T.workspace_bytes(cfg) > T.workspace_bytes(small)
+
+
+def _ws(sh, **kw):
+    return T.workspace_bytes(T.config_from_shape(sh, **kw))
+
+
+def test_split_activations_double_the_fp16_activation_copies():
+    # act_split = 1 stores every fp16 activation copy as [hi | lo] rows: three copies (norm output,
+    # attention output: d wide; SwiGLU output: ffn wide) for the prompt rows and again for the boundary
+    # stage's scratch (max_lanes rows), each twice as wide
+    sh = S.M407
+    cap = dict(max_lanes=4, max_seq=128, L_max=8, max_prefill_tokens=512)
+    single = _ws(sh, act_split=2, **cap)
+    split = _ws(sh, act_split=1, **cap)
+    rows, lanes = 512, 4
+    extra = (rows + lanes) * (2 * sh.d + sh.ffn) * 2
+    assert extra <= split - single <= extra + 6 * 256  # up to one alignment pad per region
+
+
+def test_split_activations_automatic_past_48_blocks():
+    # automatic: split when n_pre + L_max * n_loop_layers > 48 (the 407M-class model at L_max = 32 crosses
+    # 34 blocks, the 1.4B-class layout at L_max = 4 crosses 96)
+    m407 = dict(max_lanes=2, max_seq=64, max_prefill_tokens=64)
+    assert _ws(S.M407, L_max=32, act_split=0, **m407) == _ws(S.M407, L_max=32, act_split=2, **m407)
+    assert _ws(S.M407, L_max=47, act_split=0, **m407) == _ws(S.M407, L_max=47, act_split=1, **m407)
+    mini = dict(max_lanes=2, max_seq=64, max_prefill_tokens=64)
+    assert _ws(S.M1B4_MINI, L_max=16, act_split=0, **mini) == _ws(S.M1B4_MINI, L_max=16, act_split=2, **mini)
+    assert _ws(S.M1B4_MINI, L_max=17, act_split=0, **mini) == _ws(S.M1B4_MINI, L_max=17, act_split=1, **mini)
+
+
+def test_workspace_holds_a_resident_fp16_copy_of_every_block():
+    # every block's five matrices in fp16: (3d*d + d*d + 2*ffn*d + d*ffn) halves per block
+    sh = S.M407
+    cfg = T.config_from_shape(sh, max_lanes=1, max_seq=64, L_max=2)
+    ws = T.workspace_bytes(cfg)
+    weights = T.weights_bytes(cfg)
+    copies = (sh.n_pre + sh.n_loop_layers) * (4 * sh.d * sh.d + 3 * sh.d * sh.ffn) * 2
+    assert ws > weights + copies
