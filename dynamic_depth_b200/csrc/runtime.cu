@@ -1994,7 +1994,7 @@ static int capture_body(tl_ctx* c, cudaGraph_t body, int64_t* n_kernels, F fn) {
 // parameters.
 //   plan -+-> SWITCH { norm, head, argmax + token + embedding: GEMV | tensor cores }
 //         |     -> SWITCH { entering lanes: pre blocks + first loop iteration: GEMV | TC }  (boundary scratch)
-//         +-> loop body + exit rule of the other lanes: plain nodes (both variants) for a body of
+//         +-> loop body + exit rule of the other lanes: plain nodes (loop_path) for a body of
 //             <= 2 layers, else SWITCH { GEMV | tensor cores }                            (main scratch)
 //   (the two branches join at the end of the tick: "Depth-adaptive Inference of Looped Language Models via
 //   Continuous Depth Batching", boundary stages queued apart from loop steps, overlapped with them)
@@ -2045,10 +2045,9 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
   c->prio = 0;
   // loop rows -> loop body.  The bodies of a graph's conditional nodes were measured to start one after
   // another (each once the previous body's last kernel was launched), which kept this branch waiting for
-  // the boundary stage's head.  So a short body runs as plain kernel nodes, which start at once, with both
-  // projection variants captured (the one that does not apply to the device-side row count returns at
-  // once); a long body (the 24-layer one) keeps its conditional node, where doubling every projection's
-  // launches measured slower (7.0k against 7.9k tokens/s on 256 lanes).  Plain nodes for the boundary
+  // the boundary stage's head.  So a short body runs as plain kernel nodes, which start at once, on the
+  // projection path loop_path chooses; a long body (the 24-layer one) keeps its conditional node, where
+  // doubling every projection's launches measured slower (7.0k against 7.9k tokens/s on 256 lanes).  Plain nodes for the boundary
   // stage too measured slower again (2.0k against 1.8k tokens/s for one lane at L = 8).
   c->tick_loop_kernels = 0;
   kcount[4] = kcount[5] = 0;
