@@ -389,6 +389,7 @@ def run_ours(args, rank, world, local_rank):
         "depth_histogram": {int(k): int(v) for k, v in zip(*np.unique(depths[:, 1:], return_counts=True))},
         "ticks_per_step": units["ticks"],
         "loop_steps_per_step": int(st1["loop_steps"] - st0["loop_steps"]) // args.steps,
+        "boundary_stages_per_step": int(st1["boundary_stages"] - st0["boundary_stages"]) // args.steps,
         "tick_layout": TICK_LAYOUTS.get(int(st1["tick_layout"]), str(st1["tick_layout"])),
         "early_exit_tokens": exited,
         "early_exit_fired": exited > 0,

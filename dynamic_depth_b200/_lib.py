@@ -33,6 +33,7 @@ class TlStats(C.Structure):
         ("loop_steps", C.c_int64), ("lane_iterations", C.c_int64), ("tokens_emitted", C.c_int64),
         ("prefill_tokens", C.c_int64), ("kernel_launches", C.c_int64), ("device_status", C.c_int32),
         ("kv_pages_used", C.c_int32), ("entry_in_boundary", C.c_int32), ("tick_layout", C.c_int32),
+        ("boundary_stages", C.c_int64),
     ]
 
 

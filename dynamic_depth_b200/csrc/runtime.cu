@@ -402,7 +402,7 @@ struct tl_ctx {
   std::vector<int32_t> lane_L;        // prefill depth per lane (0 = empty)
   int32_t* pinned_alive = nullptr;    // ring of (alive lanes, loop rows)
   cudaEvent_t alive_ev[4];
-  int64_t steps = 0, prefill_tokens = 0, launches = 0;
+  int64_t steps = 0, prefill_tokens = 0, launches = 0, bnd_stages = 0;
   // profiling ring (tl_profile_begin / tl_profile_end)
   int prof_mask = 0;
   std::vector<std::array<cudaEvent_t, 2>> prof_ev;
@@ -2236,6 +2236,7 @@ static int decode_async(tl_ctx* c, int n_lanes, int n_new) {
     TL_CUDA(cudaGraphLaunch(c->bnd_exec, c->bstream));
     TL_CUDA(cudaEventRecord(c->b_ev[nb % kBRing], c->bstream));
     ++nb;
+    c->bnd_stages++;
     c->launches += c->bnd_launches;
     return TL_OK;
   };
@@ -2360,6 +2361,7 @@ extern "C" int tl_stats_get(tl_ctx* c, tl_stats* out) {
   out->kv_pages_used = c->lay.n_pages - (int32_t)c->free_pages.size();
   out->entry_in_boundary = c->entry_iter;
   out->tick_layout = c->layout;
+  out->boundary_stages = c->bnd_stages;
   return TL_OK;
 }
 

@@ -118,6 +118,9 @@ typedef struct tl_stats {
                                     next tick (0); see tl_set_tick_overlap      */
     int32_t tick_layout;         /* the layout the last decode ran: 1, 2 or 3 (see
                                     tl_set_tick_overlap)                         */
+    int64_t boundary_stages;     /* boundary stages launched apart from the loop
+                                    steps (layout 3; in layouts 1 and 2 every tick
+                                    holds one)                                    */
 } tl_stats;
 
 /* ---------------------------------------------------------------- sizes -- */

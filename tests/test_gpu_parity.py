@@ -244,9 +244,11 @@ def test_tiny_async_stages_early_exit_and_repeat(exit_rule):
     else:
         ref = [D.generate_lane(W, P[i], Ls[i], 9) for i in range(24)]
     for _ in range(2):
+        b0 = m.stats()["boundary_stages"]
         tok, dep = m.generate(P, Ls, 9)
         st = status_clean(m)
         assert st["tick_layout"] == 3
+        assert st["boundary_stages"] > b0
         for i in range(24):
             assert dep[i].tolist() == ref[i].depths.tolist(), i
             _check_tokens(ref[i].tokens, ref[i].logits, tok[i])
