@@ -413,7 +413,7 @@ struct tl_ctx {
 
 static constexpr int kAliveRing = 4;
 static constexpr int kBRing = 4;  // boundary stages queued at once, at most (layout 3)
-static constexpr int kLoopStepsPerGraph = 4;  // layout 3
+static constexpr int kLoopStepsPerGraph = 6;  // layout 3
 static constexpr int kProfRing = 4096;
 
 namespace {
@@ -2076,9 +2076,12 @@ static int capture_tick(tl_ctx* c, int n_lanes, int n_new, int32_t* tok_out, int
 // orders the hand-offs, so a lane's own steps keep their order while the two
 // streams run side by side at their own cadence.
 // kLoopStepsPerGraph loop steps per graph launch (each plans its own rows):
-// fewer graph boundaries, each of which cost ~10 us between two steps (64
-// lanes: 31.2k tokens/s with 2 steps per graph, 32.0-32.5k with 4, 31.5k
-// with 8, whose empty steps at the end of a decode cost more than they save).
+// fewer graph boundaries, each of which cost ~10 us between two steps.  A
+// boundary stage is launched (at most) once per graph launch, so the count
+// also sets the boundary stages' cadence.  Measured at 64 lanes with the
+// current kernels: 41.4-41.8k tokens/s with 4 steps per graph (2,556 steps
+// per pass), 45.7-46.1k with 6 (2,310), 41.1k with 8 (3,072: empty steps at
+// the end of a decode cost more than they save).
 static int capture_loop_step(tl_ctx* c, int n_lanes, int32_t* kcount) {
   const bool plain_loop = c->cfg.n_loop_layers <= 2;  // as in the tick graph
   const int64_t l0 = c->launches;
